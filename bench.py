@@ -1,0 +1,429 @@
+"""Benchmark of one POEM prefill attention layer (score -> select -> block-sparse
+attention) on B200.
+
+Default workload: the Llama-3.1-8B-shaped layer at 128K tokens (32 query heads,
+8 KV heads, head dim 128, 128x128 blocks, RoPE base 500000, heavy-block
+synthetic Q/K/V from seed 0, tau = 0.05).  One step = poem_score + poem_select
++ bsa_fwd over that layer with the inputs resident in HBM (inputs are larger
+than L2, so no flush is needed between steps).  Prints one JSON line.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+With N > 1 (torchrun, one rank per GPU) every rank runs an independent replica
+of the layer (the path needs no exchange step); the reported ms/layer is the
+whole job's: max-over-ranks time / (N * K).
+
+--impl reference times the fp64 CPU oracle (test infrastructure; the reference
+arm of this benchmark) on a bounded sample of the same layer's (head, tile)
+units on the host cores and extrapolates to ms/layer by the work per unit.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import poem_synth  # noqa: E402
+
+METRIC = "128K-token prefill attention ms/layer; retained-block TFLOP/s vs BF16 tensor peak"
+
+WORKLOADS = {
+    # name: (n_tokens, Hq, Hkv, d, block, rope_base, tau)
+    "llama3.1-8b-layer-128k": (131072, 32, 8, 128, 128, 500000.0, 0.05),
+    "llama3.1-8b-layer-32k": (32768, 32, 8, 128, 128, 500000.0, 0.05),
+    "qwen3-14b-layer-64k": (65536, 40, 8, 128, 128, 1000000.0, 0.05),
+}
+# Roofline denominators measured on this machine's B200s (copied from the driver's
+# measurement; MEASURED_PEAKS.json, when present, takes precedence).
+FALLBACK_PEAKS = {"bf16_tflops": 1667.9, "bf16_tflops_sustained": 1378.8, "hbm_gbs": 6452.5}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured (MEASURED_PEAKS.json)"
+    return dict(FALLBACK_PEAKS), "measured (copy in BASELINE.md)"
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling during the timed region."""
+
+    FIELDS = "index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active," \
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown," \
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap"
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": float(max(smax)), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def retained_flops(row_ptr: np.ndarray, col_idx: np.ndarray, n_tiles: int, d: int, B: int) -> float:
+    """4 d (kept query-key pairs): full blocks B^2 pairs, the diagonal block B(B+1)/2."""
+    rows = len(row_ptr) - 1
+    counts = np.diff(row_ptr).astype(np.int64)
+    tiles = np.arange(rows) % n_tiles
+    # diagonal present? (lists are ascending: last entry == tile)
+    last = np.where(counts > 0, col_idx[np.maximum(row_ptr[1:] - 1, 0)], -1)
+    diag = (last == tiles).astype(np.int64)
+    pairs = (counts - diag) * B * B + diag * (B * (B + 1) // 2)
+    return float(4 * d * pairs.sum())
+
+
+def dense_flops(n: int, hq: int, d: int) -> float:
+    return float(2 * d * hq * n * (n + 1))
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    return world, rank, local
+
+
+def run_ours(args):
+    import block_sparse_attention_poem_b200 as poem
+
+    world, rank, local = dist_setup()
+    dev = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(dev)
+    n, hq, hkv, d, B, base, tau = WORKLOADS[args.workload]
+    T = n // B
+    x = poem_synth.heavy_block_layer(n, hq, hkv, d, block=B, rope_base=base, seed=args.seed)
+    q, k, v = x["q"].to(dev), x["k"].to(dev), x["v"].to(dev)
+    layer = poem.alloc_layer(q, k, block=B)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        if ev:
+            ev[0].record(stream)
+        poem.poem_score(q, k, v, layer.I_hat, layer.m_hat, layer.ws_score, shape=layer.shape)
+        if ev:
+            ev[1].record(stream)
+        poem.poem_select(layer.shape, layer.I_hat, layer.m_hat, tau, layer.row_ptr, layer.col_idx, layer.ws_select,
+                         order=layer.order)
+        if ev:
+            ev[2].record(stream)
+        poem.bsa_fwd(q, k, v, layer.row_ptr, layer.col_idx, layer.o, layer.ws_fwd, order=layer.order,
+                     shape=layer.shape)
+        if ev:
+            ev[3].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    for ws in (layer.ws_score, layer.ws_select, layer.ws_fwd):
+        poem.poem_check(ws)
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    clocks = ClockSampler(dev.index if dev.index is not None else 0)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for s in range(args.steps):
+        step(evs[s])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    if world > 1:
+        torch.distributed.barrier()
+    total_ms = t_start.elapsed_time(t_end)
+    score_ms = float(np.mean([e[0].elapsed_time(e[1]) for e in evs]))
+    select_ms = float(np.mean([e[1].elapsed_time(e[2]) for e in evs]))
+    fwd_ms = float(np.mean([e[2].elapsed_time(e[3]) for e in evs]))
+    if world > 1:
+        import torch.distributed as dist
+
+        tt = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        total_ms = float(tt.item())
+    ms_per_step = total_ms / args.steps
+    ms_per_layer = total_ms / (args.steps * world)
+
+    for ws in (layer.ws_score, layer.ws_select, layer.ws_fwd):
+        poem.poem_check(ws)
+    rp = layer.row_ptr.cpu().numpy()
+    ci = layer.col_idx[: int(rp[-1])].cpu().numpy()
+    kept = int(rp[-1])
+    visible = hq * T * (T + 1) // 2
+    rflops = retained_flops(rp, ci, T, d, B)
+    dflops = dense_flops(n, hq, d)
+    peaks, peak_src = load_peaks()
+    fwd_tflops = rflops / (fwd_ms * 1e-3) / 1e12
+
+    # end-to-end through the public API with host buffers: H2D of Q/K/V from pinned
+    # memory, the three calls, D2H of O, every step.
+    e2e = None
+    if not args.no_e2e:
+        hq_h = x["q"].pin_memory()
+        hk_h = x["k"].pin_memory()
+        hv_h = x["v"].pin_memory()
+        ho = torch.empty(q.shape, dtype=torch.bfloat16).pin_memory()
+        torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            q.copy_(hq_h, non_blocking=True)
+            k.copy_(hk_h, non_blocking=True)
+            v.copy_(hv_h, non_blocking=True)
+            step()
+            ho.copy_(layer.o, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = e0.elapsed_time(e1)
+        if world > 1:
+            import torch.distributed as dist
+
+            tt = torch.tensor([e2e_ms], device=dev)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            e2e_ms = float(tt.item())
+        e2e = {"value": e2e_ms / (args.e2e_steps * world), "unit": "ms/layer",
+               "h2d_bytes_per_step": int(hq_h.numel() * 2 + hk_h.numel() * 2 + hv_h.numel() * 2),
+               "d2h_bytes_per_step": int(ho.numel() * 2)}
+
+    extra = {}
+    if not args.no_quality and rank == 0:
+        extra = quality_report(poem, q, k, v, layer, tau, n, hq, T, B, dev)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(x, n, hq, hkv, d, B, tau, args.cpu_budget_s)
+
+    launches_per_step = 2 + 3 + 1 + 1  # score(2) + select(3 + order) + bsa_fwd
+    line = {
+        "metric": METRIC,
+        "value": round(ms_per_layer, 4),
+        "unit": "ms/layer",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": False,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded heavy-block generator; no model weights or datasets)",
+        "config": {"workload": args.workload, "n_tokens": n, "n_q_heads": hq, "n_kv_heads": hkv, "head_dim": d,
+                   "block": B, "n_sample": 16, "tau": tau, "seed": args.seed,
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": "inputs larger than L2 (no flush needed)"},
+        "breakdown_ms": {"poem_score": round(score_ms, 4), "poem_select": round(select_ms, 4),
+                         "bsa_fwd": round(fwd_ms, 4)},
+        "density": round(kept / visible, 5),
+        "dense_equiv_tflops": round(dflops / (ms_per_step * 1e-3) / 1e12, 2),
+        "retained_tflops": round(rflops / (ms_per_step * 1e-3) / 1e12, 2),
+        "score_select_over_fwd": round((score_ms + select_ms) / fwd_ms, 4),
+        "roofline": {"bound": "tensor", "kernel": "bsa_fwd", "achieved": round(fwd_tflops, 2),
+                     "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                     "frac": round(fwd_tflops / peaks["bf16_tflops_sustained"], 4),
+                     "frac_of_burst_peak": round(fwd_tflops / peaks["bf16_tflops"], 4),
+                     "peak_source": peak_src + ", sustained bf16 (kernel timed inside a long step)",
+                     "algorithmic_flops_per_launch": rflops, "traffic": None},
+        "clocks": clk,
+        "e2e": e2e,
+        "gpu_launches": launches_per_step * args.steps,
+        "cpu_baseline": cpu,
+    }
+    line.update(extra)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+def quality_report(poem, q, k, v, layer, tau, n, hq, T, B, dev):
+    """Output error of the POEM lists and of mass-only lists at the same budget,
+    both against dense attention (bsa_fwd over every causal block)."""
+    rp_all, ci_all = poem_synth.random_block_lists(1, T, 1.0, seed=0)
+    counts = np.diff(rp_all)
+    rp_dense = np.concatenate([[0], np.cumsum(np.tile(counts, hq))]).astype(np.int32)
+    ci_dense = np.tile(ci_all, hq).astype(np.int32)
+    rpd = torch.from_numpy(rp_dense).to(dev)
+    cid = torch.from_numpy(ci_dense).to(dev)
+    o_dense = torch.empty_like(q)
+    poem.bsa_fwd(q, k, v, rpd, cid, o_dense, layer.ws_fwd, shape=layer.shape)
+    # mass-only at matched per-row budget
+    rp_m = torch.empty_like(layer.row_ptr)
+    ci_m = torch.empty_like(layer.col_idx)
+    poem.poem_select_mass_only(layer.shape, layer.m_hat, layer.row_ptr, rp_m, ci_m, layer.ws_select)
+    o_mass = torch.empty_like(q)
+    poem.bsa_fwd(q, k, v, rp_m, ci_m, o_mass, layer.ws_fwd, shape=layer.shape)
+    torch.cuda.synchronize()
+    poem.poem_check(layer.ws_fwd)
+    poem.poem_check(layer.ws_select)
+
+    def err(o):
+        diff = (o.float() - o_dense.float())
+        return {"max_abs": float(diff.abs().max()), "mean_abs": float(diff.abs().mean()),
+                "rel_fro": float(diff.norm() / o_dense.float().norm()),
+                "max_row_l2": float(diff.norm(dim=-1).max())}
+
+    return {"err_vs_dense": {"poem": err(layer.o), "mass_only_same_budget": err(o_mass)}}
+
+
+def cpu_baseline(x, n, hq, hkv, d, B, tau, budget_s):
+    """Oracle (fp64, host cores) on a bounded sample of (head, tile) units, scaled to
+    a whole layer by work per unit (score ~ i+1 blocks, masked attention ~ kept
+    blocks; selection is negligible)."""
+    import oracle
+
+    oracle.build()
+    T = n // B
+    prob = oracle.Problem(q=poem_synth.bf16_bits(x["q"]), k=poem_synth.bf16_bits(x["k"]),
+                          v=poem_synth.bf16_bits(x["v"]), block=B, n_sample=16)
+    # sample: tiles spread over the causal range, growing until the budget is used
+    units = []
+    per_unit = []
+    t_total = 0.0
+    cand_tiles = [max(0, int(T * f) - 1) for f in (1 / 64, 1 / 16, 1 / 8, 1 / 4)]
+    h = 0
+    for i in cand_tiles:
+        if t_total > budget_s:
+            break
+        t0 = time.perf_counter()
+        Ih, mh = prob.score_units([(h, i)])
+        off = oracle.tri_offset(T, h, i)
+        keep, _ = oracle.select_row(i, Ih[off:off + i + 1], mh[off:off + i + 1], tau)
+        rp = np.zeros(hq * T + 1, dtype=np.int32)
+        r = h * T + i
+        rp[r + 1:] = len(keep)
+        ci = np.zeros(hq * T, dtype=np.int32)
+        ci[: len(keep)] = keep
+        rp2 = rp.copy()
+        rp2[: r + 1] = 0
+        prob.masked_units([(h, i)], rp2, np.asarray(keep, dtype=np.int32))
+        dt = time.perf_counter() - t0
+        t_total += dt
+        units.append((h, i))
+        per_unit.append(dt / (i + 1))
+        h = (h + 1) % hq
+    rate = float(np.mean(per_unit))  # seconds per visible block of a unit
+    total_blocks = hq * T * (T + 1) / 2
+    est_ms = rate * total_blocks * 1e3
+    return {"value": round(est_ms, 1), "unit": "ms/layer", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{len(units)} (head, tile) units at tiles {[u[1] for u in units]} (score + select + masked "
+                      f"attention), {t_total:.1f} s, scaled by visible blocks per unit to the whole layer",
+            "extrapolated": True}
+
+
+def run_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    n, hq, hkv, d, B, base, tau = WORKLOADS[args.workload]
+    x = poem_synth.heavy_block_layer(n, hq, hkv, d, block=B, rope_base=base, seed=args.seed)
+    budget = max(2.0, args.ref_step_budget_s)
+    vals = []
+    cb = None
+    for s in range(args.warmup + args.steps):
+        cb = cpu_baseline(x, n, hq, hkv, d, B, tau, budget)
+        if s >= args.warmup:
+            vals.append(cb["value"])
+    v = float(np.mean(vals))
+    line = {
+        "metric": METRIC, "value": round(v, 1), "unit": "ms/layer", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(v, 1), "higher_is_better": False, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded heavy-block generator)",
+        "config": {"workload": args.workload, "n_tokens": n, "n_q_heads": hq, "n_kv_heads": hkv, "head_dim": d,
+                   "block": B, "n_sample": 16, "tau": tau, "seed": args.seed},
+        "impl": "reference",
+        "cpu_baseline": {"value": round(v, 1), "unit": "ms/layer", "cores": cb["cores"], "kind": "oracle",
+                         "sample": cb["sample"]},
+        "e2e": {"value": round(v, 1), "unit": "ms/layer", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="llama3.1-8b-layer-128k")
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-quality", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget-s", type=float, default=15.0)
+    ap.add_argument("--ref-step-budget-s", type=float, default=8.0)
+    args = ap.parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,232 @@
+"""Python binding of libpoem (include/poem.h): POEM output-relative block-sparse
+attention prefill on B200 (sm_100a).
+
+Argument marshalling only: every step of the path runs in the CUDA kernels of
+``libpoem.so``; PyTorch supplies device memory and the current stream.  The
+library is loaded from this package directory and there is no fallback: if it
+is missing or fails to load, importing the binding raises.
+
+Functions carry the C names:
+    poem_workspace_size(shape) -> (score_bytes, select_bytes, fwd_bytes)
+    poem_score(q, k, v, I_hat, m_hat, ws, block=128, n_sample=16, scale=0.0)
+    poem_select(I_hat, m_hat, tau, row_ptr, col_idx, ws, shape..., order=None)
+    poem_select_mass_only(m_hat, ref_row_ptr, row_ptr, col_idx, ws, ...)
+    bsa_fwd(q, k, v, row_ptr, col_idx, o, ws, lse=None, order=None, block=128)
+    poem_check(ws) -> raises on a device-side error
+and ``prefill_layer`` chains the three calls for one attention layer.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libpoem.so")
+
+POEM_OK = 0
+STATUS = {
+    0: "POEM_OK", 1: "POEM_ERR_INVALID_ARG", 2: "POEM_ERR_UNSUPPORTED", 3: "POEM_ERR_CUDA",
+    4: "POEM_ERR_TIMEOUT", 5: "POEM_ERR_CAPACITY", 6: "POEM_ERR_WORKSPACE", 7: "POEM_ERR_BAD_LIST",
+}
+
+EXPORTED = (
+    "poem_workspace_size", "poem_score", "poem_select", "poem_select_mass_only", "bsa_fwd",
+    "poem_check", "poem_set_wait_limit_ns", "poem_status_string", "poem_last_error",
+)
+
+
+class PoemError(RuntimeError):
+    def __init__(self, status: int, where: str, detail: str = ""):
+        self.status = status
+        super().__init__(f"{where}: {STATUS.get(status, status)}" + (f" ({detail})" if detail else ""))
+
+
+class Shape(ctypes.Structure):
+    _fields_ = [
+        ("n_tokens", ctypes.c_int32), ("n_q_heads", ctypes.c_int32), ("n_kv_heads", ctypes.c_int32),
+        ("head_dim", ctypes.c_int32), ("block", ctypes.c_int32), ("n_sample", ctypes.c_int32),
+        ("softmax_scale", ctypes.c_float), ("reserved0", ctypes.c_int32),
+        ("q_stride_tok", ctypes.c_int64), ("q_stride_head", ctypes.c_int64),
+        ("kv_stride_tok", ctypes.c_int64), ("kv_stride_head", ctypes.c_int64),
+        ("o_stride_tok", ctypes.c_int64), ("o_stride_head", ctypes.c_int64),
+    ]
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"libpoem.so not built at {LIB_PATH}; run block_sparse_attention_poem_b200/build.py")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, sp, i64, sz = ctypes.c_void_p, ctypes.POINTER(Shape), ctypes.c_int64, ctypes.c_size_t
+    st = ctypes.c_int
+    lib.poem_workspace_size.argtypes = [sp, ctypes.POINTER(sz), ctypes.POINTER(sz), ctypes.POINTER(sz)]
+    lib.poem_workspace_size.restype = st
+    lib.poem_score.argtypes = [sp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.poem_score.restype = st
+    lib.poem_select.argtypes = [sp, vp, vp, ctypes.c_float, vp, vp, i64, vp, vp, sz, vp]
+    lib.poem_select.restype = st
+    lib.poem_select_mass_only.argtypes = [sp, vp, vp, vp, vp, i64, vp, vp, sz, vp]
+    lib.poem_select_mass_only.restype = st
+    lib.bsa_fwd.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.bsa_fwd.restype = st
+    lib.poem_check.argtypes = [vp, vp]
+    lib.poem_check.restype = st
+    lib.poem_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
+    lib.poem_set_wait_limit_ns.restype = None
+    lib.poem_status_string.argtypes = [st]
+    lib.poem_status_string.restype = ctypes.c_char_p
+    lib.poem_last_error.argtypes = []
+    lib.poem_last_error.restype = ctypes.c_char_p
+    return lib
+
+
+_lib = _load()
+
+
+def _raise(status: int, where: str):
+    if status != POEM_OK:
+        raise PoemError(status, where, _lib.poem_last_error().decode(errors="replace"))
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def make_shape(q: torch.Tensor, k: torch.Tensor, block: int = 128, n_sample: int = 16, scale: float = 0.0,
+               o: torch.Tensor | None = None) -> Shape:
+    """Shape of a layer from q [N, Hq, d] and k/v [N, Hkv, d] (any strides with a
+    contiguous head dimension); o defaults to q's strides."""
+    n, hq, d = q.shape
+    hkv = k.shape[1]
+    if q.stride(2) != 1 or k.stride(2) != 1:
+        raise ValueError("the head dimension must be contiguous")
+    o_st = (o.stride(0), o.stride(1)) if o is not None else (q.stride(0), q.stride(1))
+    return Shape(n, hq, hkv, d, block, n_sample, float(scale), 0, q.stride(0), q.stride(1), k.stride(0),
+                 k.stride(1), o_st[0], o_st[1])
+
+
+def poem_workspace_size(shape: Shape):
+    a, b, c = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
+    _raise(_lib.poem_workspace_size(ctypes.byref(shape), ctypes.byref(a), ctypes.byref(b), ctypes.byref(c)),
+           "poem_workspace_size")
+    return a.value, b.value, c.value
+
+
+def alloc_workspace(nbytes: int, device="cuda") -> torch.Tensor:
+    """Zero-filled workspace buffer (the error word must start clear)."""
+    return torch.zeros(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+def n_score_entries(n_q_heads: int, n_tiles: int) -> int:
+    return n_q_heads * n_tiles * (n_tiles + 1) // 2
+
+
+def _check_bf16(*ts):
+    for t in ts:
+        if t.dtype != torch.bfloat16 or not t.is_cuda:
+            raise TypeError("q, k, v, o must be CUDA bfloat16 tensors")
+
+
+def poem_score(q, k, v, I_hat, m_hat, ws, shape: Shape | None = None, stream=None, **shape_kw):
+    _check_bf16(q, k, v)
+    shape = shape or make_shape(q, k, **shape_kw)
+    _raise(_lib.poem_score(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(I_hat), _ptr(m_hat), _ptr(ws),
+                           ws.numel() * ws.element_size(), _stream(stream)), "poem_score")
+
+
+def poem_select(shape: Shape, I_hat, m_hat, tau: float, row_ptr, col_idx, ws, order=None, stream=None):
+    _raise(_lib.poem_select(ctypes.byref(shape), _ptr(I_hat), _ptr(m_hat), ctypes.c_float(tau), _ptr(row_ptr),
+                            _ptr(col_idx), col_idx.numel(), _ptr(order), _ptr(ws), ws.numel() * ws.element_size(),
+                            _stream(stream)), "poem_select")
+
+
+def poem_select_mass_only(shape: Shape, m_hat, ref_row_ptr, row_ptr, col_idx, ws, order=None, stream=None):
+    _raise(_lib.poem_select_mass_only(ctypes.byref(shape), _ptr(m_hat), _ptr(ref_row_ptr), _ptr(row_ptr),
+                                      _ptr(col_idx), col_idx.numel(), _ptr(order), _ptr(ws),
+                                      ws.numel() * ws.element_size(), _stream(stream)), "poem_select_mass_only")
+
+
+def bsa_fwd(q, k, v, row_ptr, col_idx, o, ws, lse=None, order=None, shape: Shape | None = None, stream=None,
+            **shape_kw):
+    _check_bf16(q, k, v, o)
+    shape = shape or make_shape(q, k, o=o, **shape_kw)
+    _raise(_lib.bsa_fwd(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(row_ptr), _ptr(col_idx), _ptr(order),
+                        _ptr(o), _ptr(lse), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)), "bsa_fwd")
+
+
+def poem_check(ws, stream=None):
+    """Synchronise and raise PoemError if a kernel recorded a device-side error."""
+    _raise(_lib.poem_check(_stream(stream), _ptr(ws)), "poem_check")
+
+
+def poem_check_status(ws, stream=None) -> int:
+    return int(_lib.poem_check(_stream(stream), _ptr(ws)))
+
+
+def poem_set_wait_limit_ns(ns: int):
+    _lib.poem_set_wait_limit_ns(int(ns))
+
+
+def poem_status_string(status: int) -> str:
+    return _lib.poem_status_string(int(status)).decode()
+
+
+def poem_last_error() -> str:
+    return _lib.poem_last_error().decode(errors="replace")
+
+
+@dataclass
+class Layer:
+    """Device buffers of one prefill layer (reused across calls)."""
+    shape: Shape
+    I_hat: torch.Tensor
+    m_hat: torch.Tensor
+    row_ptr: torch.Tensor
+    col_idx: torch.Tensor
+    order: torch.Tensor
+    o: torch.Tensor
+    lse: torch.Tensor | None
+    ws_score: torch.Tensor
+    ws_select: torch.Tensor
+    ws_fwd: torch.Tensor
+
+
+def alloc_layer(q, k, block: int = 128, n_sample: int = 16, with_lse: bool = False) -> Layer:
+    shape = make_shape(q, k, block=block, n_sample=n_sample)
+    n, hq, d = q.shape
+    T = n // block
+    s_b, sel_b, f_b = poem_workspace_size(shape)
+    dev = q.device
+    ne = n_score_entries(hq, T)
+    return Layer(
+        shape=shape,
+        I_hat=torch.empty(ne, dtype=torch.float32, device=dev),
+        m_hat=torch.empty(ne, dtype=torch.float32, device=dev),
+        row_ptr=torch.empty(hq * T + 1, dtype=torch.int32, device=dev),
+        col_idx=torch.empty(ne, dtype=torch.int32, device=dev),
+        order=torch.empty(hq * T, dtype=torch.int32, device=dev),
+        o=torch.empty_like(q),
+        lse=torch.empty(hq, n, dtype=torch.float32, device=dev) if with_lse else None,
+        ws_score=alloc_workspace(s_b, dev),
+        ws_select=alloc_workspace(sel_b, dev),
+        ws_fwd=alloc_workspace(f_b, dev),
+    )
+
+
+def prefill_layer(q, k, v, tau: float, layer: Layer | None = None, block: int = 128, stream=None) -> Layer:
+    """Score, select and attend for one layer; returns the buffers (o in layer.o)."""
+    layer = layer or alloc_layer(q, k, block=block)
+    poem_score(q, k, v, layer.I_hat, layer.m_hat, layer.ws_score, shape=layer.shape, stream=stream)
+    poem_select(layer.shape, layer.I_hat, layer.m_hat, tau, layer.row_ptr, layer.col_idx, layer.ws_select,
+                order=layer.order, stream=stream)
+    bsa_fwd(q, k, v, layer.row_ptr, layer.col_idx, layer.o, layer.ws_fwd, lse=layer.lse, order=layer.order,
+            shape=layer.shape, stream=stream)
+    return layer

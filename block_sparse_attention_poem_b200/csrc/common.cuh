@@ -1,0 +1,87 @@
+// common.cuh -- parameter blocks shared by the host entry points and the kernels.
+#pragma once
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "sm100.cuh"
+
+namespace poem {
+
+constexpr int kWsHeader = 256;          // bytes reserved at the start of every workspace
+constexpr int kThreadsFwd = 192;        // 4 softmax warps + 1 TMA warp + 1 MMA warp
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+// Launch order of the (head, tile) rows of a layer when no explicit order is
+// given: KV-head-major (so the CTAs that run together share one KV head's keys
+// and values in L2), last tile first (longest causal rows first), and the query
+// heads of a group next to each other.
+__host__ __device__ __forceinline__ int default_row_of_unit(int u, int n_tiles, int group) {
+  const int per_g = n_tiles * group;
+  const int g = u / per_g;
+  const int rem = u - g * per_g;
+  const int i = n_tiles - 1 - rem / group;
+  const int h = g * group + rem % group;
+  return h * n_tiles + i;
+}
+
+struct FwdParams {
+  const int32_t* row_ptr;
+  const int32_t* col_idx;
+  const int32_t* order;
+  __nv_bfloat16* o;
+  float* lse;
+  int64_t o_stride_tok;
+  int64_t o_stride_head;
+  int n_tokens;
+  int n_q_heads;
+  int n_tiles;
+  int group;          // query heads per KV head
+  float scale_log2;   // softmax_scale * log2(e)
+  DevErr err;
+};
+
+struct ScoreParams {
+  float* I_hat;        // packed lower-triangular [Hq, T(T+1)/2]
+  float* m_hat;
+  float* ws_o;         // [Hq, T, S, D] fp32 dense outputs of the sampled queries
+  float* ws_lse;       // [Hq, T, S] fp32 log2-domain log-sum-exp (scaled logits)
+  int n_tokens;
+  int n_q_heads;
+  int n_kv_heads;
+  int n_tiles;
+  int group;
+  int n_sample;        // S
+  int sample_stride;   // B / S
+  float scale_log2;
+  DevErr err;
+};
+
+struct SelectParams {
+  const float* I_hat;
+  const float* m_hat;
+  const int32_t* ref_row_ptr;  // mass-only: budget source (nullable)
+  int32_t* counts;             // [rows] list lengths
+  int32_t* scratch;            // [Hq * T(T+1)/2] ids at each row's triangular offset
+  int32_t* row_ptr;
+  int32_t* col_idx;
+  int32_t* order;
+  int64_t col_capacity;
+  int n_q_heads;
+  int n_tiles;
+  int group;
+  double tau;
+  int mass_only;
+  DevErr err;
+};
+
+// Launchers (defined in the kernel translation units).
+cudaError_t launch_bsa_fwd(int head_dim, int block, const CUtensorMap& tmQ, const CUtensorMap& tmK,
+                           const CUtensorMap& tmV, const FwdParams& p, int n_units, cudaStream_t stream);
+cudaError_t launch_score(int head_dim, int block, const CUtensorMap& tmQs, const CUtensorMap& tmK,
+                         const CUtensorMap& tmV, const ScoreParams& p, cudaStream_t stream);
+cudaError_t launch_select(const SelectParams& p, cudaStream_t stream);
+
+}  // namespace poem

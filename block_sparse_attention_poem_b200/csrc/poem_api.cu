@@ -1,0 +1,315 @@
+// poem_api.cu -- host side of the C ABI declared in include/poem.h: argument
+// validation, workspace layout, TMA descriptor encoding and kernel launches.
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/poem.h"
+#include "common.cuh"
+
+namespace {
+
+thread_local char g_last_error[512] = {0};
+uint64_t g_wait_limit_ns = 2000000000ull;
+
+poem_status cuda_fail(cudaError_t e, const char* where) {
+  std::snprintf(g_last_error, sizeof g_last_error, "%s: %s (%s)", where, cudaGetErrorName(e), cudaGetErrorString(e));
+  return POEM_ERR_CUDA;
+}
+
+poem_status arg_fail(poem_status s, const char* what) {
+  std::snprintf(g_last_error, sizeof g_last_error, "%s", what);
+  return s;
+}
+
+bool aligned16(const void* p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+struct Layout {
+  int T;       // tiles
+  int G;       // query heads per KV head
+  float scale; // softmax scale
+};
+
+constexpr int kMaxTiles = 8192;
+
+// Shape checks shared by every entry point.
+poem_status check_shape(const poem_shape* s, Layout* out) {
+  if (!s) return arg_fail(POEM_ERR_INVALID_ARG, "shape is NULL");
+  if (s->n_tokens <= 0 || s->n_q_heads <= 0 || s->n_kv_heads <= 0 || s->head_dim <= 0 || s->block <= 0)
+    return arg_fail(POEM_ERR_INVALID_ARG, "sizes must be positive");
+  if (s->n_q_heads % s->n_kv_heads) return arg_fail(POEM_ERR_INVALID_ARG, "n_q_heads % n_kv_heads != 0");
+  if (s->n_tokens % s->block) return arg_fail(POEM_ERR_INVALID_ARG, "n_tokens % block != 0");
+  if (!(s->softmax_scale >= 0.f) || !std::isfinite(s->softmax_scale))
+    return arg_fail(POEM_ERR_INVALID_ARG, "softmax_scale must be finite and >= 0");
+  if (s->head_dim != 64 && s->head_dim != 128) return arg_fail(POEM_ERR_UNSUPPORTED, "head_dim must be 64 or 128");
+  if (s->block != 64 && s->block != 128) return arg_fail(POEM_ERR_UNSUPPORTED, "block must be 64 or 128");
+  if (s->n_tokens / s->block > kMaxTiles) return arg_fail(POEM_ERR_UNSUPPORTED, "more than 8192 tiles");
+  const int64_t strides[6] = {s->q_stride_tok, s->q_stride_head, s->kv_stride_tok,
+                              s->kv_stride_head, s->o_stride_tok, s->o_stride_head};
+  for (int64_t st : strides)
+    if (st <= 0 || (st % 8) != 0 || st >= (int64_t(1) << 38))
+      return arg_fail(POEM_ERR_INVALID_ARG, "strides must be positive multiples of 8 elements");
+  out->T = s->n_tokens / s->block;
+  out->G = s->n_q_heads / s->n_kv_heads;
+  out->scale = s->softmax_scale > 0.f ? s->softmax_scale : 1.0f / std::sqrt((float)s->head_dim);
+  return POEM_OK;
+}
+
+size_t tri_entries(const poem_shape* s, int T) { return (size_t)s->n_q_heads * (size_t)T * (size_t)(T + 1) / 2; }
+
+size_t score_ws_bytes(const poem_shape* s, int T) {
+  const size_t rows = (size_t)s->n_q_heads * T * s->n_sample;
+  return poem::kWsHeader + round_up(rows * s->head_dim * sizeof(float), 256) + round_up(rows * sizeof(float), 256);
+}
+
+size_t select_ws_bytes(const poem_shape* s, int T) {
+  const size_t rows = (size_t)s->n_q_heads * T;
+  return poem::kWsHeader + round_up(rows * sizeof(int32_t), 256) + round_up(tri_entries(s, T) * sizeof(int32_t), 256);
+}
+
+size_t fwd_ws_bytes(const poem_shape*, int) { return poem::kWsHeader; }
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// [n_tokens, n_heads, head_dim] bf16 viewed as a 3-D tensor (head_dim, head, token);
+// box = 64 elements x 1 head x box_rows tokens, 128-byte swizzle.
+poem_status make_map_3d(CUtensorMap* m, const void* base, int head_dim, int n_heads, int n_tokens, int64_t st_head,
+                        int64_t st_tok, int box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return arg_fail(POEM_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
+  cuuint64_t dims[3] = {(cuuint64_t)head_dim, (cuuint64_t)n_heads, (cuuint64_t)n_tokens};
+  cuuint64_t strides[2] = {(cuuint64_t)st_head * 2, (cuuint64_t)st_tok * 2};
+  cuuint32_t box[3] = {64, 1, (cuuint32_t)box_rows};
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    std::snprintf(g_last_error, sizeof g_last_error, "cuTensorMapEncodeTiled (3d) failed: %d", (int)r);
+    return POEM_ERR_CUDA;
+  }
+  return POEM_OK;
+}
+
+// Sampled queries of q viewed as (head_dim, head, sample j, tile i): token iB + j*stride.
+poem_status make_map_sampled(CUtensorMap* m, const void* base, const poem_shape* s, int T) {
+  auto fn = encode_fn();
+  if (!fn) return arg_fail(POEM_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
+  const int stride = s->block / s->n_sample;
+  cuuint64_t dims[4] = {(cuuint64_t)s->head_dim, (cuuint64_t)s->n_q_heads, (cuuint64_t)s->n_sample, (cuuint64_t)T};
+  cuuint64_t strides[3] = {(cuuint64_t)s->q_stride_head * 2, (cuuint64_t)s->q_stride_tok * 2 * stride,
+                           (cuuint64_t)s->q_stride_tok * 2 * s->block};
+  cuuint32_t box[4] = {64, 1, (cuuint32_t)s->n_sample, 1};
+  cuuint32_t es[4] = {1, 1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    std::snprintf(g_last_error, sizeof g_last_error, "cuTensorMapEncodeTiled (4d) failed: %d", (int)r);
+    return POEM_ERR_CUDA;
+  }
+  return POEM_OK;
+}
+
+poem::DevErr dev_err(void* ws) { return poem::DevErr{reinterpret_cast<uint32_t*>(ws), g_wait_limit_ns}; }
+
+}  // namespace
+
+extern "C" {
+
+poem_status poem_workspace_size(const poem_shape* shape, size_t* score_bytes, size_t* select_bytes,
+                                size_t* fwd_bytes) {
+  Layout L;
+  poem_status st = check_shape(shape, &L);
+  if (st != POEM_OK) return st;
+  if (score_bytes) *score_bytes = score_ws_bytes(shape, L.T);
+  if (select_bytes) *select_bytes = select_ws_bytes(shape, L.T);
+  if (fwd_bytes) *fwd_bytes = fwd_ws_bytes(shape, L.T);
+  return POEM_OK;
+}
+
+poem_status poem_score(const poem_shape* shape, const poem_bf16* q, const poem_bf16* k, const poem_bf16* v,
+                       float* I_hat, float* m_hat, void* ws, size_t ws_bytes, void* stream) {
+  Layout L;
+  poem_status st = check_shape(shape, &L);
+  if (st != POEM_OK) return st;
+  if (shape->n_sample != 16 || shape->block % shape->n_sample)
+    return arg_fail(POEM_ERR_UNSUPPORTED, "n_sample must be 16");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(I_hat) || !aligned16(m_hat) || !aligned16(ws))
+    return arg_fail(POEM_ERR_INVALID_ARG, "pointers must be non-NULL and 16-byte aligned");
+  if (ws_bytes < score_ws_bytes(shape, L.T)) return arg_fail(POEM_ERR_WORKSPACE, "score workspace too small");
+  CUtensorMap tmQs, tmK, tmV;
+  if ((st = make_map_sampled(&tmQs, q, shape, L.T)) != POEM_OK) return st;
+  if ((st = make_map_3d(&tmK, k, shape->head_dim, shape->n_kv_heads, shape->n_tokens, shape->kv_stride_head,
+                        shape->kv_stride_tok, shape->block)) != POEM_OK)
+    return st;
+  if ((st = make_map_3d(&tmV, v, shape->head_dim, shape->n_kv_heads, shape->n_tokens, shape->kv_stride_head,
+                        shape->kv_stride_tok, shape->block)) != POEM_OK)
+    return st;
+  const size_t rows = (size_t)shape->n_q_heads * L.T * shape->n_sample;
+  uint8_t* base = reinterpret_cast<uint8_t*>(ws);
+  poem::ScoreParams p{};
+  p.I_hat = I_hat;
+  p.m_hat = m_hat;
+  p.ws_o = reinterpret_cast<float*>(base + poem::kWsHeader);
+  p.ws_lse = reinterpret_cast<float*>(base + poem::kWsHeader + round_up(rows * shape->head_dim * sizeof(float), 256));
+  p.n_tokens = shape->n_tokens;
+  p.n_q_heads = shape->n_q_heads;
+  p.n_kv_heads = shape->n_kv_heads;
+  p.n_tiles = L.T;
+  p.group = L.G;
+  p.n_sample = shape->n_sample;
+  p.sample_stride = shape->block / shape->n_sample;
+  p.scale_log2 = L.scale * poem::kLog2e;
+  p.err = dev_err(ws);
+  cudaError_t e = poem::launch_score(shape->head_dim, shape->block, tmQs, tmK, tmV, p, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "poem_score launch");
+  return POEM_OK;
+}
+
+static poem_status select_common(const poem_shape* shape, const float* I_hat, const float* m_hat,
+                                 const int32_t* ref_row_ptr, double tau, int mass_only, int32_t* row_ptr,
+                                 int32_t* col_idx, int64_t col_capacity, int32_t* order, void* ws, size_t ws_bytes,
+                                 void* stream) {
+  Layout L;
+  poem_status st = check_shape(shape, &L);
+  if (st != POEM_OK) return st;
+  if ((!mass_only && !aligned16(I_hat)) || !aligned16(m_hat) || !aligned16(row_ptr) || !aligned16(ws) ||
+      (col_capacity > 0 && !aligned16(col_idx)) || (order && !aligned16(order)) ||
+      (mass_only && !aligned16(ref_row_ptr)))
+    return arg_fail(POEM_ERR_INVALID_ARG, "pointers must be non-NULL and 16-byte aligned");
+  if (col_capacity < 0) return arg_fail(POEM_ERR_INVALID_ARG, "col_capacity < 0");
+  if (!mass_only && (!std::isfinite(tau) || tau < 0.0)) return arg_fail(POEM_ERR_INVALID_ARG, "tau must be finite and >= 0");
+  if (ws_bytes < select_ws_bytes(shape, L.T)) return arg_fail(POEM_ERR_WORKSPACE, "select workspace too small");
+  if (order && L.G * L.T > (1 << 14)) return arg_fail(POEM_ERR_UNSUPPORTED, "work order needs group*tiles <= 16384");
+  const size_t rows = (size_t)shape->n_q_heads * L.T;
+  uint8_t* base = reinterpret_cast<uint8_t*>(ws);
+  poem::SelectParams p{};
+  p.I_hat = I_hat;
+  p.m_hat = m_hat;
+  p.ref_row_ptr = ref_row_ptr;
+  p.counts = reinterpret_cast<int32_t*>(base + poem::kWsHeader);
+  p.scratch = reinterpret_cast<int32_t*>(base + poem::kWsHeader + round_up(rows * sizeof(int32_t), 256));
+  p.row_ptr = row_ptr;
+  p.col_idx = col_idx;
+  p.order = order;
+  p.col_capacity = col_capacity;
+  p.n_q_heads = shape->n_q_heads;
+  p.n_tiles = L.T;
+  p.group = L.G;
+  p.tau = tau;
+  p.mass_only = mass_only;
+  p.err = dev_err(ws);
+  cudaError_t e = poem::launch_select(p, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "poem_select launch");
+  return POEM_OK;
+}
+
+poem_status poem_select(const poem_shape* shape, const float* I_hat, const float* m_hat, float tau,
+                        int32_t* row_ptr, int32_t* col_idx, int64_t col_capacity, int32_t* order, void* ws,
+                        size_t ws_bytes, void* stream) {
+  if (!std::isfinite(tau) || tau < 0.f) return arg_fail(POEM_ERR_INVALID_ARG, "tau must be finite and >= 0");
+  return select_common(shape, I_hat, m_hat, nullptr, (double)tau, 0, row_ptr, col_idx, col_capacity, order, ws,
+                       ws_bytes, stream);
+}
+
+poem_status poem_select_mass_only(const poem_shape* shape, const float* m_hat, const int32_t* ref_row_ptr,
+                                  int32_t* row_ptr, int32_t* col_idx, int64_t col_capacity, int32_t* order,
+                                  void* ws, size_t ws_bytes, void* stream) {
+  return select_common(shape, nullptr, m_hat, ref_row_ptr, 0.0, 1, row_ptr, col_idx, col_capacity, order, ws,
+                       ws_bytes, stream);
+}
+
+poem_status bsa_fwd(const poem_shape* shape, const poem_bf16* q, const poem_bf16* k, const poem_bf16* v,
+                    const int32_t* row_ptr, const int32_t* col_idx, const int32_t* order, poem_bf16* o, float* lse,
+                    void* ws, size_t ws_bytes, void* stream) {
+  Layout L;
+  poem_status st = check_shape(shape, &L);
+  if (st != POEM_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(row_ptr) || !aligned16(o) || !aligned16(ws) ||
+      (col_idx && !aligned16(col_idx)) || (order && !aligned16(order)) || (lse && !aligned16(lse)))
+    return arg_fail(POEM_ERR_INVALID_ARG, "pointers must be non-NULL and 16-byte aligned");
+  if (ws_bytes < fwd_ws_bytes(shape, L.T)) return arg_fail(POEM_ERR_WORKSPACE, "fwd workspace too small");
+  CUtensorMap tmQ, tmK, tmV;
+  if ((st = make_map_3d(&tmQ, q, shape->head_dim, shape->n_q_heads, shape->n_tokens, shape->q_stride_head,
+                        shape->q_stride_tok, 128)) != POEM_OK)
+    return st;
+  if ((st = make_map_3d(&tmK, k, shape->head_dim, shape->n_kv_heads, shape->n_tokens, shape->kv_stride_head,
+                        shape->kv_stride_tok, shape->block)) != POEM_OK)
+    return st;
+  if ((st = make_map_3d(&tmV, v, shape->head_dim, shape->n_kv_heads, shape->n_tokens, shape->kv_stride_head,
+                        shape->kv_stride_tok, shape->block)) != POEM_OK)
+    return st;
+  poem::FwdParams p{};
+  p.row_ptr = row_ptr;
+  p.col_idx = col_idx;
+  p.order = order;
+  p.o = reinterpret_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.o_stride_tok = shape->o_stride_tok;
+  p.o_stride_head = shape->o_stride_head;
+  p.n_tokens = shape->n_tokens;
+  p.n_q_heads = shape->n_q_heads;
+  p.n_tiles = L.T;
+  p.group = L.G;
+  p.scale_log2 = L.scale * poem::kLog2e;
+  p.err = dev_err(ws);
+  cudaError_t e = poem::launch_bsa_fwd(shape->head_dim, shape->block, tmQ, tmK, tmV, p, shape->n_q_heads * L.T,
+                                       (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "bsa_fwd launch");
+  return POEM_OK;
+}
+
+poem_status poem_check(void* stream, void* ws) {
+  if (!aligned16(ws)) return arg_fail(POEM_ERR_INVALID_ARG, "ws must be non-NULL and 16-byte aligned");
+  cudaStream_t s = (cudaStream_t)stream;
+  uint32_t word = 0;
+  cudaError_t e = cudaMemcpyAsync(&word, ws, sizeof word, cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "poem_check");
+  if (word) {
+    e = cudaMemsetAsync(ws, 0, sizeof word, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_fail(e, "poem_check reset");
+  }
+  if (word & poem::kErrTimeout) return POEM_ERR_TIMEOUT;
+  if (word & poem::kErrBadList) return POEM_ERR_BAD_LIST;
+  if (word & poem::kErrCapacity) return POEM_ERR_CAPACITY;
+  return POEM_OK;
+}
+
+void poem_set_wait_limit_ns(uint64_t ns) { g_wait_limit_ns = ns; }
+
+const char* poem_status_string(poem_status s) {
+  switch (s) {
+    case POEM_OK: return "POEM_OK";
+    case POEM_ERR_INVALID_ARG: return "POEM_ERR_INVALID_ARG";
+    case POEM_ERR_UNSUPPORTED: return "POEM_ERR_UNSUPPORTED";
+    case POEM_ERR_CUDA: return "POEM_ERR_CUDA";
+    case POEM_ERR_TIMEOUT: return "POEM_ERR_TIMEOUT";
+    case POEM_ERR_CAPACITY: return "POEM_ERR_CAPACITY";
+    case POEM_ERR_WORKSPACE: return "POEM_ERR_WORKSPACE";
+    case POEM_ERR_BAD_LIST: return "POEM_ERR_BAD_LIST";
+  }
+  return "POEM_ERR_UNKNOWN";
+}
+
+const char* poem_last_error(void) { return g_last_error; }
+
+}  // extern "C"

@@ -1,0 +1,328 @@
+// poem_select.cu -- threshold block selection and CSR emission (sm_100a, CUDA cores).
+//
+// Per (head h, query tile i) row, from the aggregated scores I_hat[h, i, 0..i] and
+// masses m_hat[h, i, 0..i]:
+//   mandatory  {0, i-1, i}       (sink, local and diagonal blocks)
+//   candidates {1, .., i-2}, ranked by (I_hat desc, id asc)
+//   D_k        the candidates ranked k, k+1, ..  (dropped when the top k are kept)
+//   keep the top k for the smallest k with  S_m(k) < 1  and  S_I(k) <= tau (1 - S_m(k)),
+//   S_I(k) = sum_{D_k} I_hat,  S_m(k) = sum_{D_k} m_hat   (fp64 suffix sums),
+// which makes the triangle bound of the reading note "Attention deletion error",
+// Equation (4), hold with the max-aggregated scores.  Equal scores favour the
+// smaller id and lists are emitted in ascending id order, as in the appendix
+// "Block ordering" of the "Block-Filtered Long-Context Attention" page.
+//
+// Kernels (all on the caller's stream):
+//   select_rows   one CTA per row: bitonic sort of 64-bit keys (~bits(score) : id)
+//                 in shared memory, fp64 suffix scan, min-reduce of the cut,
+//                 ascending compaction into the row's triangular scratch slot.
+//   scan_counts   one CTA: exclusive scan of the list lengths -> row_ptr.
+//   gather_lists  one CTA per row: scratch -> col_idx (bounded by the capacity).
+//   work_order    one CTA per KV head: rows of the head group by list length desc.
+#include "common.cuh"
+
+namespace poem {
+namespace {
+
+constexpr int kSelThreads = 256;
+
+__device__ __forceinline__ int64_t tri_off(int n_tiles, int h, int i) {
+  return (int64_t)h * ((int64_t)n_tiles * (n_tiles + 1) / 2) + (int64_t)i * (i + 1) / 2;
+}
+
+// Ascending bitonic sort of n (power of two) 64-bit keys in shared memory.
+__device__ void bitonic_sort_u64(uint64_t* a, int n) {
+  for (int k = 2; k <= n; k <<= 1) {
+    for (int jj = k >> 1; jj > 0; jj >>= 1) {
+      for (int t = threadIdx.x; t < n; t += blockDim.x) {
+        const int partner = t ^ jj;
+        if (partner > t) {
+          const bool up = ((t & k) == 0);
+          const uint64_t x = a[t], y = a[partner];
+          if ((x > y) == up) {
+            a[t] = y;
+            a[partner] = x;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+}
+
+__device__ void bitonic_sort_u32(uint32_t* a, int n) {
+  for (int k = 2; k <= n; k <<= 1) {
+    for (int jj = k >> 1; jj > 0; jj >>= 1) {
+      for (int t = threadIdx.x; t < n; t += blockDim.x) {
+        const int partner = t ^ jj;
+        if (partner > t) {
+          const bool up = ((t & k) == 0);
+          const uint32_t x = a[t], y = a[partner];
+          if ((x > y) == up) {
+            a[t] = y;
+            a[partner] = x;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+}
+
+// Block-wide exclusive scan of one int per thread (blockDim.x == kSelThreads).
+__device__ int block_excl_scan_int(int v, int* tmp, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) tmp[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int w = (lane < kSelThreads / 32) ? tmp[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += y;
+    }
+    if (lane < kSelThreads / 32) tmp[lane] = w;
+  }
+  __syncthreads();
+  const int base = (warp > 0) ? tmp[warp - 1] : 0;
+  *total = tmp[kSelThreads / 32 - 1];
+  __syncthreads();
+  return base + x - v;
+}
+
+// Block-wide exclusive *suffix* scan (sum over higher thread ids) of a double pair.
+__device__ void block_suffix_scan_d2(double a, double b, double* tmpa, double* tmpb, double& ea, double& eb) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  double xa = a, xb = b;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const double ya = __shfl_down_sync(0xffffffffu, xa, o);
+    const double yb = __shfl_down_sync(0xffffffffu, xb, o);
+    if (lane + o < 32) {
+      xa += ya;
+      xb += yb;
+    }
+  }
+  // xa: inclusive suffix within the warp; the exclusive one is the next lane's.
+  double na = __shfl_down_sync(0xffffffffu, xa, 1);
+  double nb = __shfl_down_sync(0xffffffffu, xb, 1);
+  if (lane == 31) {
+    na = 0.0;
+    nb = 0.0;
+  }
+  if (lane == 0) {
+    tmpa[warp] = xa;
+    tmpb[warp] = xb;
+  }
+  __syncthreads();
+  double wa = 0.0, wb = 0.0;
+  for (int w = kSelThreads / 32 - 1; w > warp; --w) {
+    wa += tmpa[w];
+    wb += tmpb[w];
+  }
+  ea = na + wa;
+  eb = nb + wb;
+  __syncthreads();
+}
+
+__global__ void __launch_bounds__(kSelThreads) select_rows_kernel(const SelectParams p) {
+  extern __shared__ __align__(16) uint8_t sm[];
+  const int row = blockIdx.x;
+  const int T = p.n_tiles;
+  const int h = row / T;
+  const int i = row - h * T;
+  const int nc = max(0, i - 2);
+  int P = 1;
+  while (P < nc) P <<= 1;
+  uint64_t* keys = reinterpret_cast<uint64_t*>(sm);                      // [P]
+  int* keep = reinterpret_cast<int*>(sm + sizeof(uint64_t) * (size_t)max(P, 1));  // [T]
+  __shared__ double tmpa[kSelThreads / 32], tmpb[kSelThreads / 32];
+  __shared__ int tmpi[kSelThreads / 32];
+  __shared__ int s_kcut;
+
+  const int64_t off = tri_off(T, h, i);
+  const float* Ih = p.I_hat + off;
+  const float* mh = p.m_hat + off;
+  const float* rank_src = p.mass_only ? mh : Ih;
+
+  for (int t = threadIdx.x; t < P; t += blockDim.x) {
+    uint64_t key = ~0ull;
+    if (t < nc) {
+      const int id = t + 1;
+      const float sc = fmaxf(rank_src[id], 0.f);  // canonical +0 for zero scores
+      key = ((uint64_t)(~__float_as_uint(sc)) << 32) | (uint32_t)id;
+    }
+    keys[t] = key;
+  }
+  for (int b = threadIdx.x; b <= i; b += blockDim.x) keep[b] = 0;
+  if (threadIdx.x == 0) s_kcut = nc;
+  __syncthreads();
+  if (nc > 1) bitonic_sort_u64(keys, P);
+
+  int kcut = nc;
+  if (p.mass_only) {
+    const int ref = p.ref_row_ptr[row + 1] - p.ref_row_ptr[row];
+    const int n_mand = (i == 0) ? 1 : (i == 1 ? 2 : 3);
+    kcut = min(max(ref - n_mand, 0), nc);
+  } else if (nc > 0) {
+    // Each thread owns a contiguous run of ranks; suffix sums inside the run, then
+    // a block suffix scan of the run totals.
+    const int E = (nc + kSelThreads - 1) / kSelThreads;
+    const int r0 = threadIdx.x * E;
+    const int r1 = min(nc, r0 + E);
+    double ta = 0.0, tb = 0.0;
+    for (int r = r1 - 1; r >= r0; --r) {
+      const int id = (int)(keys[r] & 0xffffffffu);
+      ta += (double)Ih[id];
+      tb += (double)mh[id];
+    }
+    double ca, cb;
+    block_suffix_scan_d2(ta, tb, tmpa, tmpb, ca, cb);
+    // Walk the run from its end toward its start, accumulating onto the carry.
+    int best = nc;
+    double sa = ca, sb2 = cb;
+    for (int r = r1 - 1; r >= r0; --r) {
+      const int id = (int)(keys[r] & 0xffffffffu);
+      sa += (double)Ih[id];
+      sb2 += (double)mh[id];
+      if (sb2 < 1.0 && sa <= p.tau * (1.0 - sb2)) best = r;
+    }
+    if (best < nc) atomicMin(&s_kcut, best);
+    __syncthreads();
+    kcut = s_kcut;
+  }
+  // Mark kept blocks: mandatory + top kcut candidates.
+  for (int r = threadIdx.x; r < kcut; r += blockDim.x) keep[(int)(keys[r] & 0xffffffffu)] = 1;
+  if (threadIdx.x == 0) {
+    keep[0] = 1;
+    keep[i] = 1;
+    if (i >= 1) keep[i - 1] = 1;
+  }
+  __syncthreads();
+  // Ascending compaction over block ids 0..i.
+  const int n = i + 1;
+  const int E2 = (n + kSelThreads - 1) / kSelThreads;
+  const int b0 = threadIdx.x * E2;
+  const int b1 = min(n, b0 + E2);
+  int cnt = 0;
+  for (int b = b0; b < b1; ++b) cnt += keep[b];
+  int total;
+  int pos = block_excl_scan_int(cnt, tmpi, &total);
+  int32_t* dst = p.scratch + off;
+  for (int b = b0; b < b1; ++b)
+    if (keep[b]) dst[pos++] = b;
+  if (threadIdx.x == 0) p.counts[row] = total;
+}
+
+// Exclusive scan of counts[0..rows) into row_ptr[0..rows] (single CTA).
+__global__ void __launch_bounds__(1024) scan_counts_kernel(const int32_t* counts, int32_t* row_ptr, int rows) {
+  __shared__ int warp_tot[32];
+  __shared__ int carry;
+  if (threadIdx.x == 0) carry = 0;
+  __syncthreads();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int base = 0; base < rows; base += 1024) {
+    const int idx = base + threadIdx.x;
+    const int v = (idx < rows) ? counts[idx] : 0;
+    int x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (lane == 31) warp_tot[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+      int w = warp_tot[lane];
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, w, o);
+        if (lane >= o) w += y;
+      }
+      warp_tot[lane] = w;
+    }
+    __syncthreads();
+    const int excl = carry + ((warp > 0) ? warp_tot[warp - 1] : 0) + x - v;
+    if (idx < rows) row_ptr[idx] = excl;
+    __syncthreads();
+    if (threadIdx.x == 0) carry += warp_tot[31];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) row_ptr[rows] = carry;
+}
+
+__global__ void __launch_bounds__(128) gather_lists_kernel(const SelectParams p) {
+  const int row = blockIdx.x;
+  const int T = p.n_tiles;
+  const int h = row / T;
+  const int i = row - h * T;
+  const int64_t start = p.row_ptr[row];
+  const int n = p.counts[row];
+  const int32_t* src = p.scratch + tri_off(T, h, i);
+  const int64_t cap = p.col_capacity;
+  for (int x = threadIdx.x; x < n; x += blockDim.x) {
+    const int64_t d = start + x;
+    if (d < cap) p.col_idx[d] = src[x];
+  }
+  if (threadIdx.x == 0 && start + n > cap) raise_err(p.err, kErrCapacity);
+}
+
+// Rows of one KV head's query-head group, by list length descending, ties by row id.
+__global__ void __launch_bounds__(1024) work_order_kernel(const SelectParams p, int seg_pow2) {
+  extern __shared__ __align__(16) uint8_t sm[];
+  uint32_t* keys = reinterpret_cast<uint32_t*>(sm);
+  const int seg = p.group * p.n_tiles;
+  const int base = blockIdx.x * seg;
+  for (int t = threadIdx.x; t < seg_pow2; t += blockDim.x) {
+    uint32_t key = 0xffffffffu;
+    if (t < seg) {
+      const int len = min(p.row_ptr[base + t + 1] - p.row_ptr[base + t], 4095);
+      key = ((uint32_t)(4095 - len) << 20) | (uint32_t)t;
+    }
+    keys[t] = key;
+  }
+  __syncthreads();
+  bitonic_sort_u32(keys, seg_pow2);
+  for (int t = threadIdx.x; t < seg; t += blockDim.x) p.order[base + t] = base + (int)(keys[t] & 0xfffffu);
+}
+
+}  // namespace
+
+cudaError_t launch_select(const SelectParams& p, cudaStream_t stream) {
+  const int rows = p.n_q_heads * p.n_tiles;
+  if (rows <= 0) return cudaSuccess;
+  int P = 1;
+  while (P < p.n_tiles) P <<= 1;
+  const size_t smem = sizeof(uint64_t) * (size_t)P + sizeof(int) * (size_t)p.n_tiles + 16;
+  static size_t configured = 0;
+  if (smem > 48 * 1024 && smem > configured) {
+    cudaError_t e = cudaFuncSetAttribute(select_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    configured = smem;
+  }
+  select_rows_kernel<<<rows, kSelThreads, smem, stream>>>(p);
+  scan_counts_kernel<<<1, 1024, 0, stream>>>(p.counts, p.row_ptr, rows);
+  gather_lists_kernel<<<rows, 128, 0, stream>>>(p);
+  if (p.order) {
+    const int seg = p.group * p.n_tiles;
+    int sp = 1;
+    while (sp < seg) sp <<= 1;
+    const size_t osmem = sizeof(uint32_t) * (size_t)sp;
+    static size_t oconf = 0;
+    if (osmem > 48 * 1024 && osmem > oconf) {
+      cudaError_t e = cudaFuncSetAttribute(work_order_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)osmem);
+      if (e != cudaSuccess) return e;
+      oconf = osmem;
+    }
+    work_order_kernel<<<p.n_q_heads / p.group, 1024, osmem, stream>>>(p, sp);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace poem

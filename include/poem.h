@@ -1,0 +1,181 @@
+/*
+ * poem.h -- C ABI of libpoem, a B200 (sm_100a) implementation of the hot path of
+ * POEM-style output-relative block-sparse attention prefill.
+ *
+ * The method (Wu et al., "POEM: Output-Relative Block-Sparse Attention for
+ * Long-Context Prefilling", as summarised in the reading note "Attention
+ * deletion error", Section 4.1 and Equations (3)-(4)): for one query and one
+ * head, a visible key block b has softmax mass m_b and attention-weighted mean
+ * value v_b; the dense output is o = sum_b m_b v_b; dropping a set D of blocks
+ * with mass delta < 1 gives o~ = (o - sum_D m_b v_b) / (1 - delta), and
+ *     || o - o~ || <= sum_{b in D} I_b / (1 - delta),   I_b = m_b || v_b - o ||.
+ *
+ * Three calls form one prefill layer, all asynchronous on the caller's stream:
+ *   poem_score   exact m_b and I_b on a strided subset of the queries of each
+ *                query tile, max-aggregated per (head, tile, visible block)
+ *   poem_select  mandatory blocks + blocks in descending I_b until the bound
+ *                above is <= tau; CSR block list per (head, tile)
+ *   bsa_fwd      causal GQA block-sparse attention over the listed blocks
+ *
+ * Conventions for every entry point
+ *   - All pointers are device pointers unless stated, 16-byte aligned.  The
+ *     caller owns every buffer; the library never allocates device memory and
+ *     never synchronises a stream (poem_check excepted).
+ *   - q, k, v, o hold bf16 values (poem_bf16 = raw bf16 bits); the head
+ *     dimension is contiguous; token and head strides are given in elements
+ *     and must be multiples of 8 (16 bytes).
+ *   - Each call validates its arguments on the host before any launch and
+ *     returns POEM_ERR_INVALID_ARG / POEM_ERR_UNSUPPORTED without launching.
+ *   - Conditions found on the device (a bounded wait that gave up, a block id
+ *     outside the causal range, a col_idx buffer that is too small) are OR-ed
+ *     into an error word at the start of the call's workspace; poem_check
+ *     reads and clears it.  Workspaces must be zero-filled once before first
+ *     use (the library keeps the error word clear otherwise).
+ *   - Supported in this version: head_dim in {64, 128}, block in {64, 128},
+ *     n_sample in {16} dividing block, n_tokens % block == 0,
+ *     n_q_heads % n_kv_heads == 0.  Anything else: POEM_ERR_UNSUPPORTED.
+ *   - There is no CPU fallback and no other backend.
+ */
+#ifndef POEM_H
+#define POEM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t poem_bf16; /* raw bfloat16 bit pattern */
+
+typedef enum poem_status {
+  POEM_OK = 0,
+  POEM_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size, tau < 0 or NaN ...   */
+  POEM_ERR_UNSUPPORTED = 2, /* valid but not implemented (head_dim, block, n_sample)    */
+  POEM_ERR_CUDA = 3,        /* a CUDA runtime/driver call failed; see poem_last_error  */
+  POEM_ERR_TIMEOUT = 4,     /* device: a bounded wait gave up (reported by poem_check)  */
+  POEM_ERR_CAPACITY = 5,    /* col_capacity too small (device: reported by poem_check)  */
+  POEM_ERR_WORKSPACE = 6,   /* ws_bytes smaller than poem_workspace_size reports        */
+  POEM_ERR_BAD_LIST = 7     /* device: a listed block id outside 0..tile (skipped)      */
+} poem_status;
+
+/*
+ * Problem shape of one attention layer.
+ *   q: [n_tokens, n_q_heads, head_dim], element (t, h, c) at
+ *      q[t*q_stride_tok + h*q_stride_head + c]; k, v: [n_tokens, n_kv_heads,
+ *      head_dim] with kv_stride_*; o like q with o_stride_*.
+ *   Query head h reads KV head h / (n_q_heads / n_kv_heads) (GQA).
+ *   block: key block size = query tile size B; T = n_tokens / B tiles; tile i
+ *      holds queries iB..iB+B-1 and sees key blocks 0..i (causal).
+ *   n_sample: S sampled queries per tile for scoring, rows iB + j*(B/S).
+ *   softmax_scale: logit scale; 0 selects 1/sqrt(head_dim).
+ */
+typedef struct poem_shape {
+  int32_t n_tokens;
+  int32_t n_q_heads;
+  int32_t n_kv_heads;
+  int32_t head_dim;
+  int32_t block;
+  int32_t n_sample;
+  float softmax_scale;
+  int32_t reserved0;
+  int64_t q_stride_tok, q_stride_head;
+  int64_t kv_stride_tok, kv_stride_head;
+  int64_t o_stride_tok, o_stride_head;
+} poem_shape;
+
+/*
+ * Workspace bytes each call needs for this shape (any output pointer may be
+ * NULL).  Every workspace starts with a 256-byte header holding the error word.
+ */
+poem_status poem_workspace_size(const poem_shape* shape, size_t* score_bytes, size_t* select_bytes,
+                                size_t* fwd_bytes);
+
+/*
+ * poem_score -- exact block scores on the sampled queries.
+ * Section 4.1 (m_b, v_b, o) and Equation (4) (I_b = m_b ||v_b - o||) of the
+ * reading note; sampling (S strided queries per tile) and max-aggregation are
+ * the hot-path contract's choices.
+ * For each query head h, tile i and visible block b <= i:
+ *   I_hat[h, i, b] = max_j I_b(q_j),  m_hat[h, i, b] = max_j m_b(q_j)
+ * over the sampled queries q_j = iB + j*(B/S), j = 0..S-1, with dense causal
+ * softmax attention of q_j over keys 0..q_j.
+ * Outputs (fp32, packed lower-triangular): entry (h, i, b) at
+ *   h*T*(T+1)/2 + i*(i+1)/2 + b; n_q_heads*T*(T+1)/2 entries each.
+ * ws: at least score_bytes (holds per-sampled-query dense outputs and
+ *   log-sum-exps between the two passes).
+ */
+poem_status poem_score(const poem_shape* shape, const poem_bf16* q, const poem_bf16* k, const poem_bf16* v,
+                       float* I_hat, float* m_hat, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * poem_select -- threshold selection per (head, tile), Equation (4).
+ * Row r = h*T + i.  Mandatory: sink block 0, local block i-1 (i >= 1) and the
+ * diagonal block i.  Candidates 1..i-2 are ranked by (I_hat desc, id asc) --
+ * equal scores favour the smaller id, the convention of the "Block-Filtered
+ * Long-Context Attention" page, Appendix "Block ordering".  With D_k the
+ * candidates ranked k, k+1, ..., S_I = sum_{D_k} I_hat and S_m = sum_{D_k}
+ * m_hat (fp64), the row keeps the top k for the smallest k with
+ *     S_m < 1  and  S_I <= tau * (1 - S_m).
+ * Outputs: row_ptr[n_q_heads*T + 1] (int32, exclusive scan of list lengths)
+ *   and col_idx[row_ptr[r] .. row_ptr[r+1]) the kept ids of row r in
+ *   ascending order.  col_capacity: entries available in col_idx; when the
+ *   lists need more, col_idx holds a truncated prefix and POEM_ERR_CAPACITY is
+ *   reported by poem_check (n_q_heads*T*(T+1)/2 always suffices).
+ * order (nullable): int32[n_q_heads*T], a work order for bsa_fwd -- rows grouped
+ *   by KV head, longest list first, ties by row id.
+ * tau: absolute bound on the per-query head-output error in V's units; must be
+ *   finite and >= 0 (tau = 0 keeps every candidate with I_hat > 0).
+ */
+poem_status poem_select(const poem_shape* shape, const float* I_hat, const float* m_hat, float tau,
+                        int32_t* row_ptr, int32_t* col_idx, int64_t col_capacity, int32_t* order, void* ws,
+                        size_t ws_bytes, void* stream);
+
+/*
+ * poem_select_mass_only -- the mass-only baseline at a matched budget: row r
+ * keeps the mandatory blocks and the (ref_row_ptr[r+1] - ref_row_ptr[r] -
+ * |mandatory|) candidates of largest m_hat (ties: smaller id).  Same outputs
+ * and workspace as poem_select.  ref_row_ptr is a device pointer.
+ */
+poem_status poem_select_mass_only(const poem_shape* shape, const float* m_hat, const int32_t* ref_row_ptr,
+                                  int32_t* row_ptr, int32_t* col_idx, int64_t col_capacity, int32_t* order,
+                                  void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * bsa_fwd -- causal GQA block-sparse attention forward.
+ * Query t of head h in tile i attends, with softmax, to the keys u <= t whose
+ * block is listed in col_idx[row_ptr[r] .. row_ptr[r+1]), r = h*T + i
+ * (the renormalised output o~ of Section 4.1).  Lists must be ascending and
+ * hold ids in 0..i; an id outside that range is skipped and reported as
+ * POEM_ERR_BAD_LIST by poem_check.  A row with no visible key outputs 0 and
+ * lse = -inf.
+ * o: bf16 output with o_stride_*; lse (nullable): fp32 [n_q_heads, n_tokens],
+ *   natural-log log-sum-exp of the scaled logits over the kept keys.
+ * order (nullable): permutation of the rows giving the launch order; NULL
+ *   selects KV-head-major, last tile first.
+ */
+poem_status bsa_fwd(const poem_shape* shape, const poem_bf16* q, const poem_bf16* k, const poem_bf16* v,
+                    const int32_t* row_ptr, const int32_t* col_idx, const int32_t* order, poem_bf16* o,
+                    float* lse, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Synchronise `stream`, read and clear the error word at the start of `ws`
+ * (a workspace passed to one of the calls above) and map it to a status:
+ * POEM_ERR_TIMEOUT, POEM_ERR_BAD_LIST, POEM_ERR_CAPACITY, or POEM_OK.
+ */
+poem_status poem_check(void* stream, void* ws);
+
+/* Upper bound, in nanoseconds, of every on-device wait (default 2e9).  A
+ * process-wide setting read at launch time. */
+void poem_set_wait_limit_ns(uint64_t ns);
+
+const char* poem_status_string(poem_status s);
+
+/* Text of the last CUDA error seen by this thread (empty if none). */
+const char* poem_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* POEM_H */

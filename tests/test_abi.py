@@ -1,0 +1,116 @@
+"""The C-ABI library loads and exports every entry point of include/poem.h, and
+the host-side argument checks reject bad calls before any device work.  These
+tests make no CUDA call and need no GPU."""
+import ctypes
+import math
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "poem.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\*?\s*([a-z_][a-z0-9_]*)\s*\(", src, flags=re.M)
+    return sorted(set(names))
+
+
+@pytest.fixture(scope="module")
+def poem():
+    from block_sparse_attention_poem_b200 import build
+
+    build.build()
+    import block_sparse_attention_poem_b200 as m
+
+    return m
+
+
+def test_header_declares_the_entry_points():
+    names = _declared()
+    for n in ("poem_workspace_size", "poem_score", "poem_select", "poem_select_mass_only", "bsa_fwd",
+              "poem_check", "poem_set_wait_limit_ns", "poem_status_string", "poem_last_error"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(poem):
+    lib = ctypes.CDLL(poem.LIB_PATH)
+    for name in _declared():
+        assert hasattr(lib, name), name
+    assert set(_declared()) <= set(poem.EXPORTED)
+
+
+def _shape(poem, **kw):
+    base = dict(n_tokens=1024, n_q_heads=4, n_kv_heads=2, head_dim=128, block=128, n_sample=16, softmax_scale=0.0,
+                reserved0=0, q_stride_tok=512, q_stride_head=128, kv_stride_tok=256, kv_stride_head=128,
+                o_stride_tok=512, o_stride_head=128)
+    base.update(kw)
+    return poem.Shape(**base)
+
+
+def _ws(poem, shape):
+    a, b, c = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
+    st = poem._lib.poem_workspace_size(ctypes.byref(shape), ctypes.byref(a), ctypes.byref(b), ctypes.byref(c))
+    return st, a.value, b.value, c.value
+
+
+def test_workspace_sizes(poem):
+    st, s, sel, f = _ws(poem, _shape(poem))
+    assert st == 0
+    T, hq = 8, 4
+    assert s >= 256 + hq * T * 16 * 128 * 4 + hq * T * 16 * 4
+    assert sel >= 256 + hq * T * 4 + hq * T * (T + 1) // 2 * 4
+    assert f >= 256
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(n_tokens=1000), 1),            # N % block
+    (dict(n_q_heads=3), 1),              # Hq % Hkv
+    (dict(n_tokens=0), 1),
+    (dict(head_dim=96), 2),
+    (dict(block=32), 2),
+    (dict(q_stride_tok=500), 1),         # not a multiple of 8 elements
+    (dict(softmax_scale=float("nan")), 1),
+    (dict(softmax_scale=-1.0), 1),
+])
+def test_shape_validation(poem, kw, status):
+    st, *_ = _ws(poem, _shape(poem, **kw))
+    assert st == status, poem.poem_status_string(st)
+
+
+def test_null_and_misaligned_pointers_rejected(poem):
+    sh = _shape(poem)
+    ok = ctypes.c_void_p(1 << 20)
+    mis = ctypes.c_void_p((1 << 20) + 8)
+    st = poem._lib.bsa_fwd(ctypes.byref(sh), None, ok, ok, ok, ok, None, ok, None, ok, 4096, None)
+    assert st == 1
+    st = poem._lib.bsa_fwd(ctypes.byref(sh), mis, ok, ok, ok, ok, None, ok, None, ok, 4096, None)
+    assert st == 1
+    st = poem._lib.poem_score(ctypes.byref(sh), ok, ok, ok, ok, ok, ok, 16, None)
+    assert st == 6  # workspace too small
+    st = poem._lib.poem_score(ctypes.byref(_shape(poem, n_sample=8)), ok, ok, ok, ok, ok, ok, 1 << 30, None)
+    assert st == 2
+    assert "16-byte" in poem.poem_last_error() or "n_sample" in poem.poem_last_error()
+
+
+@pytest.mark.parametrize("tau", [-0.1, float("nan"), float("inf")])
+def test_select_rejects_bad_tau(poem, tau):
+    sh = _shape(poem)
+    ok = ctypes.c_void_p(1 << 20)
+    st = poem._lib.poem_select(ctypes.byref(sh), ok, ok, ctypes.c_float(tau), ok, ok, 100, None, ok, 1 << 30, None)
+    assert st == 1
+
+
+def test_select_rejects_small_workspace_and_negative_capacity(poem):
+    sh = _shape(poem)
+    ok = ctypes.c_void_p(1 << 20)
+    assert poem._lib.poem_select(ctypes.byref(sh), ok, ok, ctypes.c_float(0.05), ok, ok, 100, None, ok, 8, None) == 6
+    assert poem._lib.poem_select(ctypes.byref(sh), ok, ok, ctypes.c_float(0.05), ok, ok, -1, None, ok, 1 << 30,
+                                 None) == 1
+
+
+def test_status_strings(poem):
+    for code, name in poem.STATUS.items():
+        assert poem.poem_status_string(code) == name
