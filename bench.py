@@ -212,6 +212,10 @@ def run_ours(args):
     ci = layer.col_idx[: int(rp[-1])].cpu().numpy()
     kept = int(rp[-1])
     visible = hq * T * (T + 1) // 2
+    # realised heavy-mass fraction: visible (head, tile, block) with m_hat > 10 / (i + 1)
+    mh = layer.m_hat.cpu().numpy()
+    tile_of = np.tile(np.repeat(np.arange(T), np.arange(1, T + 1)), hq)
+    heavy_frac = float(np.mean(mh > 10.0 / (tile_of + 1)))
     rflops = retained_flops(rp, ci, T, d, B)
     dflops = dense_flops(n, hq, d)
     peaks, peak_src = load_peaks()
@@ -279,6 +283,7 @@ def run_ours(args):
         "breakdown_ms": {"poem_score": round(score_ms, 4), "poem_select": round(select_ms, 4),
                          "bsa_fwd": round(fwd_ms, 4)},
         "density": round(kept / visible, 5),
+        "heavy_mass_block_fraction": round(heavy_frac, 4),
         "dense_equiv_tflops": round(dflops / (ms_per_step * 1e-3) / 1e12, 2),
         "retained_tflops": round(rflops / (ms_per_step * 1e-3) / 1e12, 2),
         "score_select_over_fwd": round((score_ms + select_ms) / fwd_ms, 4),

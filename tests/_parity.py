@@ -43,17 +43,24 @@ def compare_fwd(o_gpu: torch.Tensor, O_ref: np.ndarray, units, block: int):
     return float(e.max()), float(e.mean())
 
 
-def score_rel_err(gpu: np.ndarray, ref: np.ndarray, n_q_heads: int, n_tiles: int):
-    """Max relative error of packed scores, floored at 1e-3 of each row's max."""
-    worst = 0.0
-    for h in range(n_q_heads):
-        for i in range(n_tiles):
-            off = oracle.tri_offset(n_tiles, h, i)
-            r = ref[off:off + i + 1]
-            g = gpu[off:off + i + 1]
-            floor = 1e-3 * max(float(r.max()), 1e-30)
-            worst = max(worst, float(np.max(np.abs(g - r) / np.maximum(r, floor))))
-    return worst
+def score_err_excess(gpu_I, ref_I, gpu_m, ref_m, R: float):
+    """Largest violation ratio of the score tolerances (<= 1 passes):
+      |dI_b| <= SCORE_REL * I_b + 1e-5 * m_b * R
+      |dm_b| <= SCORE_REL * m_b + 1e-9
+    where R = max_t ||v_t||.  The absolute terms cover exact cancellation (e.g. the
+    single visible block of tile 0, where v_b = o and I_b = 0): r_b = P_b V_b - m_b o
+    is formed in fp32 from P split into bf16 hi/lo (about 2^-17 relative per weight),
+    leaving ~2^-17 m_b R absolute error; masses below ~1e-9 sit at the fp32
+    flush-to-zero limit of the exponential."""
+    gI, rI = np.asarray(gpu_I, np.float64), np.asarray(ref_I, np.float64)
+    gm, rm = np.asarray(gpu_m, np.float64), np.asarray(ref_m, np.float64)
+    tolI = SCORE_REL * rI + 1e-5 * rm * R + 1e-30
+    tolm = SCORE_REL * rm + 1e-9
+    return float(max(np.max(np.abs(gI - rI) / tolI), np.max(np.abs(gm - rm) / tolm)))
+
+
+def max_value_norm(v: torch.Tensor) -> float:
+    return float(v.float().norm(dim=-1).max())
 
 
 def lists_agree_at_cut(gpu_rows, ref_rows, Ihat_ref, mhat_ref, n_q_heads, n_tiles, tau):
