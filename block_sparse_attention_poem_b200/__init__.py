@@ -34,7 +34,7 @@ STATUS = {
 
 EXPORTED = (
     "poem_workspace_size", "poem_score", "poem_select", "poem_select_mass_only", "bsa_fwd",
-    "poem_check", "poem_set_wait_limit_ns", "poem_status_string", "poem_last_error",
+    "poem_check", "poem_set_wait_limit_ns", "poem_status_string", "poem_last_error", "poem_select_noalloc",
 )
 
 
@@ -69,6 +69,8 @@ def _load():
     lib.poem_select.restype = st
     lib.poem_select_mass_only.argtypes = [sp, vp, vp, vp, vp, i64, vp, vp, sz, vp]
     lib.poem_select_mass_only.restype = st
+    lib.poem_select_noalloc.argtypes = [sp, vp, vp, ctypes.c_float, vp, vp, i64, vp, vp]
+    lib.poem_select_noalloc.restype = st
     lib.bsa_fwd.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.bsa_fwd.restype = st
     lib.poem_check.argtypes = [vp, vp]
@@ -152,6 +154,16 @@ def poem_select_mass_only(shape: Shape, m_hat, ref_row_ptr, row_ptr, col_idx, ws
     _raise(_lib.poem_select_mass_only(ctypes.byref(shape), _ptr(m_hat), _ptr(ref_row_ptr), _ptr(row_ptr),
                                       _ptr(col_idx), col_idx.numel(), _ptr(order), _ptr(ws),
                                       ws.numel() * ws.element_size(), _stream(stream)), "poem_select_mass_only")
+
+
+def poem_select_noalloc(shape: Shape, I_hat, m_hat, tau: float, row_ptr, col_idx, order=None, stream=None):
+    """poem_select without a workspace, for callers that cannot allocate device
+    memory: the scratch is a fixed 8 MiB array inside the library (shared by all
+    calls -- do not overlap calls on the GPU).  Check row_ptr[-1] against
+    col_idx.numel() afterwards; there is no error word to poll."""
+    _raise(_lib.poem_select_noalloc(ctypes.byref(shape), _ptr(I_hat), _ptr(m_hat), ctypes.c_float(tau),
+                                    _ptr(row_ptr), _ptr(col_idx), col_idx.numel(), _ptr(order), _stream(stream)),
+           "poem_select_noalloc")
 
 
 def bsa_fwd(q, k, v, row_ptr, col_idx, o, ws, lse=None, order=None, shape: Shape | None = None, stream=None,

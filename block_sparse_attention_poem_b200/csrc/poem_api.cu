@@ -131,6 +131,10 @@ poem::DevErr dev_err(void* ws) { return poem::DevErr{reinterpret_cast<uint32_t*>
 
 }  // namespace
 
+namespace poem {
+void set_last_error(const char* msg) { std::snprintf(g_last_error, sizeof g_last_error, "%s", msg); }
+}  // namespace poem
+
 extern "C" {
 
 poem_status poem_workspace_size(const poem_shape* shape, size_t* score_bytes, size_t* select_bytes,

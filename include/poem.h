@@ -142,6 +142,30 @@ poem_status poem_select_mass_only(const poem_shape* shape, const float* m_hat, c
                                   void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * poem_select_noalloc -- poem_select for callers that cannot allocate device
+ * memory.  (An addition of this library; the method description has no
+ * counterpart.)  Some callers own no allocator: a serving runtime that reserves
+ * all device memory up front and must not let a library grow its footprint while
+ * it serves, or a plug-in that is only handed pointers by its host.  This entry
+ * point takes the same inputs and outputs as poem_select but no workspace: its
+ * scratch lives in a fixed 8 MiB array inside the library's device image, which
+ * every GPU that loads the library holds until the process exits.  It calls no
+ * allocator of any kind.
+ *   - Shapes whose selection scratch (poem_workspace_size's select_bytes) exceeds
+ *     8 MiB are rejected with POEM_ERR_WORKSPACE and a message in poem_last_error
+ *     (e.g. 32 heads x 256 tiles fits; 32 heads x 1024 tiles does not).
+ *   - All calls share the array and each call overwrites it: calls whose kernels
+ *     overlap on the GPU (other streams, other host threads) race; serialise them.
+ *   - The first call on a device resolves the array's device address with that
+ *     device current; make that first call before any stream capture.
+ *   - There is no workspace error word to poll: a col_idx that is too small is
+ *     seen by comparing row_ptr[n_q_heads*T] with col_capacity after the call.
+ */
+poem_status poem_select_noalloc(const poem_shape* shape, const float* I_hat, const float* m_hat, float tau,
+                                int32_t* row_ptr, int32_t* col_idx, int64_t col_capacity, int32_t* order,
+                                void* stream);
+
+/*
  * bsa_fwd -- causal GQA block-sparse attention forward.
  * Query t of head h in tile i attends, with softmax, to the keys u <= t whose
  * block is listed in col_idx[row_ptr[r] .. row_ptr[r+1]), r = h*T + i
