@@ -67,6 +67,54 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, Fw
 
 constexpr uint64_t kDrainNs = 2000000000ull;  // waits for already-issued async work
 
+// Exponentials of one S row (re-read from TMEM in 64-column halves), the bf16 P
+// written over the first BN/2 TMEM columns of S, and the row sum added to *l.  One pair in kPolyEvery is evaluated on the FMA pipe (exp2_pair_poly) to
+// unload MUFU; the diagonal block (masked columns already -inf) uses MUFU only,
+// so masked weights are exactly zero.
+constexpr int kPolyEvery = 4;
+
+template <int BN, bool DIAG>
+__device__ __forceinline__ void exp_pack_store(uint32_t tS, float sl2, float m_use, int lim, float* l) {
+  const uint64_t scale2 = f2_pack(sl2, sl2);
+  const uint64_t negm2 = f2_pack(-m_use, -m_use);
+  uint64_t acc = f2_pack(0.f, 0.f);
+#pragma unroll
+  for (int hf = 0; hf < BN / 64; ++hf) {
+    // re-read 64 S columns; the P words of this half go to columns [32 hf, 32 hf + 32),
+    // which hold S values already read
+    uint32_t a[2][32];
+    tmem_ld32(tS + hf * 64, a[0]);
+    tmem_ld32(tS + hf * 64 + 32, a[1]);
+    tmem_ld_wait();
+    tmem_reg_fence(a[0]);
+    tmem_reg_fence(a[1]);
+    uint32_t packed[32];
+#pragma unroll
+    for (int x = 0; x < 32; ++x) {
+      const uint32_t* src = a[x >> 4];
+      const int k = (2 * x) & 31;
+      const uint64_t xv = f2_fma(f2_pack(__uint_as_float(src[k]), __uint_as_float(src[k + 1])), scale2, negm2);
+      float x0, x1, y0, y1;
+      f2_unpack(xv, x0, x1);
+      if (DIAG) {
+        y0 = (hf * 64 + 2 * x <= lim) ? ex2_approx(x0) : 0.f;
+        y1 = (hf * 64 + 2 * x + 1 <= lim) ? ex2_approx(x1) : 0.f;
+      } else if ((x % kPolyEvery) == kPolyEvery - 1) {
+        exp2_pair_poly(x0, x1, y0, y1);
+      } else {
+        y0 = ex2_approx(x0);
+        y1 = ex2_approx(x1);
+      }
+      acc = f2_add(acc, f2_pack(y0, y1));
+      packed[x] = pack_bf16x2(y0, y1);
+    }
+    tmem_st32(tS + hf * 32, packed);
+  }
+  float a0, a1;
+  f2_unpack(acc, a0, a1);
+  *l += a0 + a1;
+}
+
 template <int D, int BN>
 __global__ void __launch_bounds__(kThreadsFwd, 2)
     bsa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -218,73 +266,74 @@ __global__ void __launch_bounds__(kThreadsFwd, 2)
     const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
     const uint32_t tS = lane_base + C::kColS;
     const uint32_t tO = lane_base + C::kColO;
+    const float sl2 = p.scale_log2;
     float m_run = -INFINITY;                 // running max, log2 units of scaled logits
-    float l_run = 0.f;                       // running sum of (bf16-rounded) weights
+    float l_run = 0.f;                       // running sum of the weights
     int it = 0;
     bool ok = true;
+    int id = (beg < end) ? p.col_idx[beg] : -1;
     for (int e = beg; e < end; ++e) {
-      const int id = p.col_idx[e];
-      if (!block_ok(id, tile)) continue;
-      // tcgen05.ld is warp-collective: every lane of the warp takes the same branch.
-      if (!__all_sync(0xffffffffu, wait_or_abort(&sb->s_full, it & 1, sb, p.err))) { ok = false; break; }
-      tc_fence_after();
-      float s[BN];
+      const int id_next = (e + 1 < end) ? p.col_idx[e + 1] : -1;  // prefetched a block ahead
+      if (block_ok(id, tile)) {
+        // tcgen05.ld is warp-collective: every lane of the warp takes the same branch.
+        if (!__all_sync(0xffffffffu, wait_or_abort(&sb->s_full, it & 1, sb, p.err))) { ok = false; break; }
+        tc_fence_after();
+        const bool diag = (id == tile);
+        const int lim = qpos - id * BN;  // on the diagonal block, columns <= lim are visible
+        // row max of S_j (all column chunks, one wait)
+        float mx = -INFINITY;
+        {
+          uint32_t sv[BN / 32][32];
 #pragma unroll
-      for (int c = 0; c < BN / 32; ++c) {
-        uint32_t raw[32];
-        tmem_ld32(tS + c * 32, raw);
-        tmem_ld_wait();
-#pragma unroll
-        for (int x = 0; x < 32; ++x) s[c * 32 + x] = __uint_as_float(raw[x]);
-      }
-      if (id == tile) {
-        const int lim = qpos - id * BN;      // keys with column <= lim are visible
-#pragma unroll
-        for (int c = 0; c < BN; ++c)
-          if (c > lim) s[c] = -INFINITY;
-      }
-      float mx = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < BN; ++c) mx = fmaxf(mx, s[c]);
-      const float m_new = fmaxf(m_run, mx * p.scale_log2);
-      const bool grow = (m_new > m_run + 8.0f);
-      float alpha = 1.f;
-      if (grow) {
-        alpha = (m_run == -INFINITY) ? 0.f : ex2_approx(m_run - m_new);
-        m_run = m_new;
-      }
-      // O must be rescaled when this row's reference max moved (S_j complete implies
-      // the previous P V_{j-1} is complete: the MMAs run in issue order).
-      if (it > 0 && __any_sync(0xffffffffu, grow)) {
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t raw[32];
-          tmem_ld32(tO + c * 32, raw);
+          for (int c = 0; c < BN / 32; ++c) tmem_ld32(tS + c * 32, sv[c]);
           tmem_ld_wait();
 #pragma unroll
-          for (int x = 0; x < 32; ++x) raw[x] = __float_as_uint(__uint_as_float(raw[x]) * alpha);
-          tmem_st32(tO + c * 32, raw);
-        }
-      }
-      l_run *= alpha;
-      const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
+          for (int c = 0; c < BN / 32; ++c) tmem_reg_fence(sv[c]);
+          if (diag) {  // uniform branch
 #pragma unroll
-      for (int c = 0; c < BN / 64; ++c) {
-        uint32_t packed[32];
+            for (int c = 0; c < BN / 32; ++c)
 #pragma unroll
-        for (int x = 0; x < 32; ++x) {
-          const float p0 = ex2_approx(fmaf(s[c * 64 + 2 * x], p.scale_log2, -m_use));
-          const float p1 = ex2_approx(fmaf(s[c * 64 + 2 * x + 1], p.scale_log2, -m_use));
-          const uint32_t w = pack_bf16x2(p0, p1);
-          l_run += bf16lo_to_f32(w) + bf16hi_to_f32(w);
-          packed[x] = w;
+              for (int x = 0; x < 32; ++x) mx = fmaxf(mx, (c * 32 + x <= lim) ? __uint_as_float(sv[c][x]) : -INFINITY);
+          } else {
+#pragma unroll
+            for (int c = 0; c < BN / 32; ++c)
+#pragma unroll
+              for (int x = 0; x < 32; x += 2) mx = fmax3(mx, __uint_as_float(sv[c][x]), __uint_as_float(sv[c][x + 1]));
+          }
         }
-        tmem_st32(tS + c * 32, packed);
+        const float m_new = fmaxf(m_run, mx * sl2);
+        const bool grow = (m_new > m_run + 8.0f);
+        float alpha = 1.f;
+        if (grow) {
+          alpha = (m_run == -INFINITY) ? 0.f : ex2_approx(m_run - m_new);
+          m_run = m_new;
+        }
+        // O must be rescaled when this row's reference max moved (S_j complete implies
+        // the previous P V_{j-1} is complete: the MMAs run in issue order).
+        if (it > 0 && __any_sync(0xffffffffu, grow)) {
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t ov[32];
+            tmem_ld32(tO + c * 32, ov);
+            tmem_ld_wait();
+            tmem_reg_fence(ov);
+#pragma unroll
+            for (int x = 0; x < 32; ++x) ov[x] = __float_as_uint(__uint_as_float(ov[x]) * alpha);
+            tmem_st32(tO + c * 32, ov);
+          }
+        }
+        l_run *= alpha;
+        const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
+        if (diag)
+          exp_pack_store<BN, true>(tS, sl2, m_use, lim, &l_run);
+        else
+          exp_pack_store<BN, false>(tS, sl2, m_use, lim, &l_run);
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&sb->p_full);
+        ++it;
       }
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(&sb->p_full);
-      ++it;
+      id = id_next;
     }
     // ---- epilogue ----
     if (__all_sync(0xffffffffu, ok && !sb->abort_flag)) {
@@ -294,16 +343,18 @@ __global__ void __launch_bounds__(kThreadsFwd, 2)
         if (__all_sync(0xffffffffu, wait_or_abort(&sb->o_full, 0, sb, p.err))) {
           tc_fence_after();
           const float inv_l = (l_run > 0.f) ? 1.f / l_run : 0.f;
+          uint32_t ov[D / 32][32];
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) tmem_ld32(tO + c * 32, ov[c]);
+          tmem_ld_wait();
 #pragma unroll
           for (int c = 0; c < D / 32; ++c) {
-            uint32_t raw[32];
-            tmem_ld32(tO + c * 32, raw);
-            tmem_ld_wait();
+            tmem_reg_fence(ov[c]);
             if (store) {
               uint32_t w[16];
 #pragma unroll
               for (int x = 0; x < 16; ++x)
-                w[x] = pack_bf16x2(__uint_as_float(raw[2 * x]) * inv_l, __uint_as_float(raw[2 * x + 1]) * inv_l);
+                w[x] = pack_bf16x2(__uint_as_float(ov[c][2 * x]) * inv_l, __uint_as_float(ov[c][2 * x + 1]) * inv_l);
               uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
 #pragma unroll
               for (int x = 0; x < 4; ++x) dst[x] = make_uint4(w[4 * x], w[4 * x + 1], w[4 * x + 2], w[4 * x + 3]);

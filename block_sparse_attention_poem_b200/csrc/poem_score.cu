@@ -221,25 +221,28 @@ __global__ void __launch_bounds__(kThreadsFwd, 2)
     const float lse2 = (PASS == 2 && valid) ? p.ws_lse[srow] : 0.f;
     const float* orow = p.ws_o + srow * D;
     bool ok = true;
+    const float sl2 = p.scale_log2;
     for (int b = 0; b < nb; ++b) {
       if (!__all_sync(0xffffffffu, wait_or_abort(&sb->s_full, b & 1, sb, p.err))) { ok = false; break; }
       tc_fence_after();
-      float s[BN];
-#pragma unroll
-      for (int c = 0; c < BN / 32; ++c) {
-        uint32_t raw[32];
-        tmem_ld32(tS + c * 32, raw);
-        tmem_ld_wait();
-#pragma unroll
-        for (int x = 0; x < 32; ++x) s[c * 32 + x] = __uint_as_float(raw[x]);
-      }
       const int lim = qpos - b * BN;  // columns <= lim are visible to this query
       float m_use = 0.f;
       if (PASS == 1) {
+        // phase 1: row max over the visible columns (one wait for all chunks)
         float mx = -INFINITY;
+        {
+          uint32_t raw[BN / 32][32];
 #pragma unroll
-        for (int c = 0; c < BN; ++c) mx = fmaxf(mx, (c <= lim) ? s[c] : -INFINITY);
-        const float m_new = fmaxf(m_run, mx * p.scale_log2);
+          for (int c = 0; c < BN / 32; ++c) tmem_ld32(tS + c * 32, raw[c]);
+          tmem_ld_wait();
+#pragma unroll
+          for (int c = 0; c < BN / 32; ++c) {
+            tmem_reg_fence(raw[c]);
+#pragma unroll
+            for (int x = 0; x < 32; ++x) mx = fmaxf(mx, (c * 32 + x <= lim) ? __uint_as_float(raw[c][x]) : -INFINITY);
+          }
+        }
+        const float m_new = fmaxf(m_run, mx * sl2);
         const bool grow = (m_new > m_run + 8.0f);
         float alpha = 1.f;
         if (grow) {
@@ -247,14 +250,16 @@ __global__ void __launch_bounds__(kThreadsFwd, 2)
           m_run = m_new;
         }
         if (b > 0 && __any_sync(0xffffffffu, grow)) {
+          uint32_t ov[D / 32][32];
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) tmem_ld32(tO + c * 32, ov[c]);
+          tmem_ld_wait();
 #pragma unroll
           for (int c = 0; c < D / 32; ++c) {
-            uint32_t raw[32];
-            tmem_ld32(tO + c * 32, raw);
-            tmem_ld_wait();
+            tmem_reg_fence(ov[c]);
 #pragma unroll
-            for (int x = 0; x < 32; ++x) raw[x] = __float_as_uint(__uint_as_float(raw[x]) * alpha);
-            tmem_st32(tO + c * 32, raw);
+            for (int x = 0; x < 32; ++x) ov[c][x] = __float_as_uint(__uint_as_float(ov[c][x]) * alpha);
+            tmem_st32(tO + c * 32, ov[c]);
           }
         }
         l_run *= alpha;
@@ -262,17 +267,25 @@ __global__ void __launch_bounds__(kThreadsFwd, 2)
       } else {
         m_use = lse2;
       }
-      // P = P_hi + P_lo; hi pairs to columns [0, BN/4) ... as bf16x2 words: P_hi at
-      // word columns [0, BN/2), P_lo at [BN/2, BN).
+      // phase 2: p (masked), split P = P_hi + P_lo in bf16.  Half hf reads S columns
+      // [64 hf, 64 hf + 64) and writes P_hi words to [32 hf, +32) and P_lo words to
+      // [BN/2 + 32 hf, +32): only S columns already read are overwritten.
       float msum = 0.f;
 #pragma unroll
-      for (int c = 0; c < BN / 64; ++c) {
+      for (int hf = 0; hf < BN / 64; ++hf) {
+        uint32_t a[2][32];
+        tmem_ld32(tS + hf * 64, a[0]);
+        tmem_ld32(tS + hf * 64 + 32, a[1]);
+        tmem_ld_wait();
+        tmem_reg_fence(a[0]);
+        tmem_reg_fence(a[1]);
         uint32_t hi[32], lo[32];
 #pragma unroll
         for (int x = 0; x < 32; ++x) {
-          const int c0 = c * 64 + 2 * x;
-          const float p0 = (c0 <= lim) ? ex2_approx(fmaf(s[c0], p.scale_log2, -m_use)) : 0.f;
-          const float p1 = (c0 + 1 <= lim) ? ex2_approx(fmaf(s[c0 + 1], p.scale_log2, -m_use)) : 0.f;
+          const int c0 = hf * 64 + 2 * x;
+          const uint32_t r0 = a[x >> 4][(2 * x) & 31], r1 = a[x >> 4][(2 * x + 1) & 31];
+          const float p0 = (c0 <= lim) ? ex2_approx(fmaf(__uint_as_float(r0), sl2, -m_use)) : 0.f;
+          const float p1 = (c0 + 1 <= lim) ? ex2_approx(fmaf(__uint_as_float(r1), sl2, -m_use)) : 0.f;
           const uint32_t wh = pack_bf16x2(p0, p1);
           const float h0 = bf16lo_to_f32(wh), h1 = bf16hi_to_f32(wh);
           const uint32_t wl = pack_bf16x2(p0 - h0, p1 - h1);
@@ -280,8 +293,41 @@ __global__ void __launch_bounds__(kThreadsFwd, 2)
           hi[x] = wh;
           lo[x] = wl;
         }
-        tmem_st32(tS + c * 32, hi);
-        tmem_st32(tS + BN / 2 + c * 32, lo);
+        // Half 1's P_hi words land in [32, 64), whose S columns half 0 already read;
+        // P_lo words land in [BN/2 + 32 hf, ...), at or past the columns being read
+        // now -- so with BN = 128 the P_lo store of half 0 waits until half 1 is read.
+        tmem_st32(tS + hf * 32, hi);
+        if (BN == 64) {
+          tmem_st32(tS + BN / 2 + hf * 32, lo);
+        } else if (hf == 0) {
+          // keep lo of half 0 until the S columns [64, 96) it overwrites are read
+#pragma unroll
+          for (int x = 0; x < 32; ++x) a[0][x] = lo[x];
+          uint32_t b2[2][32];
+          tmem_ld32(tS + 64, b2[0]);
+          tmem_ld32(tS + 96, b2[1]);
+          tmem_ld_wait();
+          tmem_reg_fence(b2[0]);
+          tmem_reg_fence(b2[1]);
+          tmem_st32(tS + BN / 2, a[0]);
+          uint32_t hi2[32], lo2[32];
+#pragma unroll
+          for (int x = 0; x < 32; ++x) {
+            const int c0 = 64 + 2 * x;
+            const uint32_t r0 = b2[x >> 4][(2 * x) & 31], r1 = b2[x >> 4][(2 * x + 1) & 31];
+            const float p0 = (c0 <= lim) ? ex2_approx(fmaf(__uint_as_float(r0), sl2, -m_use)) : 0.f;
+            const float p1 = (c0 + 1 <= lim) ? ex2_approx(fmaf(__uint_as_float(r1), sl2, -m_use)) : 0.f;
+            const uint32_t wh = pack_bf16x2(p0, p1);
+            const float h0 = bf16lo_to_f32(wh), h1 = bf16hi_to_f32(wh);
+            const uint32_t wl = pack_bf16x2(p0 - h0, p1 - h1);
+            msum += (h0 + bf16lo_to_f32(wl)) + (h1 + bf16hi_to_f32(wl));
+            hi2[x] = wh;
+            lo2[x] = wl;
+          }
+          tmem_st32(tS + 32, hi2);
+          tmem_st32(tS + BN / 2 + 32, lo2);
+          break;
+        }
       }
       if (PASS == 1) l_run += msum;
       tmem_st_wait();
@@ -292,21 +338,23 @@ __global__ void __launch_bounds__(kThreadsFwd, 2)
         // r_b = P_b V_b - m_b o ;  I_b = || r_b ||
         if (!__all_sync(0xffffffffu, wait_or_abort(&sb->o_full, b & 1, sb, p.err))) { ok = false; break; }
         tc_fence_after();
+        uint32_t pv[D / 32][32];
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) tmem_ld32(tO + c * 32, pv[c]);
+        tmem_ld_wait();
         float acc = 0.f;
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
-          uint32_t raw[32];
-          tmem_ld32(tO + c * 32, raw);
-          tmem_ld_wait();
+          tmem_reg_fence(pv[c]);
           if (valid) {
             const float4* o4 = reinterpret_cast<const float4*>(orow + c * 32);
 #pragma unroll
             for (int x = 0; x < 8; ++x) {
               const float4 ov = o4[x];
-              const float e0 = fmaf(-msum, ov.x, __uint_as_float(raw[4 * x + 0]));
-              const float e1 = fmaf(-msum, ov.y, __uint_as_float(raw[4 * x + 1]));
-              const float e2 = fmaf(-msum, ov.z, __uint_as_float(raw[4 * x + 2]));
-              const float e3 = fmaf(-msum, ov.w, __uint_as_float(raw[4 * x + 3]));
+              const float e0 = fmaf(-msum, ov.x, __uint_as_float(pv[c][4 * x + 0]));
+              const float e1 = fmaf(-msum, ov.y, __uint_as_float(pv[c][4 * x + 1]));
+              const float e2 = fmaf(-msum, ov.z, __uint_as_float(pv[c][4 * x + 2]));
+              const float e3 = fmaf(-msum, ov.w, __uint_as_float(pv[c][4 * x + 3]));
               acc = fmaf(e0, e0, fmaf(e1, e1, fmaf(e2, e2, fmaf(e3, e3, acc))));
             }
           }
@@ -330,17 +378,19 @@ __global__ void __launch_bounds__(kThreadsFwd, 2)
         tc_fence_after();
         const float inv_l = (l_run > 0.f) ? 1.f / l_run : 0.f;
         float* dst = p.ws_o + srow * D;
+        uint32_t ov[D / 32][32];
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) tmem_ld32(tO + c * 32, ov[c]);
+        tmem_ld_wait();
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
-          uint32_t raw[32];
-          tmem_ld32(tO + c * 32, raw);
-          tmem_ld_wait();
+          tmem_reg_fence(ov[c]);
           if (valid) {
             float4* d4 = reinterpret_cast<float4*>(dst + c * 32);
 #pragma unroll
             for (int x = 0; x < 8; ++x)
-              d4[x] = make_float4(__uint_as_float(raw[4 * x]) * inv_l, __uint_as_float(raw[4 * x + 1]) * inv_l,
-                                  __uint_as_float(raw[4 * x + 2]) * inv_l, __uint_as_float(raw[4 * x + 3]) * inv_l);
+              d4[x] = make_float4(__uint_as_float(ov[c][4 * x]) * inv_l, __uint_as_float(ov[c][4 * x + 1]) * inv_l,
+                                  __uint_as_float(ov[c][4 * x + 2]) * inv_l, __uint_as_float(ov[c][4 * x + 3]) * inv_l);
           }
         }
         if (valid) p.ws_lse[srow] = (l_run > 0.f) ? m_run + __log2f(l_run) : -INFINITY;
