@@ -45,7 +45,7 @@ struct ScoreCfg {
   // TMEM columns) are resident on an SM and tcgen05.alloc never has to wait.
   static constexpr int kSmemBytes = (kOffBar + 128 + 1024) > 81920 ? (kOffBar + 128 + 1024) : 81920;
   static constexpr uint32_t kTmemCols = 256;
-  static constexpr uint32_t kColS = 0;     // S (fp32) / P_hi at [0, BN/2) and P_lo at [BN/2, BN)
+  static constexpr uint32_t kColS = 0;     // S (fp32), then P_hi / P_lo interleaved per 16-key k-step
   static constexpr uint32_t kColO = 128;   // O (pass 1) or P_b V_b (pass 2)
   static constexpr uint32_t kIdescQK = idesc_bf16_f32(M, BN, 0);
   static constexpr uint32_t kIdescPV = idesc_bf16_f32(M, D, 1);
@@ -81,6 +81,52 @@ __device__ __forceinline__ void score_cta_coords(int cta, int ctas_per_g, int& g
   z0 = c * 8;
 }
 
+// p = 2^(s * scale * log2e - m) for one row's BN scores (masked columns > lim when
+// MASKED), written back over S as interleaved bf16 P_hi / P_lo words; *msum += sum p.
+// (Summing the unrounded p instead of P_hi + P_lo changes m_b by an unbiased
+// ~2^-18 relative error per weight.)
+template <int BN, bool MASKED>
+__device__ __forceinline__ void split_chunks(uint32_t tS, float sl2, float m_use, int lim, float* msum) {
+  const uint64_t scale2 = f2_pack(sl2, sl2);
+  const uint64_t negm2 = f2_pack(-m_use, -m_use);
+  uint64_t acc = f2_pack(0.f, 0.f);
+#pragma unroll
+  for (int cp = 0; cp < BN / 64; ++cp) {
+    uint32_t a[2][32];
+    tmem_ld32(tS + cp * 64, a[0]);
+    tmem_ld32(tS + cp * 64 + 32, a[1]);
+    tmem_ld_wait();
+    tmem_reg_fence(a[0]);
+    tmem_reg_fence(a[1]);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      uint32_t out[32];
+#pragma unroll
+      for (int x = 0; x < 16; ++x) {
+        const int col = cp * 64 + h * 32 + 2 * x;
+        const uint64_t xv = f2_fma(f2_pack(__uint_as_float(a[h][2 * x]), __uint_as_float(a[h][2 * x + 1])), scale2, negm2);
+        float x0, x1;
+        f2_unpack(xv, x0, x1);
+        float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+        if (MASKED) {
+          if (col > lim) p0 = 0.f;
+          if (col + 1 > lim) p1 = 0.f;
+        }
+        acc = f2_add(acc, f2_pack(p0, p1));
+        const uint32_t wh = pack_bf16x2(p0, p1);
+        const uint32_t wl = pack_bf16x2(p0 - bf16lo_to_f32(wh), p1 - bf16hi_to_f32(wh));
+        // k-step (x / 8): words 0-7 P_hi, 8-15 P_lo
+        out[(x >> 3) * 16 + (x & 7)] = wh;
+        out[(x >> 3) * 16 + 8 + (x & 7)] = wl;
+      }
+      tmem_st32(tS + cp * 64 + h * 32, out);
+    }
+  }
+  float a0, a1;
+  f2_unpack(acc, a0, a1);
+  *msum += a0 + a1;
+}
+
 template <int D, int BN, int PASS>
 __global__ void __launch_bounds__(kThreadsFwd, 2)
     poem_score_kernel(const __grid_constant__ CUtensorMap tmQs, const __grid_constant__ CUtensorMap tmK,
@@ -103,6 +149,7 @@ __global__ void __launch_bounds__(kThreadsFwd, 2)
   score_cta_coords(blockIdx.x, ctas_per_g, g, z0);
   const int z_last = min(z0 + 7, n_groups - 1);
   const int nb = z_last / G + 1;  // key blocks 0 .. largest tile of the CTA
+  const int i_lo = z0 / G;        // smallest tile of the CTA: blocks < i_lo need no mask
 
   if (tid == 0) {
     mbar_init(&sb->q_full, 1);
@@ -169,13 +216,13 @@ __global__ void __launch_bounds__(kThreadsFwd, 2)
         tc_fence_after();
         if (!wait_or_abort(&sb->v_full, j & 1, sb, p.err)) return false;
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-#pragma unroll
-          for (int kk = 0; kk < BN / 16; ++kk) {
-            const uint64_t bdesc = smem_desc_sw128(aV + kk * 2048, BN * 128, 1024);
-            const bool fresh = (PASS == 2 || j == 0) && half == 0 && kk == 0;
-            mma_ts(tO, tS + half * (BN / 2) + kk * 8, bdesc, C::kIdescPV, fresh ? 0u : 1u);
-          }
+        for (int kk = 0; kk < BN / 16; ++kk) {
+          // P for keys [16 kk, 16 kk + 16): P_hi words at TMEM columns [16 kk, +8),
+          // P_lo words at [16 kk + 8, +8)
+          const uint64_t bdesc = smem_desc_sw128(aV + kk * 2048, BN * 128, 1024);
+          const bool fresh = (PASS == 2 || j == 0) && kk == 0;
+          mma_ts(tO, tS + kk * 16, bdesc, C::kIdescPV, fresh ? 0u : 1u);
+          mma_ts(tO, tS + kk * 16 + 8, bdesc, C::kIdescPV, 1u);
         }
         mma_commit(&sb->v_empty);
         if (PASS == 2) mma_commit(&sb->o_full);  // P_b V_b of this block is ready
@@ -236,10 +283,18 @@ __global__ void __launch_bounds__(kThreadsFwd, 2)
           for (int c = 0; c < BN / 32; ++c) tmem_ld32(tS + c * 32, raw[c]);
           tmem_ld_wait();
 #pragma unroll
-          for (int c = 0; c < BN / 32; ++c) {
-            tmem_reg_fence(raw[c]);
+          for (int c = 0; c < BN / 32; ++c) tmem_reg_fence(raw[c]);
+          if (b < i_lo) {
 #pragma unroll
-            for (int x = 0; x < 32; ++x) mx = fmaxf(mx, (c * 32 + x <= lim) ? __uint_as_float(raw[c][x]) : -INFINITY);
+            for (int c = 0; c < BN / 32; ++c)
+#pragma unroll
+              for (int x = 0; x < 32; x += 2)
+                mx = fmax3(mx, __uint_as_float(raw[c][x]), __uint_as_float(raw[c][x + 1]));
+          } else {
+#pragma unroll
+            for (int c = 0; c < BN / 32; ++c)
+#pragma unroll
+              for (int x = 0; x < 32; ++x) mx = fmaxf(mx, (c * 32 + x <= lim) ? __uint_as_float(raw[c][x]) : -INFINITY);
           }
         }
         const float m_new = fmaxf(m_run, mx * sl2);
@@ -267,68 +322,14 @@ __global__ void __launch_bounds__(kThreadsFwd, 2)
       } else {
         m_use = lse2;
       }
-      // phase 2: p (masked), split P = P_hi + P_lo in bf16.  Half hf reads S columns
-      // [64 hf, 64 hf + 64) and writes P_hi words to [32 hf, +32) and P_lo words to
-      // [BN/2 + 32 hf, +32): only S columns already read are overwritten.
+      // phase 2: p, split P = P_hi + P_lo in bf16, in place: the 32 S columns of a
+      // chunk (two 16-key k-steps) become, per k-step, 8 P_hi words then 8 P_lo words.
+      // Rows of a CTA whose tiles all lie past this block need no mask (uniform).
       float msum = 0.f;
-#pragma unroll
-      for (int hf = 0; hf < BN / 64; ++hf) {
-        uint32_t a[2][32];
-        tmem_ld32(tS + hf * 64, a[0]);
-        tmem_ld32(tS + hf * 64 + 32, a[1]);
-        tmem_ld_wait();
-        tmem_reg_fence(a[0]);
-        tmem_reg_fence(a[1]);
-        uint32_t hi[32], lo[32];
-#pragma unroll
-        for (int x = 0; x < 32; ++x) {
-          const int c0 = hf * 64 + 2 * x;
-          const uint32_t r0 = a[x >> 4][(2 * x) & 31], r1 = a[x >> 4][(2 * x + 1) & 31];
-          const float p0 = (c0 <= lim) ? ex2_approx(fmaf(__uint_as_float(r0), sl2, -m_use)) : 0.f;
-          const float p1 = (c0 + 1 <= lim) ? ex2_approx(fmaf(__uint_as_float(r1), sl2, -m_use)) : 0.f;
-          const uint32_t wh = pack_bf16x2(p0, p1);
-          const float h0 = bf16lo_to_f32(wh), h1 = bf16hi_to_f32(wh);
-          const uint32_t wl = pack_bf16x2(p0 - h0, p1 - h1);
-          msum += (h0 + bf16lo_to_f32(wl)) + (h1 + bf16hi_to_f32(wl));
-          hi[x] = wh;
-          lo[x] = wl;
-        }
-        // Half 1's P_hi words land in [32, 64), whose S columns half 0 already read;
-        // P_lo words land in [BN/2 + 32 hf, ...), at or past the columns being read
-        // now -- so with BN = 128 the P_lo store of half 0 waits until half 1 is read.
-        tmem_st32(tS + hf * 32, hi);
-        if (BN == 64) {
-          tmem_st32(tS + BN / 2 + hf * 32, lo);
-        } else if (hf == 0) {
-          // keep lo of half 0 until the S columns [64, 96) it overwrites are read
-#pragma unroll
-          for (int x = 0; x < 32; ++x) a[0][x] = lo[x];
-          uint32_t b2[2][32];
-          tmem_ld32(tS + 64, b2[0]);
-          tmem_ld32(tS + 96, b2[1]);
-          tmem_ld_wait();
-          tmem_reg_fence(b2[0]);
-          tmem_reg_fence(b2[1]);
-          tmem_st32(tS + BN / 2, a[0]);
-          uint32_t hi2[32], lo2[32];
-#pragma unroll
-          for (int x = 0; x < 32; ++x) {
-            const int c0 = 64 + 2 * x;
-            const uint32_t r0 = b2[x >> 4][(2 * x) & 31], r1 = b2[x >> 4][(2 * x + 1) & 31];
-            const float p0 = (c0 <= lim) ? ex2_approx(fmaf(__uint_as_float(r0), sl2, -m_use)) : 0.f;
-            const float p1 = (c0 + 1 <= lim) ? ex2_approx(fmaf(__uint_as_float(r1), sl2, -m_use)) : 0.f;
-            const uint32_t wh = pack_bf16x2(p0, p1);
-            const float h0 = bf16lo_to_f32(wh), h1 = bf16hi_to_f32(wh);
-            const uint32_t wl = pack_bf16x2(p0 - h0, p1 - h1);
-            msum += (h0 + bf16lo_to_f32(wl)) + (h1 + bf16hi_to_f32(wl));
-            hi2[x] = wh;
-            lo2[x] = wl;
-          }
-          tmem_st32(tS + 32, hi2);
-          tmem_st32(tS + BN / 2 + 32, lo2);
-          break;
-        }
-      }
+      if (b < i_lo)
+        split_chunks<BN, false>(tS, sl2, m_use, lim, &msum);
+      else
+        split_chunks<BN, true>(tS, sl2, m_use, lim, &msum);
       if (PASS == 1) l_run += msum;
       tmem_st_wait();
       tc_fence_before();
@@ -342,7 +343,8 @@ __global__ void __launch_bounds__(kThreadsFwd, 2)
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) tmem_ld32(tO + c * 32, pv[c]);
         tmem_ld_wait();
-        float acc = 0.f;
+        uint64_t acc2 = f2_pack(0.f, 0.f);
+        const uint64_t negm2 = f2_pack(-msum, -msum);
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           tmem_reg_fence(pv[c]);
@@ -351,14 +353,18 @@ __global__ void __launch_bounds__(kThreadsFwd, 2)
 #pragma unroll
             for (int x = 0; x < 8; ++x) {
               const float4 ov = o4[x];
-              const float e0 = fmaf(-msum, ov.x, __uint_as_float(pv[c][4 * x + 0]));
-              const float e1 = fmaf(-msum, ov.y, __uint_as_float(pv[c][4 * x + 1]));
-              const float e2 = fmaf(-msum, ov.z, __uint_as_float(pv[c][4 * x + 2]));
-              const float e3 = fmaf(-msum, ov.w, __uint_as_float(pv[c][4 * x + 3]));
-              acc = fmaf(e0, e0, fmaf(e1, e1, fmaf(e2, e2, fmaf(e3, e3, acc))));
+              const uint64_t e01 = f2_fma(negm2, f2_pack(ov.x, ov.y),
+                                          f2_pack(__uint_as_float(pv[c][4 * x]), __uint_as_float(pv[c][4 * x + 1])));
+              const uint64_t e23 = f2_fma(negm2, f2_pack(ov.z, ov.w),
+                                          f2_pack(__uint_as_float(pv[c][4 * x + 2]), __uint_as_float(pv[c][4 * x + 3])));
+              acc2 = f2_fma(e01, e01, acc2);
+              acc2 = f2_fma(e23, e23, acc2);
             }
           }
         }
+        float acc0, acc1;
+        f2_unpack(acc2, acc0, acc1);
+        const float acc = acc0 + acc1;
         float Ib = valid ? sqrtf(acc) : 0.f;
         float mb = valid ? msum : 0.f;
 #pragma unroll
