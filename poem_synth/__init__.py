@@ -152,14 +152,15 @@ def random_block_lists(n_q_heads: int, n_tiles: int, density: float, seed: int =
     lists = []
     for h in range(n_q_heads):
         for i in range(n_tiles):
-            mand = {0, i}
-            if local_block and i >= 1:
-                mand.add(i - 1)
-            pool = np.array([b for b in range(1, i) if b not in mand], dtype=np.int64)
+            mand = [0] if i == 0 else [0, i]
+            if local_block and i >= 2:
+                mand = [0, i - 1, i]
+            hi = i - 1 if (local_block and i >= 2) else i  # pool: 1 .. hi-1
+            pool = np.arange(1, max(hi, 1), dtype=np.int64)
             total = max(len(mand), int(round(density * (i + 1))))
             extra = min(total - len(mand), pool.size)
             pick = rng.choice(pool, size=extra, replace=False) if extra > 0 else np.zeros(0, np.int64)
-            row = np.sort(np.concatenate([np.array(sorted(mand), dtype=np.int64), pick]))
+            row = np.sort(np.concatenate([np.array(mand, dtype=np.int64), pick]))
             lists.append(row)
             counts[h * n_tiles + i] = row.size
     row_ptr = np.zeros(n_q_heads * n_tiles + 1, dtype=np.int32)

@@ -1,0 +1,123 @@
+"""GPU parity at the full layer sizes, in the launch configuration bench.py times
+(poem_score -> poem_select with a work order -> bsa_fwd following that order).
+
+The oracle cannot run a whole 128K layer, so it checks a deterministic sample of
+(head, tile) units -- the first and last tiles of several heads and a few in
+between.  Units are independent in every step, so each sampled unit is an exact
+check of that unit: its scores I_hat/m_hat for all visible blocks, its block
+list (against the oracle's selection on the oracle's own scores, cut rule), and
+all 128 output rows of bsa_fwd (against oracle masked attention on the GPU's
+list)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import poem_synth
+from _parity import (FWD_MAX_ABS, FWD_MEAN_ABS, compare_fwd, csr_rows, lists_agree_at_cut, max_value_norm,
+                     problem_from, score_err_excess)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def poem():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from block_sparse_attention_poem_b200 import build
+
+    build.build()
+    oracle.build()
+    import block_sparse_attention_poem_b200 as m
+
+    return m
+
+
+def _sample_units(hq, T, extra):
+    units = {(0, 0), (0, 1), (0, 2), (hq - 1, T - 1), (hq // 2, T - 1), (1, T // 2)}
+    units |= set(extra)
+    return sorted(units)
+
+
+def _check_layer(poem, x, B, tau, units):
+    q, k, v = x["q"].cuda(), x["k"].cuda(), x["v"].cuda()
+    hq = q.shape[1]
+    T = q.shape[0] // B
+    layer = poem.prefill_layer(q, k, v, tau, block=B)
+    for ws in (layer.ws_score, layer.ws_select, layer.ws_fwd):
+        poem.poem_check(ws)
+    prob = problem_from(x, B)
+    Ir, mr = prob.score_units(units)
+    Ig = layer.I_hat.cpu().numpy()
+    mg = layer.m_hat.cpu().numpy()
+    idx = np.concatenate([np.arange(oracle.tri_offset(T, h, i), oracle.tri_offset(T, h, i) + i + 1) for h, i in units])
+    assert score_err_excess(Ig[idx], Ir[idx], mg[idx], mr[idx], max_value_norm(x["v"])) <= 1.0
+    rp = layer.row_ptr.cpu().numpy()
+    ci = layer.col_idx[: int(rp[-1])].cpu().numpy()
+    gpu_rows = csr_rows(rp, ci)
+    # oracle selection on the oracle's scores, for the sampled rows only
+    ref_rows = {}
+    for h, i in units:
+        off = oracle.tri_offset(T, h, i)
+        ref_rows[h * T + i] = oracle.select_row(i, Ir[off:off + i + 1], mr[off:off + i + 1], tau)[0].tolist()
+    full_ref = [ref_rows.get(r, gpu_rows[r]) for r in range(hq * T)]
+    _, bad = lists_agree_at_cut(gpu_rows, full_ref, Ir, mr, hq, T, tau)
+    assert not bad, bad
+    O_ref, _ = prob.masked_units(units, rp, ci)
+    mx, mean = compare_fwd(layer.o, O_ref, units, B)
+    assert mx <= FWD_MAX_ABS and mean <= FWD_MEAN_ABS, (mx, mean)
+    # work order: a permutation of the rows
+    assert sorted(layer.order.cpu().numpy().tolist()) == list(range(hq * T))
+    return rp
+
+
+def test_llama_layer_128k(poem):
+    """Llama-3.1-8B-shaped layer, 131072 tokens, tau = 0.05 (the benchmark workload)."""
+    n, hq, hkv, d, B = 131072, 32, 8, 128, 128
+    x = poem_synth.heavy_block_layer(n, hq, hkv, d, block=B, rope_base=500000.0, seed=0)
+    T = n // B
+    rp = _check_layer(poem, x, B, 0.05, _sample_units(hq, T, [(7, 300), (20, 1000)]))
+    assert rp[-1] > 0
+
+
+def test_qwen3_14b_layer_64k(poem):
+    """Qwen3-14B-shaped layer: 40 query / 8 KV heads (5-way GQA), 65536 tokens, RoPE base 1e6."""
+    n, hq, hkv, d, B = 65536, 40, 8, 128, 128
+    x = poem_synth.heavy_block_layer(n, hq, hkv, d, block=B, rope_base=1000000.0, seed=0)
+    T = n // B
+    _check_layer(poem, x, B, 0.05, _sample_units(hq, T, [(39, 255), (12, 401)]))
+
+
+@pytest.mark.parametrize("tau", [0.02, 0.05, 0.1])
+def test_llama_layer_32k(poem, tau):
+    n, hq, hkv, d, B = 32768, 32, 8, 128, 128
+    x = poem_synth.heavy_block_layer(n, hq, hkv, d, block=B, rope_base=500000.0, seed=1)
+    T = n // B
+    _check_layer(poem, x, B, tau, _sample_units(hq, T, [(3, 100)]))
+
+
+def test_single_head_recipe_end_to_end(poem):
+    """Single head, N = 1024, d = 64, 64x64 blocks, tau = 0.05: every unit checked."""
+    xs = poem_synth.single_head(1024, 64, seed=0)
+    x = {k: t.to(torch.bfloat16) for k, t in xs.items()}
+    units = [(0, i) for i in range(16)]
+    _check_layer(poem, x, 64, 0.05, units)
+
+
+@pytest.mark.parametrize("density", [0.05, 0.5])
+def test_bsa_fwd_random_masks_128k(poem, density):
+    """bsa_fwd alone on the fixed random block masks (sink + diagonal + uniform causal
+    blocks) at 131072 tokens, 32/8 heads, i.i.d. inputs."""
+    n, hq, hkv, d, B = 131072, 32, 8, 128, 128
+    T = n // B
+    x = poem_synth.iid_layer(n, hq, hkv, d, seed=3)
+    rp, ci = poem_synth.random_block_lists(hq, T, density, seed=3)
+    q, k, v = x["q"].cuda(), x["k"].cuda(), x["v"].cuda()
+    o = torch.empty_like(q)
+    ws = poem.alloc_workspace(256)
+    poem.bsa_fwd(q, k, v, torch.from_numpy(rp).cuda(), torch.from_numpy(ci).cuda(), o, ws, block=B)
+    poem.poem_check(ws)
+    units = _sample_units(hq, T, [(9, 640)])
+    O_ref, _ = problem_from(x, B).masked_units(units, rp, ci)
+    mx, mean = compare_fwd(o, O_ref, units, B)
+    assert mx <= FWD_MAX_ABS and mean <= FWD_MEAN_ABS, (mx, mean)
