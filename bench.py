@@ -44,9 +44,25 @@ WORKLOADS = {
     "llama3.1-8b-layer-32k": (32768, 32, 8, 128, 128, 500000.0, 0.05),
     "qwen3-14b-layer-64k": (65536, 40, 8, 128, 128, 1000000.0, 0.05),
 }
-# Roofline denominators measured on this machine's B200s (copied from the driver's
-# measurement; MEASURED_PEAKS.json, when present, takes precedence).
+# Roofline denominators measured on B200 (a STREAM-style copy and a bf16 GEMM;
+# MEASURED_PEAKS.json, when present, takes precedence).
 FALLBACK_PEAKS = {"bf16_tflops": 1667.9, "bf16_tflops_sustained": 1378.8, "hbm_gbs": 6452.5}
+# DRAM bytes per bsa_fwd launch on the 128K layer: the ncu capture of the 32K layer
+# (dram__bytes_read.sum + dram__bytes_write.sum = 640.7 MB per launch)
+# scaled by rows processed (x4).  Valid only for the kernel source it was taken on.
+BSA_FWD_TRAFFIC = {"bytes": 2.563e9, "source_sha256_prefix": "731b4af61dfbe7f7",
+                   "note": "ncu dram bytes of the 32K layer launch x4 rows"}
+
+
+def bsa_fwd_traffic():
+    import hashlib
+
+    path = os.path.join(ROOT, "block_sparse_attention_poem_b200", "csrc", "bsa_fwd.cu")
+    with open(path, "rb") as f:
+        digest = hashlib.sha256(f.read()).hexdigest()[:16]
+    if digest != BSA_FWD_TRAFFIC["source_sha256_prefix"]:
+        return None, "kernel changed since the ncu capture"
+    return BSA_FWD_TRAFFIC["bytes"], BSA_FWD_TRAFFIC["note"]
 
 
 def load_peaks():
@@ -55,7 +71,7 @@ def load_peaks():
         with open(p) as f:
             d = json.load(f)
         return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured (MEASURED_PEAKS.json)"
-    return dict(FALLBACK_PEAKS), "measured (copy in BASELINE.md)"
+    return dict(FALLBACK_PEAKS), "measured on B200 (values copied into the benchmark)"
 
 
 class ClockSampler:
@@ -220,6 +236,7 @@ def run_ours(args):
     dflops = dense_flops(n, hq, d)
     peaks, peak_src = load_peaks()
     fwd_tflops = rflops / (fwd_ms * 1e-3) / 1e12
+    traffic, traffic_note = bsa_fwd_traffic() if args.workload == "llama3.1-8b-layer-128k" else (None, "no capture")
 
     # end-to-end through the public API with host buffers: H2D of Q/K/V from pinned
     # memory, the three calls, D2H of O, every step.
@@ -292,7 +309,8 @@ def run_ours(args):
                      "frac": round(fwd_tflops / peaks["bf16_tflops_sustained"], 4),
                      "frac_of_burst_peak": round(fwd_tflops / peaks["bf16_tflops"], 4),
                      "peak_source": peak_src + ", sustained bf16 (kernel timed inside a long step)",
-                     "algorithmic_flops_per_launch": rflops, "traffic": None},
+                     "algorithmic_flops_per_launch": rflops, "traffic": traffic,
+                     "traffic_note": traffic_note},
         "clocks": clk,
         "e2e": e2e,
         "gpu_launches": launches_per_step * args.steps,
@@ -409,6 +427,141 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+# --------------------------------------------------------------------------
+# --report: one JSON record per configuration (measurement table)
+# --------------------------------------------------------------------------
+
+REPORT_LAYERS = [
+    # (name, generator kwargs, taus, run mass-only comparison)
+    ("single-head-1k-d64-b64", None, [0.05], False),
+    ("llama3.1-8b-layer-32k", "llama3.1-8b-layer-32k", [0.02, 0.05, 0.1], False),
+    ("llama3.1-8b-layer-128k", "llama3.1-8b-layer-128k", [0.05], True),
+    ("qwen3-14b-layer-64k", "qwen3-14b-layer-64k", [0.05], False),
+]
+SWEEP_TOKENS = [8192, 16384, 32768, 65536, 131072]
+SWEEP_DENSITY = [0.05, 0.1, 0.25, 0.5, 1.0]
+
+
+def _events(n):
+    return [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+
+
+def _report_layer(poem, name, wl, tau, steps, warmup, mass_only, cpu_budget_s):
+    if wl is None:
+        xs = poem_synth.single_head(1024, 64, seed=0)
+        x = {k: t.to(torch.bfloat16) for k, t in xs.items()}
+        n, hq, hkv, d, B = 1024, 1, 1, 64, 64
+    else:
+        n, hq, hkv, d, B, base, _ = WORKLOADS[wl]
+        x = poem_synth.heavy_block_layer(n, hq, hkv, d, block=B, rope_base=base, seed=0)
+    T = n // B
+    q, k, v = x["q"].cuda(), x["k"].cuda(), x["v"].cuda()
+    layer = poem.alloc_layer(q, k, block=B)
+    ph = {"poem_score": [], "poem_select": [], "bsa_fwd": []}
+    for it in range(warmup + steps):
+        ev = _events(4)
+        ev[0].record()
+        poem.poem_score(q, k, v, layer.I_hat, layer.m_hat, layer.ws_score, shape=layer.shape)
+        ev[1].record()
+        poem.poem_select(layer.shape, layer.I_hat, layer.m_hat, tau, layer.row_ptr, layer.col_idx, layer.ws_select,
+                         order=layer.order)
+        ev[2].record()
+        poem.bsa_fwd(q, k, v, layer.row_ptr, layer.col_idx, layer.o, layer.ws_fwd, order=layer.order,
+                     shape=layer.shape)
+        ev[3].record()
+        torch.cuda.synchronize()
+        if it >= warmup:
+            for j, key in enumerate(ph):
+                ph[key].append(ev[j].elapsed_time(ev[j + 1]))
+    for ws in (layer.ws_score, layer.ws_select, layer.ws_fwd):
+        poem.poem_check(ws)
+    ms = {key: float(np.median(val)) for key, val in ph.items()}
+    total = sum(ms.values())
+    rp = layer.row_ptr.cpu().numpy()
+    ci = layer.col_idx[: int(rp[-1])].cpu().numpy()
+    kept = int(rp[-1])
+    visible = hq * T * (T + 1) // 2
+    rfl = retained_flops(rp, ci, T, d, B)
+    peaks, _ = load_peaks()
+    fwd_tf = rfl / (ms["bsa_fwd"] * 1e-3) / 1e12
+    sel_bytes = 8.0 * visible + 4.0 * kept + 4.0 * (hq * T + 1)
+    sel_gbs = sel_bytes / (ms["poem_select"] * 1e-3) / 1e9
+    rec = {
+        "config": name, "tau": tau, "n_tokens": n, "n_q_heads": hq, "n_kv_heads": hkv, "head_dim": d, "block": B,
+        "ms": {key: round(val, 4) for key, val in ms.items()}, "ms_per_layer": round(total, 4),
+        "density": round(kept / visible, 5),
+        "dense_equiv_tflops": round(dense_flops(n, hq, d) / (total * 1e-3) / 1e12, 2),
+        "bsa_fwd_retained_tflops": round(fwd_tf, 2),
+        "bsa_fwd_frac_burst": round(fwd_tf / peaks["bf16_tflops"], 4),
+        "bsa_fwd_frac_sustained": round(fwd_tf / peaks["bf16_tflops_sustained"], 4),
+        "select_gbs": round(sel_gbs, 1), "select_frac_hbm": round(sel_gbs / peaks["hbm_gbs"], 4),
+        "score_select_over_fwd": round((ms["poem_score"] + ms["poem_select"]) / ms["bsa_fwd"], 4),
+    }
+    q_, k_, v_ = q, k, v
+    rec["err_vs_dense"] = quality_report(poem, q_, k_, v_, layer, tau, n, hq, T, B, q.device)["err_vs_dense"]
+    if not mass_only:
+        rec["err_vs_dense"].pop("mass_only_same_budget", None)
+    if cpu_budget_s > 0:
+        cb = cpu_baseline(x, n, hq, hkv, d, B, tau, cpu_budget_s)
+        rec["oracle_ms_per_layer"] = cb["value"]
+        rec["oracle_cores"] = cb["cores"]
+        rec["oracle_note"] = cb["sample"]
+    del layer, q, k, v
+    torch.cuda.empty_cache()
+    return rec
+
+
+def _report_sweep(poem, steps, warmup):
+    out = []
+    peaks, _ = load_peaks()
+    hq, hkv, d, B = 32, 8, 128, 128
+    for n in SWEEP_TOKENS:
+        x = poem_synth.iid_layer(n, hq, hkv, d, seed=0)
+        q, k, v = x["q"].cuda(), x["k"].cuda(), x["v"].cuda()
+        T = n // B
+        o = torch.empty_like(q)
+        ws = poem.alloc_workspace(256)
+        for dens in SWEEP_DENSITY:
+            rp, ci = poem_synth.random_block_lists(hq, T, dens, seed=0)
+            rpd, cid = torch.from_numpy(rp).cuda(), torch.from_numpy(ci).cuda()
+            times = []
+            for it in range(warmup + steps):
+                ev = _events(2)
+                ev[0].record()
+                poem.bsa_fwd(q, k, v, rpd, cid, o, ws, block=B)
+                ev[1].record()
+                torch.cuda.synchronize()
+                if it >= warmup:
+                    times.append(ev[0].elapsed_time(ev[1]))
+            poem.poem_check(ws)
+            t = float(np.median(times))
+            rfl = retained_flops(rp, ci, T, d, B)
+            tf = rfl / (t * 1e-3) / 1e12
+            out.append({"config": "bsa_fwd-sweep", "n_tokens": n, "density_target": dens,
+                        "density": round(int(rp[-1]) / (hq * T * (T + 1) / 2), 5), "ms": round(t, 4),
+                        "retained_tflops": round(tf, 2), "frac_burst": round(tf / peaks["bf16_tflops"], 4),
+                        "frac_sustained": round(tf / peaks["bf16_tflops_sustained"], 4),
+                        "dense_equiv_tflops": round(dense_flops(n, hq, d) / (t * 1e-3) / 1e12, 2)})
+        del q, k, v, o
+        torch.cuda.empty_cache()
+    return out
+
+
+def run_report(args):
+    import block_sparse_attention_poem_b200 as poem
+
+    torch.cuda.set_device(0)
+    clocks = ClockSampler(0)
+    clocks.start()
+    for name, wl, taus, mass_only in REPORT_LAYERS:
+        for tau in taus:
+            rec = _report_layer(poem, name, wl, tau, args.steps, args.warmup, mass_only, args.cpu_budget_s)
+            print(json.dumps(rec), flush=True)
+    for rec in _report_sweep(poem, args.steps, args.warmup):
+        print(json.dumps(rec), flush=True)
+    print(json.dumps({"config": "clocks", "clocks": clocks.stop()}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -423,8 +576,12 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget-s", type=float, default=15.0)
     ap.add_argument("--ref-step-budget-s", type=float, default=8.0)
+    ap.add_argument("--report", action="store_true",
+                    help="measure every configuration (one JSON record each) instead of the benchmark line")
     args = ap.parse_args()
-    if args.impl == "reference":
+    if args.report:
+        run_report(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)
