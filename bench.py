@@ -145,6 +145,25 @@ def dense_flops(n: int, hq: int, d: int) -> float:
     return float(2 * d * hq * n * (n + 1))
 
 
+def reduce_max(value: float) -> float:
+    """Max of a per-rank value over the process group (identity without one).
+    Works with any backend: the tensor lives on the GPU for NCCL, on the CPU else."""
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    dev = torch.device("cuda", torch.cuda.current_device()) if dist.get_backend() == "nccl" else torch.device("cpu")
+    t = torch.tensor([float(value)], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_ms_per_layer(max_rank_ms: float, steps: int, world: int) -> float:
+    """Every rank runs `steps` layers (independent replicas); the job's ms per layer is
+    the slowest rank's time over all layers the job processed."""
+    return max_rank_ms / (steps * world)
+
+
 def dist_setup():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -213,14 +232,9 @@ def run_ours(args):
     score_ms = float(np.mean([e[0].elapsed_time(e[1]) for e in evs]))
     select_ms = float(np.mean([e[1].elapsed_time(e[2]) for e in evs]))
     fwd_ms = float(np.mean([e[2].elapsed_time(e[3]) for e in evs]))
-    if world > 1:
-        import torch.distributed as dist
-
-        tt = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        total_ms = float(tt.item())
+    total_ms = reduce_max(total_ms)
     ms_per_step = total_ms / args.steps
-    ms_per_layer = total_ms / (args.steps * world)
+    ms_per_layer = whole_job_ms_per_layer(total_ms, args.steps, world)
 
     for ws in (layer.ws_score, layer.ws_select, layer.ws_fwd):
         poem.poem_check(ws)
@@ -260,14 +274,8 @@ def run_ours(args):
             ho.copy_(layer.o, non_blocking=True)
         e1.record(stream)
         torch.cuda.synchronize()
-        e2e_ms = e0.elapsed_time(e1)
-        if world > 1:
-            import torch.distributed as dist
-
-            tt = torch.tensor([e2e_ms], device=dev)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            e2e_ms = float(tt.item())
-        e2e = {"value": e2e_ms / (args.e2e_steps * world), "unit": "ms/layer",
+        e2e_ms = reduce_max(e0.elapsed_time(e1))
+        e2e = {"value": whole_job_ms_per_layer(e2e_ms, args.e2e_steps, world), "unit": "ms/layer",
                "h2d_bytes_per_step": int(hq_h.numel() * 2 + hk_h.numel() * 2 + hv_h.numel() * 2),
                "d2h_bytes_per_step": int(ho.numel() * 2)}
 
