@@ -68,11 +68,8 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, Fw
 constexpr uint64_t kDrainNs = 2000000000ull;  // waits for already-issued async work
 
 // Exponentials of one S row (re-read from TMEM in 64-column halves), the bf16 P
-// written over the first BN/2 TMEM columns of S, and the row sum added to *l.  One pair in kPolyEvery is evaluated on the FMA pipe (exp2_pair_poly) to
-// unload MUFU; the diagonal block (masked columns already -inf) uses MUFU only,
-// so masked weights are exactly zero.
-constexpr int kPolyEvery = 4;
-
+// written over the first BN/2 TMEM columns of S, and the row sum added to *l.
+// On the diagonal block the masked columns get weight exactly zero.
 template <int BN, bool DIAG>
 __device__ __forceinline__ void exp_pack_store(uint32_t tS, float sl2, float m_use, int lim, float* l) {
   const uint64_t scale2 = f2_pack(sl2, sl2);
@@ -99,8 +96,6 @@ __device__ __forceinline__ void exp_pack_store(uint32_t tS, float sl2, float m_u
       if (DIAG) {
         y0 = (hf * 64 + 2 * x <= lim) ? ex2_approx(x0) : 0.f;
         y1 = (hf * 64 + 2 * x + 1 <= lim) ? ex2_approx(x1) : 0.f;
-      } else if ((x % kPolyEvery) == kPolyEvery - 1) {
-        exp2_pair_poly(x0, x1, y0, y1);
       } else {
         y0 = ex2_approx(x0);
         y1 = ex2_approx(x1);
@@ -289,17 +284,22 @@ __global__ void __launch_bounds__(kThreadsFwd, 2)
           tmem_ld_wait();
 #pragma unroll
           for (int c = 0; c < BN / 32; ++c) tmem_reg_fence(sv[c]);
+          // four independent partial maxima (short dependency chains)
+          float pm[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
           if (diag) {  // uniform branch
 #pragma unroll
             for (int c = 0; c < BN / 32; ++c)
 #pragma unroll
-              for (int x = 0; x < 32; ++x) mx = fmaxf(mx, (c * 32 + x <= lim) ? __uint_as_float(sv[c][x]) : -INFINITY);
+              for (int x = 0; x < 32; ++x)
+                pm[x & 3] = fmaxf(pm[x & 3], (c * 32 + x <= lim) ? __uint_as_float(sv[c][x]) : -INFINITY);
           } else {
 #pragma unroll
             for (int c = 0; c < BN / 32; ++c)
 #pragma unroll
-              for (int x = 0; x < 32; x += 2) mx = fmax3(mx, __uint_as_float(sv[c][x]), __uint_as_float(sv[c][x + 1]));
+              for (int x = 0; x < 32; x += 2)
+                pm[(x >> 1) & 3] = fmax3(pm[(x >> 1) & 3], __uint_as_float(sv[c][x]), __uint_as_float(sv[c][x + 1]));
           }
+          mx = fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3]));
         }
         const float m_new = fmaxf(m_run, mx * sl2);
         const bool grow = (m_new > m_run + 8.0f);

@@ -266,36 +266,6 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return r;
 }
 
-// 2^x for a pair of floats on the FMA/ALU pipes instead of MUFU (Cody-Waite style
-// range reduction): x = j + f with j = round-to-nearest(x) obtained by adding
-// 1.5 * 2^23, f in [-1/2, 1/2]; 2^f from a degree-3 polynomial whose coefficients
-// are the relative-error minimax fit on [-1/2, 1/2] (Remez exchange, computed for
-// this library; max relative error 7.5e-5 in fp32, far below the 2^-9 rounding of
-// the bf16 weights it feeds); j is added to the exponent field.  Inputs below
-// -126 are clamped there (results ~1e-38).
-constexpr float kExp2C0 = 9.999280572e-01f;
-constexpr float kExp2C1 = 6.932609677e-01f;
-constexpr float kExp2C2 = 2.426111251e-01f;
-constexpr float kExp2C3 = 5.517166853e-02f;
-__device__ __forceinline__ void exp2_pair_poly(float x0, float x1, float& y0, float& y1) {
-  const float kMagic = 12582912.0f;  // 1.5 * 2^23
-  x0 = fmaxf(x0, -126.f);
-  x1 = fmaxf(x1, -126.f);
-  const uint64_t x = f2_pack(x0, x1);
-  const uint64_t t = f2_add(x, f2_pack(kMagic, kMagic));             // round(x) in the low bits
-  const uint64_t j = f2_add(t, f2_pack(-kMagic, -kMagic));           // round(x) as float
-  const uint64_t f = f2_fma(j, f2_pack(-1.f, -1.f), x);               // x - round(x)
-  uint64_t p = f2_fma(f2_pack(kExp2C3, kExp2C3), f, f2_pack(kExp2C2, kExp2C2));
-  p = f2_fma(p, f, f2_pack(kExp2C1, kExp2C1));
-  p = f2_fma(p, f, f2_pack(kExp2C0, kExp2C0));
-  float p0, p1, t0, t1;
-  f2_unpack(p, p0, p1);
-  f2_unpack(t, t0, t1);
-  // (bits(t) << 23) == round(x) << 23 (mod 2^32): the magic's own bits shift out.
-  y0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
-  y1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
-}
-
 // Round two floats to bf16 (nearest-even) and pack: lo in bits [0,16), hi in [16,32).
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
