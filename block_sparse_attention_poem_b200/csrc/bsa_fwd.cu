@@ -13,7 +13,9 @@
 //              epilogue (O / l -> bf16, lse).
 //   warp 4     TMA producer: Q once, then K_j and V_j of every listed block.
 //   warp 5     MMA issuer (one thread): S = Q K_j^T (SS form), O += P V_j (P read
-//              from TMEM), completion tracked with tcgen05.commit -> mbarriers.
+//              from TMEM) in two 64-key halves, each started as soon as the softmax
+//              warps have written that half of P; completion tracked with
+//              tcgen05.commit -> mbarriers.
 // TMEM: 256 columns per CTA -- S/P at [0, BN), O at [128, 128 + D).  Shared
 // memory holds one Q, one K and one V tile (96 KB at D = BN = 128), so two CTAs
 // run per SM and their softmax / MMA phases interleave on the tensor cores.
@@ -43,7 +45,7 @@ struct FwdCfg {
 };
 
 struct FwdBarriers {
-  uint64_t q_full, k_full, k_empty, v_full, v_empty, s_full, p_full, o_full, drain;
+  uint64_t q_full, k_full, k_empty, v_full, v_empty, s_full, p_half[2], o_full, drain;
   uint32_t tmem_base;
   volatile int abort_flag;
 };
@@ -71,7 +73,8 @@ constexpr uint64_t kDrainNs = 2000000000ull;  // waits for already-issued async 
 // written over the first BN/2 TMEM columns of S, and the row sum added to *l.
 // On the diagonal block the masked columns get weight exactly zero.
 template <int BN, bool DIAG>
-__device__ __forceinline__ void exp_pack_store(uint32_t tS, float sl2, float m_use, int lim, float* l) {
+__device__ __forceinline__ void exp_pack_store(uint32_t tS, float sl2, float m_use, int lim, float* l,
+                                               uint64_t* p_half) {
   const uint64_t scale2 = f2_pack(sl2, sl2);
   const uint64_t negm2 = f2_pack(-m_use, -m_use);
   uint64_t acc = f2_pack(0.f, 0.f);
@@ -104,6 +107,10 @@ __device__ __forceinline__ void exp_pack_store(uint32_t tS, float sl2, float m_u
       packed[x] = pack_bf16x2(y0, y1);
     }
     tmem_st32(tS + hf * 32, packed);
+    // this half of P (and any O rescale before it) is in TMEM: its P V MMAs may start
+    tmem_st_wait();
+    tc_fence_before();
+    mbar_arrive(&p_half[hf]);
   }
   float a0, a1;
   f2_unpack(acc, a0, a1);
@@ -150,7 +157,8 @@ __global__ void __launch_bounds__(kThreadsFwd, 2)
     mbar_init(&sb->v_full, 1);
     mbar_init(&sb->v_empty, 1);
     mbar_init(&sb->s_full, 1);
-    mbar_init(&sb->p_full, 128);
+    mbar_init(&sb->p_half[0], 128);
+    mbar_init(&sb->p_half[1], 128);
     mbar_init(&sb->o_full, 1);
     mbar_init(&sb->drain, 1);
     sb->abort_flag = 0;
@@ -211,16 +219,21 @@ __global__ void __launch_bounds__(kThreadsFwd, 2)
       int it = 0;
       bool ok = true;
       bool q_ready = false;
+      // O += P_j V_j in two 64-key halves, each issued as soon as the softmax warps
+      // have written that half of P_j.
       auto issue_pv = [&](int j) -> bool {
-        if (!wait_or_abort(&sb->p_full, j & 1, sb, p.err)) return false;
-        tc_fence_after();
         if (!wait_or_abort(&sb->v_full, j & 1, sb, p.err)) return false;
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk) {
-          // V tile is MN-major (d contiguous): LBO = stride between 64-wide d chunks,
-          // SBO = stride between 8-key groups; a k-step covers 16 keys = 2 groups.
-          const uint64_t bdesc = smem_desc_sw128(aV + kk * 2048, BN * 128, 1024);
-          mma_ts(tO, tS + kk * 8, bdesc, C::kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
+        for (int hv = 0; hv < BN / 64; ++hv) {
+          if (!wait_or_abort(&sb->p_half[hv], j & 1, sb, p.err)) return false;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = hv * 4; kk < hv * 4 + 4; ++kk) {
+            // V tile is MN-major (d contiguous): LBO = stride between 64-wide d chunks,
+            // SBO = stride between 8-key groups; a k-step covers 16 keys = 2 groups.
+            const uint64_t bdesc = smem_desc_sw128(aV + kk * 2048, BN * 128, 1024);
+            mma_ts(tO, tS + kk * 8, bdesc, C::kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
+          }
         }
         mma_commit(&sb->v_empty);
         return true;
@@ -325,12 +338,9 @@ __global__ void __launch_bounds__(kThreadsFwd, 2)
         l_run *= alpha;
         const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
         if (diag)
-          exp_pack_store<BN, true>(tS, sl2, m_use, lim, &l_run);
+          exp_pack_store<BN, true>(tS, sl2, m_use, lim, &l_run, sb->p_half);
         else
-          exp_pack_store<BN, false>(tS, sl2, m_use, lim, &l_run);
-        tmem_st_wait();
-        tc_fence_before();
-        mbar_arrive(&sb->p_full);
+          exp_pack_store<BN, false>(tS, sl2, m_use, lim, &l_run, sb->p_half);
         ++it;
       }
       id = id_next;
