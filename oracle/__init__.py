@@ -18,6 +18,11 @@ Every function cites the passage of the method description it follows:
   stopping rule  S_m < 1 and S_I <= tau (1 - S_m)  over the discarded suffix.
 * "Block-Filtered Long-Context Attention", Appendix "Block ordering": equal
   scores rank the smaller block id first; lists are traversed in ascending id.
+* Practical POEM (the note's paragraph on Equation (6) and Appendix B):
+  estimated (mean-pooled) block masses and deviations, a mass shortlist, a
+  rerank by log mass + w log deviation, and a pooled-mass retention threshold.
+  The estimators and parameters are not printed; the reading is documented
+  next to the C functions.
 
 Inputs are [n_tokens, n_heads, head_dim] arrays: float64, or uint16 arrays
 holding bf16 bit patterns (widened exactly to fp64 inside the C code).
@@ -86,6 +91,14 @@ def _load():
         lib.oracle_masked_units.restype = None
         lib.oracle_dense_units.argtypes = [sp, vp, vp, vp, ctypes.c_int, ip, ip, dp, dp]
         lib.oracle_dense_units.restype = None
+        lib.oracle_pooled_units.argtypes = [sp, vp, vp, vp, ctypes.c_int, ip, ip, dp, dp]
+        lib.oracle_pooled_units.restype = None
+        lib.oracle_select_practical_row.argtypes = [ctypes.c_int, dp, dp, ctypes.c_double, ctypes.c_double,
+                                                    ctypes.c_double, ip, ip]
+        lib.oracle_select_practical_row.restype = ctypes.c_int
+        lib.oracle_select_practical_rows.argtypes = [ctypes.c_int, ctypes.c_int, ip, ip, dp, dp, ctypes.c_double,
+                                                     ctypes.c_double, ctypes.c_double, ip, ip, ip]
+        lib.oracle_select_practical_rows.restype = None
         lib.oracle_num_threads.argtypes = []
         lib.oracle_num_threads.restype = ctypes.c_int
         _lib = lib
@@ -220,6 +233,24 @@ class Problem:
         _load().oracle_masked_units(*self._ptrs(), len(units), _ip(uh), _ip(ui), _ip(rp), _ip(ci), _dp(O), _dp(lse))
         return O, lse
 
+    # -- practical scoring: pooled masses and deviations (reading of Eq. 6) ----
+    def pooled_units(self, units, m_pool=None, d_pool=None):
+        """Pooled block masses m~ and deviations d~ = ||v~_b - o~|| for the listed
+        (h, i) units, packed lower-triangular like score_units."""
+        T = self.n_tiles
+        total = self.n_q_heads * T * (T + 1) // 2
+        if m_pool is None:
+            m_pool = np.zeros(total)
+        if d_pool is None:
+            d_pool = np.zeros(total)
+        uh = np.ascontiguousarray([u[0] for u in units], dtype=np.int32)
+        ui = np.ascontiguousarray([u[1] for u in units], dtype=np.int32)
+        _load().oracle_pooled_units(*self._ptrs(), len(units), _ip(uh), _ip(ui), _dp(m_pool), _dp(d_pool))
+        return m_pool, d_pool
+
+    def pooled_all(self):
+        return self.pooled_units([(h, i) for h in range(self.n_q_heads) for i in range(self.n_tiles)])
+
     def dense_units(self, units):
         B, d = self.block, self.head_dim
         uh = np.ascontiguousarray([u[0] for u in units], dtype=np.int32)
@@ -254,6 +285,36 @@ def select_mass_only_row(i: int, mhat_row, k_free: int):
     out = np.zeros(i + 1, dtype=np.int32)
     n = _load().oracle_select_mass_only_row(i, _dp(mh), int(k_free), _ip(out))
     return out[:n].copy()
+
+
+def select_practical_row(i: int, m_pool_row, d_pool_row, w: float, gamma: float, rho: float):
+    """Practical selection of tile i: stage-1 mass shortlist (fraction rho), stage-2
+    rerank by log m~ + w log d~, keep until the pooled mass reaches gamma.
+    Returns (kept ids ascending, prefix length kept from the reranked shortlist)."""
+    m = np.ascontiguousarray(m_pool_row, dtype=np.float64)
+    dv = np.ascontiguousarray(d_pool_row, dtype=np.float64)
+    out = np.zeros(i + 1, dtype=np.int32)
+    kc = np.zeros(1, dtype=np.int32)
+    n = _load().oracle_select_practical_row(i, _dp(m), _dp(dv), float(w), float(gamma), float(rho), _ip(out),
+                                            _ip(kc))
+    return out[:n].copy(), int(kc[0])
+
+
+def select_practical_all(n_q_heads: int, n_tiles: int, m_pool, d_pool, w: float, gamma: float, rho: float):
+    rows = [(h, i) for h in range(n_q_heads) for i in range(n_tiles)]
+    rh = np.ascontiguousarray([r[0] for r in rows], dtype=np.int32)
+    ri = np.ascontiguousarray([r[1] for r in rows], dtype=np.int32)
+    m = np.ascontiguousarray(m_pool, dtype=np.float64)
+    dv = np.ascontiguousarray(d_pool, dtype=np.float64)
+    lists = np.zeros((len(rows), n_tiles), dtype=np.int32)
+    counts = np.zeros(len(rows), dtype=np.int32)
+    kcut = np.zeros(len(rows), dtype=np.int32)
+    _load().oracle_select_practical_rows(n_tiles, len(rows), _ip(rh), _ip(ri), _dp(m), _dp(dv), float(w),
+                                         float(gamma), float(rho), _ip(lists), _ip(counts), _ip(kcut))
+    row_ptr = np.zeros(len(rows) + 1, dtype=np.int32)
+    row_ptr[1:] = np.cumsum(counts)
+    col_idx = np.concatenate([lists[r, : counts[r]] for r in range(len(rows))])
+    return row_ptr, col_idx.astype(np.int32), kcut
 
 
 def select_all(n_q_heads: int, n_tiles: int, Ihat, mhat, tau: float, rows=None):

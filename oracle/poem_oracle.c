@@ -377,3 +377,126 @@ int oracle_num_threads(void) {
     return 1;
 #endif
 }
+
+/* ---- practical (estimated) scoring: pooled block statistics ----------------- */
+
+/*
+ * Practical POEM (reading note, the paragraph on Equation (6) and Appendix B)
+ * estimates the dense reference and the block outputs instead of computing
+ * them, pre-selects candidates by mass, reranks them by an approximate log mass
+ * plus a weighted log deviation, and keeps blocks in that order until the
+ * accumulated pooled mass reaches the retention threshold.  The estimators are
+ * not printed; the reading taken here is the plainest one:
+ *   q~_i = mean of the B queries of tile i,   k~_b, v~_b = means of block b,
+ *   m~_b = softmax over visible b <= i of scale * <q~_i, k~_b>,
+ *   o~_i = sum_b m~_b v~_b,   d~_b = || v~_b - o~_i ||.
+ * For each listed unit (h, i) this writes m~ and d~ of blocks 0..i at the packed
+ * offset of (h, i).  With one token per block and one query per tile the pooled
+ * quantities are the exact m_b, o and || v_b - o ||.
+ */
+void oracle_pooled_units(const oracle_shape* s, const void* q, const void* k, const void* v,
+                         int n_units, const int* unit_h, const int* unit_i, double* m_pool, double* d_pool) {
+    const int B = s->block, d = s->head_dim, T = s->n_tokens / B;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int u = 0; u < n_units; ++u) {
+        const int h = unit_h[u], i = unit_i[u], hk = kv_head_of(s, h);
+        const int nb = i + 1;
+        double* qm = (double*)calloc((size_t)d, sizeof(double));
+        double* km = (double*)calloc((size_t)nb * d, sizeof(double));
+        double* vm = (double*)calloc((size_t)nb * d, sizeof(double));
+        double* lg = (double*)malloc(sizeof(double) * (size_t)nb);
+        double* om = (double*)calloc((size_t)d, sizeof(double));
+        for (int t = i * B; t < (i + 1) * B; ++t)
+            for (int c = 0; c < d; ++c) qm[c] += elem(s, q, s->n_q_heads, t, h, c) / B;
+        for (int b = 0; b < nb; ++b)
+            for (int t = b * B; t < (b + 1) * B; ++t)
+                for (int c = 0; c < d; ++c) {
+                    km[(size_t)b * d + c] += elem(s, k, s->n_kv_heads, t, hk, c) / B;
+                    vm[(size_t)b * d + c] += elem(s, v, s->n_kv_heads, t, hk, c) / B;
+                }
+        double mx = -INFINITY;
+        for (int b = 0; b < nb; ++b) {
+            double acc = 0.0;
+            for (int c = 0; c < d; ++c) acc += qm[c] * km[(size_t)b * d + c];
+            lg[b] = s->scale * acc;
+            if (lg[b] > mx) mx = lg[b];
+        }
+        double den = 0.0;
+        for (int b = 0; b < nb; ++b) { lg[b] = exp(lg[b] - mx); den += lg[b]; }
+        double* mo = m_pool + tri_offset(T, h, i);
+        double* dv = d_pool + tri_offset(T, h, i);
+        for (int b = 0; b < nb; ++b) {
+            mo[b] = lg[b] / den;
+            for (int c = 0; c < d; ++c) om[c] += mo[b] * vm[(size_t)b * d + c];
+        }
+        for (int b = 0; b < nb; ++b) {
+            double dev2 = 0.0;
+            for (int c = 0; c < d; ++c) {
+                double e = vm[(size_t)b * d + c] - om[c];
+                dev2 += e * e;
+            }
+            dv[b] = sqrt(dev2);
+        }
+        free(qm); free(km); free(vm); free(lg); free(om);
+    }
+}
+
+/*
+ * Practical selection of tile i from pooled masses m~[0..i] and deviations
+ * d~[0..i]:
+ *   mandatory {0, i-1, i};
+ *   stage 1: candidates 1..i-2 ranked by (m~ desc, id asc), the first
+ *            ceil(rho * |Cand|) kept (rho in [0, 1]);
+ *   stage 2: that shortlist reranked by (log m~ + w log d~ desc, id asc)
+ *            (Equation (6) form; log 0 = -inf);
+ *   keep the shortest prefix of the reranked shortlist with
+ *            sum_{mandatory} m~ + sum_{prefix} m~ >= gamma
+ *            (the whole shortlist when the threshold is never reached).
+ * Writes the kept ids ascending; returns the count, *k_out = prefix length.
+ */
+static double rank_key(double m, double dv, double w) {
+    double lm = (m > 0.0) ? log(m) : -INFINITY;
+    double ld = (dv > 0.0) ? log(dv) : -INFINITY;
+    if (lm == -INFINITY || (w > 0.0 && ld == -INFINITY)) return -INFINITY;
+    return lm + w * ((w == 0.0) ? 0.0 : ld);
+}
+
+int oracle_select_practical_row(int i, const double* m_pool, const double* d_pool, double w, double gamma,
+                                double rho, int* keep_out, int* k_out) {
+    unsigned char* keep = (unsigned char*)calloc((size_t)i + 1, 1);
+    mark_mandatory(i, keep);
+    int nc = i - 2;
+    if (nc < 0) nc = 0;
+    ranked* r = (ranked*)malloc(sizeof(ranked) * (size_t)(nc > 0 ? nc : 1));
+    for (int c = 0; c < nc; ++c) { r[c].key = m_pool[c + 1]; r[c].id = c + 1; }
+    qsort(r, (size_t)nc, sizeof(ranked), ranked_cmp);
+    int n1 = (int)ceil(rho * (double)nc);
+    if (n1 > nc) n1 = nc;
+    if (n1 < 0) n1 = 0;
+    for (int c = 0; c < n1; ++c) r[c].key = rank_key(m_pool[r[c].id], d_pool[r[c].id], w);
+    qsort(r, (size_t)n1, sizeof(ranked), ranked_cmp);
+    double acc = 0.0;
+    for (int b = 0; b <= i; ++b)
+        if (keep[b]) acc += m_pool[b];
+    int kcut = 0;
+    while (kcut < n1 && acc < gamma) {
+        acc += m_pool[r[kcut].id];
+        keep[r[kcut].id] = 1;
+        ++kcut;
+    }
+    int n = emit_ascending(i, keep, keep_out);
+    if (k_out) *k_out = kcut;
+    free(r); free(keep);
+    return n;
+}
+
+void oracle_select_practical_rows(int n_tiles, int n_rows, const int* row_h, const int* row_i, const double* m_pool,
+                                  const double* d_pool, double w, double gamma, double rho, int* lists, int* counts,
+                                  int* kcut) {
+#pragma omp parallel for schedule(dynamic, 4)
+    for (int rr = 0; rr < n_rows; ++rr) {
+        size_t off = tri_offset(n_tiles, row_h[rr], row_i[rr]);
+        counts[rr] = oracle_select_practical_row(row_i[rr], m_pool + off, d_pool + off, w, gamma, rho,
+                                                 lists + (size_t)rr * n_tiles, kcut ? kcut + rr : NULL);
+    }
+}
