@@ -13,7 +13,11 @@ Functions carry the C names:
     poem_select_mass_only(m_hat, ref_row_ptr, row_ptr, col_idx, ws, ...)
     bsa_fwd(q, k, v, row_ptr, col_idx, o, ws, lse=None, order=None, block=128)
     poem_check(ws) -> raises on a device-side error
-and ``prefill_layer`` chains the three calls for one attention layer.
+    poem_pooled_workspace_size(shape) -> bytes
+    poem_score_pooled(q, k, v, m_pool, d_pool, ws, ...)
+    poem_select_practical(shape, m_pool, d_pool, w, gamma, rho, row_ptr, col_idx, ws, order=None)
+``prefill_layer`` chains the three exact calls for one attention layer and
+``prefill_layer_practical`` the practical (pooled-estimate) selector's.
 """
 from __future__ import annotations
 
@@ -35,6 +39,7 @@ STATUS = {
 EXPORTED = (
     "poem_workspace_size", "poem_score", "poem_select", "poem_select_mass_only", "bsa_fwd",
     "poem_check", "poem_set_wait_limit_ns", "poem_status_string", "poem_last_error", "poem_select_noalloc",
+    "poem_pooled_workspace_size", "poem_score_pooled", "poem_select_practical",
 )
 
 
@@ -71,6 +76,13 @@ def _load():
     lib.poem_select_mass_only.restype = st
     lib.poem_select_noalloc.argtypes = [sp, vp, vp, ctypes.c_float, vp, vp, i64, vp, vp]
     lib.poem_select_noalloc.restype = st
+    lib.poem_pooled_workspace_size.argtypes = [sp, ctypes.POINTER(sz)]
+    lib.poem_pooled_workspace_size.restype = st
+    lib.poem_score_pooled.argtypes = [sp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.poem_score_pooled.restype = st
+    dbl = ctypes.c_double
+    lib.poem_select_practical.argtypes = [sp, vp, vp, dbl, dbl, dbl, vp, vp, i64, vp, vp, sz, vp]
+    lib.poem_select_practical.restype = st
     lib.bsa_fwd.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.bsa_fwd.restype = st
     lib.poem_check.argtypes = [vp, vp]
@@ -166,6 +178,29 @@ def poem_select_noalloc(shape: Shape, I_hat, m_hat, tau: float, row_ptr, col_idx
            "poem_select_noalloc")
 
 
+def poem_pooled_workspace_size(shape: Shape) -> int:
+    a = ctypes.c_size_t()
+    _raise(_lib.poem_pooled_workspace_size(ctypes.byref(shape), ctypes.byref(a)), "poem_pooled_workspace_size")
+    return a.value
+
+
+def poem_score_pooled(q, k, v, m_pool, d_pool, ws, shape: Shape | None = None, stream=None, **shape_kw):
+    """Pooled estimates m~ and d~ (packed lower-triangular fp32) for the practical selector."""
+    _check_bf16(q, k, v)
+    shape = shape or make_shape(q, k, **shape_kw)
+    _raise(_lib.poem_score_pooled(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(m_pool), _ptr(d_pool),
+                                  _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)), "poem_score_pooled")
+
+
+def poem_select_practical(shape: Shape, m_pool, d_pool, w: float, gamma: float, rho: float, row_ptr, col_idx, ws,
+                          order=None, stream=None):
+    """Two-stage practical selection (mass shortlist, log m~ + w log d~ rerank, pooled-mass threshold gamma)."""
+    _raise(_lib.poem_select_practical(ctypes.byref(shape), _ptr(m_pool), _ptr(d_pool), ctypes.c_double(w),
+                                      ctypes.c_double(gamma), ctypes.c_double(rho), _ptr(row_ptr), _ptr(col_idx),
+                                      col_idx.numel(), _ptr(order), _ptr(ws), ws.numel() * ws.element_size(),
+                                      _stream(stream)), "poem_select_practical")
+
+
 def bsa_fwd(q, k, v, row_ptr, col_idx, o, ws, lse=None, order=None, shape: Shape | None = None, stream=None,
             **shape_kw):
     _check_bf16(q, k, v, o)
@@ -209,16 +244,25 @@ class Layer:
     ws_score: torch.Tensor
     ws_select: torch.Tensor
     ws_fwd: torch.Tensor
+    # practical selector only: pooled estimates and the pooling workspace
+    m_pool: torch.Tensor | None = None
+    d_pool: torch.Tensor | None = None
+    ws_pooled: torch.Tensor | None = None
 
 
-def alloc_layer(q, k, block: int = 128, n_sample: int = 16, with_lse: bool = False) -> Layer:
+def alloc_layer(q, k, block: int = 128, n_sample: int = 16, with_lse: bool = False, practical: bool = False) -> Layer:
     shape = make_shape(q, k, block=block, n_sample=n_sample)
     n, hq, d = q.shape
     T = n // block
     s_b, sel_b, f_b = poem_workspace_size(shape)
     dev = q.device
     ne = n_score_entries(hq, T)
-    return Layer(
+    extra = {}
+    if practical:
+        extra = dict(m_pool=torch.empty(ne, dtype=torch.float32, device=dev),
+                     d_pool=torch.empty(ne, dtype=torch.float32, device=dev),
+                     ws_pooled=alloc_workspace(poem_pooled_workspace_size(shape), dev))
+    return Layer(**extra,
         shape=shape,
         I_hat=torch.empty(ne, dtype=torch.float32, device=dev),
         m_hat=torch.empty(ne, dtype=torch.float32, device=dev),
@@ -239,6 +283,18 @@ def prefill_layer(q, k, v, tau: float, layer: Layer | None = None, block: int = 
     poem_score(q, k, v, layer.I_hat, layer.m_hat, layer.ws_score, shape=layer.shape, stream=stream)
     poem_select(layer.shape, layer.I_hat, layer.m_hat, tau, layer.row_ptr, layer.col_idx, layer.ws_select,
                 order=layer.order, stream=stream)
+    bsa_fwd(q, k, v, layer.row_ptr, layer.col_idx, layer.o, layer.ws_fwd, lse=layer.lse, order=layer.order,
+            shape=layer.shape, stream=stream)
+    return layer
+
+
+def prefill_layer_practical(q, k, v, w: float, gamma: float, rho: float, layer: Layer | None = None,
+                            block: int = 128, stream=None) -> Layer:
+    """Pooled scoring, practical selection and attention for one layer (o in layer.o)."""
+    layer = layer or alloc_layer(q, k, block=block, practical=True)
+    poem_score_pooled(q, k, v, layer.m_pool, layer.d_pool, layer.ws_pooled, shape=layer.shape, stream=stream)
+    poem_select_practical(layer.shape, layer.m_pool, layer.d_pool, w, gamma, rho, layer.row_ptr, layer.col_idx,
+                          layer.ws_select, order=layer.order, stream=stream)
     bsa_fwd(q, k, v, layer.row_ptr, layer.col_idx, layer.o, layer.ws_fwd, lse=layer.lse, order=layer.order,
             shape=layer.shape, stream=stream)
     return layer

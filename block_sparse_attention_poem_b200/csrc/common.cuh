@@ -74,6 +74,34 @@ struct SelectParams {
   int group;
   double tau;
   int mass_only;
+  // Practical selector (pooled estimates): m_hat holds m~, d_pool holds d~.
+  const float* d_pool;
+  double w;      // weight of log d~ in the rerank key
+  double gamma;  // pooled-mass retention threshold
+  double rho;    // stage-1 shortlist fraction of the candidates
+  int practical;
+  DevErr err;
+};
+
+// Mean pooling and pooled score estimates for the practical selector.
+struct PoolParams {
+  const __nv_bfloat16* q;
+  const __nv_bfloat16* k;
+  const __nv_bfloat16* v;
+  int64_t q_stride_tok, q_stride_head;
+  int64_t kv_stride_tok, kv_stride_head;
+  float* q_bar;   // [Hq, T, D] fp32 tile means of the queries
+  float* k_bar;   // [Hkv, T, D] fp32 block means of the keys
+  float* v_bar;   // [Hkv, T, D] fp32 block means of the values
+  float* m_pool;  // packed lower-triangular [Hq, T(T+1)/2]: m~
+  float* d_pool;  //                                          d~
+  int n_q_heads;
+  int n_kv_heads;
+  int n_tiles;
+  int block;
+  int group;
+  int rows_per_cta;  // R: query heads of one KV head handled by one CTA (divides group, <= 8)
+  float scale;       // softmax scale (natural-log domain)
   DevErr err;
 };
 
@@ -83,5 +111,7 @@ cudaError_t launch_bsa_fwd(int head_dim, int block, const CUtensorMap& tmQ, cons
 cudaError_t launch_score(int head_dim, int block, const CUtensorMap& tmQs, const CUtensorMap& tmK,
                          const CUtensorMap& tmV, const ScoreParams& p, cudaStream_t stream);
 cudaError_t launch_select(const SelectParams& p, cudaStream_t stream);
+cudaError_t launch_pooled(int head_dim, const PoolParams& p, cudaStream_t stream);
+int pooled_rows_per_cta(int group, int n_tiles, int head_dim);
 
 }  // namespace poem

@@ -74,6 +74,12 @@ size_t select_ws_bytes(const poem_shape* s, int T) {
 
 size_t fwd_ws_bytes(const poem_shape*, int) { return poem::kWsHeader; }
 
+// Pooled means q~ [Hq, T, D], k~ and v~ [Hkv, T, D] (fp32) after the header.
+size_t pooled_ws_bytes(const poem_shape* s, int T) {
+  const size_t qn = (size_t)s->n_q_heads * T * s->head_dim, kn = (size_t)s->n_kv_heads * T * s->head_dim;
+  return poem::kWsHeader + round_up(qn * sizeof(float), 256) + 2 * round_up(kn * sizeof(float), 256);
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   static std::once_flag once;
@@ -187,14 +193,21 @@ poem_status poem_score(const poem_shape* shape, const poem_bf16* q, const poem_b
   return POEM_OK;
 }
 
+struct PracticalArgs {
+  const float* d_pool;
+  double w, gamma, rho;
+};
+
 static poem_status select_common(const poem_shape* shape, const float* I_hat, const float* m_hat,
                                  const int32_t* ref_row_ptr, double tau, int mass_only, int32_t* row_ptr,
                                  int32_t* col_idx, int64_t col_capacity, int32_t* order, void* ws, size_t ws_bytes,
-                                 void* stream) {
+                                 void* stream, const PracticalArgs* practical = nullptr) {
   Layout L;
   poem_status st = check_shape(shape, &L);
   if (st != POEM_OK) return st;
-  if ((!mass_only && !aligned16(I_hat)) || !aligned16(m_hat) || !aligned16(row_ptr) || !aligned16(ws) ||
+  if (practical && !aligned16(practical->d_pool))
+    return arg_fail(POEM_ERR_INVALID_ARG, "pointers must be non-NULL and 16-byte aligned");
+  if ((!mass_only && !practical && !aligned16(I_hat)) || !aligned16(m_hat) || !aligned16(row_ptr) || !aligned16(ws) ||
       (col_capacity > 0 && !aligned16(col_idx)) || (order && !aligned16(order)) ||
       (mass_only && !aligned16(ref_row_ptr)))
     return arg_fail(POEM_ERR_INVALID_ARG, "pointers must be non-NULL and 16-byte aligned");
@@ -219,6 +232,13 @@ static poem_status select_common(const poem_shape* shape, const float* I_hat, co
   p.group = L.G;
   p.tau = tau;
   p.mass_only = mass_only;
+  if (practical) {
+    p.practical = 1;
+    p.d_pool = practical->d_pool;
+    p.w = practical->w;
+    p.gamma = practical->gamma;
+    p.rho = practical->rho;
+  }
   p.err = dev_err(ws);
   cudaError_t e = poem::launch_select(p, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "poem_select launch");
@@ -238,6 +258,62 @@ poem_status poem_select_mass_only(const poem_shape* shape, const float* m_hat, c
                                   void* ws, size_t ws_bytes, void* stream) {
   return select_common(shape, nullptr, m_hat, ref_row_ptr, 0.0, 1, row_ptr, col_idx, col_capacity, order, ws,
                        ws_bytes, stream);
+}
+
+poem_status poem_pooled_workspace_size(const poem_shape* shape, size_t* pooled_bytes) {
+  Layout L;
+  poem_status st = check_shape(shape, &L);
+  if (st != POEM_OK) return st;
+  if (pooled_bytes) *pooled_bytes = pooled_ws_bytes(shape, L.T);
+  return POEM_OK;
+}
+
+poem_status poem_score_pooled(const poem_shape* shape, const poem_bf16* q, const poem_bf16* k, const poem_bf16* v,
+                              float* m_pool, float* d_pool, void* ws, size_t ws_bytes, void* stream) {
+  Layout L;
+  poem_status st = check_shape(shape, &L);
+  if (st != POEM_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(m_pool) || !aligned16(d_pool) || !aligned16(ws))
+    return arg_fail(POEM_ERR_INVALID_ARG, "pointers must be non-NULL and 16-byte aligned");
+  if (ws_bytes < pooled_ws_bytes(shape, L.T)) return arg_fail(POEM_ERR_WORKSPACE, "pooled workspace too small");
+  const size_t qn = (size_t)shape->n_q_heads * L.T * shape->head_dim;
+  const size_t kn = (size_t)shape->n_kv_heads * L.T * shape->head_dim;
+  uint8_t* base = reinterpret_cast<uint8_t*>(ws) + poem::kWsHeader;
+  poem::PoolParams p{};
+  p.q = reinterpret_cast<const __nv_bfloat16*>(q);
+  p.k = reinterpret_cast<const __nv_bfloat16*>(k);
+  p.v = reinterpret_cast<const __nv_bfloat16*>(v);
+  p.q_stride_tok = shape->q_stride_tok;
+  p.q_stride_head = shape->q_stride_head;
+  p.kv_stride_tok = shape->kv_stride_tok;
+  p.kv_stride_head = shape->kv_stride_head;
+  p.q_bar = reinterpret_cast<float*>(base);
+  p.k_bar = reinterpret_cast<float*>(base + round_up(qn * sizeof(float), 256));
+  p.v_bar = reinterpret_cast<float*>(base + round_up(qn * sizeof(float), 256) + round_up(kn * sizeof(float), 256));
+  p.m_pool = m_pool;
+  p.d_pool = d_pool;
+  p.n_q_heads = shape->n_q_heads;
+  p.n_kv_heads = shape->n_kv_heads;
+  p.n_tiles = L.T;
+  p.block = shape->block;
+  p.group = L.G;
+  p.rows_per_cta = poem::pooled_rows_per_cta(L.G, L.T, shape->head_dim);
+  p.scale = L.scale;
+  p.err = dev_err(ws);
+  cudaError_t e = poem::launch_pooled(shape->head_dim, p, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "poem_score_pooled launch");
+  return POEM_OK;
+}
+
+poem_status poem_select_practical(const poem_shape* shape, const float* m_pool, const float* d_pool, double w,
+                                  double gamma, double rho, int32_t* row_ptr, int32_t* col_idx, int64_t col_capacity,
+                                  int32_t* order, void* ws, size_t ws_bytes, void* stream) {
+  if (!std::isfinite(w) || w < 0.0) return arg_fail(POEM_ERR_INVALID_ARG, "w must be finite and >= 0");
+  if (std::isnan(gamma)) return arg_fail(POEM_ERR_INVALID_ARG, "gamma is NaN");
+  if (!(rho >= 0.0 && rho <= 1.0)) return arg_fail(POEM_ERR_INVALID_ARG, "rho must lie in [0, 1]");
+  PracticalArgs pa{d_pool, w, gamma, rho};
+  return select_common(shape, nullptr, m_pool, nullptr, 0.0, 0, row_ptr, col_idx, col_capacity, order, ws, ws_bytes,
+                       stream, &pa);
 }
 
 poem_status bsa_fwd(const poem_shape* shape, const poem_bf16* q, const poem_bf16* k, const poem_bf16* v,

@@ -12,10 +12,21 @@
 // smaller id and lists are emitted in ascending id order, as in the appendix
 // "Block ordering" of the "Block-Filtered Long-Context Attention" page.
 //
+// The practical selector (pooled estimates m~, d~ of the reading note's
+// Equation (6) paragraph) keeps, per row, the mandatory blocks and the shortest
+// prefix of a two-stage ranking whose pooled mass reaches gamma:
+//   stage 1    candidates ranked by (m~ desc, id asc); the first ceil(rho |Cand|)
+//   stage 2    that shortlist reranked by (log m~ + w log d~ desc, id asc), fp64
+//   threshold  sum_{mandatory} m~ + sum_{prefix} m~ >= gamma (fp64), else the
+//              whole shortlist.
+//
 // Kernels (all on the caller's stream):
 //   select_rows   one CTA per row: bitonic sort of 64-bit keys (~bits(score) : id)
 //                 in shared memory, fp64 suffix scan, min-reduce of the cut,
 //                 ascending compaction into the row's triangular scratch slot.
+//   select_practical_rows  one CTA per row: the stage-1 sort as above, a sort of
+//                 (order-mapped fp64 key, id) pairs, an fp64 prefix scan of the
+//                 masses and a min-reduce of the cut; same compaction.
 //   scan_counts   one CTA: exclusive scan of the list lengths -> row_ptr.
 //   gather_lists  one CTA per row: scratch -> col_idx (bounded by the capacity).
 //   work_order    one CTA per KV head: rows of the head group by list length desc.
@@ -67,6 +78,74 @@ __device__ void bitonic_sort_u32(uint32_t* a, int n) {
       __syncthreads();
     }
   }
+}
+
+// Ascending bitonic sort of n (power of two) (key, id) pairs, lexicographic.
+__device__ void bitonic_sort_pairs(uint64_t* a, uint32_t* id, int n) {
+  for (int k = 2; k <= n; k <<= 1) {
+    for (int jj = k >> 1; jj > 0; jj >>= 1) {
+      for (int t = threadIdx.x; t < n; t += blockDim.x) {
+        const int partner = t ^ jj;
+        if (partner > t) {
+          const bool up = ((t & k) == 0);
+          const uint64_t x = a[t], y = a[partner];
+          const uint32_t ix = id[t], iy = id[partner];
+          const bool gt = (x > y) || (x == y && ix > iy);
+          if (gt == up) {
+            a[t] = y;
+            a[partner] = x;
+            id[t] = iy;
+            id[partner] = ix;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+}
+
+// Unsigned keys whose ascending order is the DESCENDING order of the value
+// (finite or infinite, not NaN); -0 and +0 map to the same key.
+__device__ __forceinline__ uint32_t desc_key_f32(float x) {
+  if (x == 0.f) x = 0.f;
+  const uint32_t b = __float_as_uint(x);
+  const uint32_t asc = (b >> 31) ? ~b : (b | 0x80000000u);
+  return ~asc;
+}
+
+__device__ __forceinline__ uint64_t desc_key_f64(double x) {
+  if (x == 0.0) x = 0.0;
+  const uint64_t b = (uint64_t)__double_as_longlong(x);
+  const uint64_t asc = (b >> 63) ? ~b : (b | 0x8000000000000000ull);
+  return ~asc;
+}
+
+// Stage-2 rank key log m~ + w log d~ in fp64, with log 0 = -inf; a block of zero
+// mass, or of zero deviation when w > 0, ranks last.
+__device__ __forceinline__ double practical_rank_key(float m, float d, double w) {
+  const double lm = (m > 0.f) ? log((double)m) : -INFINITY;
+  const double ld = (d > 0.f) ? log((double)d) : -INFINITY;
+  if (lm == -INFINITY || (w > 0.0 && ld == -INFINITY)) return -INFINITY;
+  return (w == 0.0) ? lm : lm + w * ld;
+}
+
+// Block-wide exclusive prefix scan (sum over lower thread ids) of one double.
+__device__ double block_excl_scan_d(double a, double* tmp) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  double x = a;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const double y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) tmp[warp] = x;
+  double ex = __shfl_up_sync(0xffffffffu, x, 1);
+  if (lane == 0) ex = 0.0;
+  __syncthreads();
+  double wsum = 0.0;
+  for (int w = 0; w < warp; ++w) wsum += tmp[w];
+  __syncthreads();
+  return wsum + ex;
 }
 
 // Block-wide exclusive scan of one int per thread (blockDim.x == kSelThreads).
@@ -129,6 +208,23 @@ __device__ void block_suffix_scan_d2(double a, double b, double* tmpa, double* t
   ea = na + wa;
   eb = nb + wb;
   __syncthreads();
+}
+
+// Ascending compaction of the kept flags of block ids 0..i into the row's
+// triangular scratch slot; the list length goes to counts[row].
+__device__ void emit_row(const SelectParams& p, const int* keep, int row, int i, int64_t off, int* tmpi) {
+  const int n = i + 1;
+  const int E2 = (n + kSelThreads - 1) / kSelThreads;
+  const int b0 = threadIdx.x * E2;
+  const int b1 = min(n, b0 + E2);
+  int cnt = 0;
+  for (int b = b0; b < b1; ++b) cnt += keep[b];
+  int total;
+  int pos = block_excl_scan_int(cnt, tmpi, &total);
+  int32_t* dst = p.scratch + off;
+  for (int b = b0; b < b1; ++b)
+    if (keep[b]) dst[pos++] = b;
+  if (threadIdx.x == 0) p.counts[row] = total;
 }
 
 __global__ void __launch_bounds__(kSelThreads) select_rows_kernel(const SelectParams p) {
@@ -205,19 +301,86 @@ __global__ void __launch_bounds__(kSelThreads) select_rows_kernel(const SelectPa
     if (i >= 1) keep[i - 1] = 1;
   }
   __syncthreads();
-  // Ascending compaction over block ids 0..i.
-  const int n = i + 1;
-  const int E2 = (n + kSelThreads - 1) / kSelThreads;
-  const int b0 = threadIdx.x * E2;
-  const int b1 = min(n, b0 + E2);
-  int cnt = 0;
-  for (int b = b0; b < b1; ++b) cnt += keep[b];
-  int total;
-  int pos = block_excl_scan_int(cnt, tmpi, &total);
-  int32_t* dst = p.scratch + off;
-  for (int b = b0; b < b1; ++b)
-    if (keep[b]) dst[pos++] = b;
-  if (threadIdx.x == 0) p.counts[row] = total;
+  emit_row(p, keep, row, i, off, tmpi);
+}
+
+__global__ void __launch_bounds__(kSelThreads) select_practical_rows_kernel(const SelectParams p) {
+  extern __shared__ __align__(16) uint8_t sm[];
+  const int row = blockIdx.x;
+  const int T = p.n_tiles;
+  const int h = row / T;
+  const int i = row - h * T;
+  const int nc = max(0, i - 2);
+  int P = 1;
+  while (P < nc) P <<= 1;
+  uint64_t* keys = reinterpret_cast<uint64_t*>(sm);                    // [P]
+  uint32_t* ids = reinterpret_cast<uint32_t*>(sm + sizeof(uint64_t) * (size_t)P);  // [P]
+  int* keep = reinterpret_cast<int*>(sm + (sizeof(uint64_t) + sizeof(uint32_t)) * (size_t)P);  // [T]
+  __shared__ double tmpd[kSelThreads / 32];
+  __shared__ int tmpi[kSelThreads / 32];
+  __shared__ int s_kcut;
+
+  const int64_t off = tri_off(T, h, i);
+  const float* mp = p.m_hat + off;
+  const float* dp = p.d_pool + off;
+
+  // Stage 1: candidates by (m~ desc, id asc).
+  for (int t = threadIdx.x; t < P; t += blockDim.x)
+    keys[t] = (t < nc) ? (((uint64_t)desc_key_f32(mp[t + 1]) << 32) | (uint32_t)(t + 1)) : ~0ull;
+  for (int b = threadIdx.x; b <= i; b += blockDim.x) keep[b] = 0;
+  if (nc > 1) {
+    __syncthreads();
+    bitonic_sort_u64(keys, P);
+  }
+  const int n1 = min(nc, max(0, (int)ceil(p.rho * (double)nc)));
+  if (threadIdx.x == 0) s_kcut = n1;
+  int P2 = 1;
+  while (P2 < n1) P2 <<= 1;
+  __syncthreads();
+  // Stage 2: the shortlist by (log m~ + w log d~ desc, id asc); each thread
+  // rewrites only the entries it reads.
+  for (int t = threadIdx.x; t < P2; t += blockDim.x) {
+    if (t < n1) {
+      const uint32_t id = (uint32_t)(keys[t] & 0xffffffffu);
+      ids[t] = id;
+      keys[t] = desc_key_f64(practical_rank_key(mp[id], dp[id], p.w));
+    } else {
+      ids[t] = 0xffffffffu;
+      keys[t] = ~0ull;
+    }
+  }
+  __syncthreads();
+  if (n1 > 1) bitonic_sort_pairs(keys, ids, P2);
+
+  // Threshold: mandatory mass (ascending ids), then the reranked prefix, in fp64.
+  double acc0 = (double)mp[0];
+  if (i >= 2) acc0 += (double)mp[i - 1];
+  if (i >= 1) acc0 += (double)mp[i];
+  const int E = (n1 + kSelThreads - 1) / kSelThreads;
+  const int r0 = min(n1, threadIdx.x * E);
+  const int r1 = min(n1, r0 + E);
+  double loc = 0.0;
+  for (int r = r0; r < r1; ++r) loc += (double)mp[ids[r]];
+  const double carry = block_excl_scan_d(loc, tmpd);
+  double run = acc0 + carry;
+  for (int r = r0; r < r1; ++r) {
+    run += (double)mp[ids[r]];
+    if (run >= p.gamma) {
+      atomicMin(&s_kcut, r + 1);
+      break;
+    }
+  }
+  if (threadIdx.x == 0 && acc0 >= p.gamma) atomicMin(&s_kcut, 0);
+  __syncthreads();
+  const int kcut = s_kcut;
+  for (int r = threadIdx.x; r < kcut; r += blockDim.x) keep[ids[r]] = 1;
+  if (threadIdx.x == 0) {
+    keep[0] = 1;
+    keep[i] = 1;
+    if (i >= 1) keep[i - 1] = 1;
+  }
+  __syncthreads();
+  emit_row(p, keep, row, i, off, tmpi);
 }
 
 // Exclusive scan of counts[0..rows) into row_ptr[0..rows] (single CTA).
@@ -299,14 +462,27 @@ cudaError_t launch_select(const SelectParams& p, cudaStream_t stream) {
   if (rows <= 0) return cudaSuccess;
   int P = 1;
   while (P < p.n_tiles) P <<= 1;
-  const size_t smem = sizeof(uint64_t) * (size_t)P + sizeof(int) * (size_t)p.n_tiles + 16;
-  static size_t configured = 0;
-  if (smem > 48 * 1024 && smem > configured) {
-    cudaError_t e = cudaFuncSetAttribute(select_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    configured = smem;
+  if (p.practical) {
+    const size_t smem = (sizeof(uint64_t) + sizeof(uint32_t)) * (size_t)P + sizeof(int) * (size_t)p.n_tiles + 16;
+    static size_t pconf = 0;
+    if (smem > 48 * 1024 && smem > pconf) {
+      cudaError_t e =
+          cudaFuncSetAttribute(select_practical_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e != cudaSuccess) return e;
+      pconf = smem;
+    }
+    select_practical_rows_kernel<<<rows, kSelThreads, smem, stream>>>(p);
+  } else {
+    const size_t smem = sizeof(uint64_t) * (size_t)P + sizeof(int) * (size_t)p.n_tiles + 16;
+    static size_t configured = 0;
+    if (smem > 48 * 1024 && smem > configured) {
+      cudaError_t e =
+          cudaFuncSetAttribute(select_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e != cudaSuccess) return e;
+      configured = smem;
+    }
+    select_rows_kernel<<<rows, kSelThreads, smem, stream>>>(p);
   }
-  select_rows_kernel<<<rows, kSelThreads, smem, stream>>>(p);
   scan_counts_kernel<<<1, 1024, 0, stream>>>(p.counts, p.row_ptr, rows);
   gather_lists_kernel<<<rows, 128, 0, stream>>>(p);
   if (p.order) {

@@ -166,6 +166,52 @@ poem_status poem_select_noalloc(const poem_shape* shape, const float* I_hat, con
                                 void* stream);
 
 /*
+ * Practical POEM selector (reading note "Attention deletion error", the
+ * paragraph on Equation (6) and Appendix B): the dense reference output and the
+ * block outputs are estimated from pooled features, candidates are preselected
+ * by mass, reranked by log mass + w * log deviation, and kept in that order
+ * until the accumulated pooled mass reaches a threshold.  The pages print
+ * neither the estimators nor w; this library's estimators are mean pooling:
+ *   q~_{h,i}  mean of the B queries of tile i, head h
+ *   k~_{g,b}, v~_{g,b}  means of the B keys / values of block b, KV head g
+ *   m~[h, i, b] = softmax over b <= i of softmax_scale * <q~_{h,i}, k~_{g,b}>
+ *   o~ = sum_b m~ v~_b,   d~[h, i, b] = || v~_b - o~ ||
+ * (with one token per block and one query per tile these are the exact m_b and
+ * ||v_b - o||).
+ */
+
+/* Workspace bytes of poem_score_pooled (256-byte header, then fp32 q~, k~, v~). */
+poem_status poem_pooled_workspace_size(const poem_shape* shape, size_t* pooled_bytes);
+
+/*
+ * poem_score_pooled -- m~ and d~ for every (head, tile, visible block).
+ * Outputs (fp32, packed lower-triangular like poem_score's): entry (h, i, b) at
+ *   h*T*(T+1)/2 + i*(i+1)/2 + b.  fp32 arithmetic throughout.
+ * ws: at least pooled_bytes; holds the pooled means after the call.
+ * n_sample is ignored.
+ */
+poem_status poem_score_pooled(const poem_shape* shape, const poem_bf16* q, const poem_bf16* k, const poem_bf16* v,
+                              float* m_pool, float* d_pool, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * poem_select_practical -- two-stage selection per (head, tile) from m~, d~.
+ * Row r = h*T + i.  Mandatory: blocks 0, i-1 (i >= 1) and i.  Candidates
+ * 1..i-2:
+ *   stage 1: ranked by (m~ desc, id asc); the first ceil(rho * |Cand|) form the
+ *            shortlist (rho in [0, 1]);
+ *   stage 2: the shortlist ranked by (log m~ + w * log d~ desc, id asc), in
+ *            fp64 with log 0 = -inf (w finite, >= 0);
+ *   the row keeps the mandatory blocks and the shortest prefix of the stage-2
+ *   order with  sum_{mandatory} m~ + sum_{prefix} m~ >= gamma  (fp64; the
+ *   whole shortlist when the sum never reaches gamma).
+ * Outputs, col_capacity, order and workspace: as poem_select (select_bytes).
+ * NaN gamma, rho outside [0, 1] or a negative / non-finite w: INVALID_ARG.
+ */
+poem_status poem_select_practical(const poem_shape* shape, const float* m_pool, const float* d_pool, double w,
+                                  double gamma, double rho, int32_t* row_ptr, int32_t* col_idx,
+                                  int64_t col_capacity, int32_t* order, void* ws, size_t ws_bytes, void* stream);
+
+/*
  * bsa_fwd -- causal GQA block-sparse attention forward.
  * Query t of head h in tile i attends, with softmax, to the keys u <= t whose
  * block is listed in col_idx[row_ptr[r] .. row_ptr[r+1]), r = h*T + i

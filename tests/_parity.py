@@ -43,6 +43,26 @@ def compare_fwd(o_gpu: torch.Tensor, O_ref: np.ndarray, units, block: int):
     return float(e.max()), float(e.mean())
 
 
+# bsa_fwd writes O in bf16: rounding to nearest bf16 (8-bit significand) moves a
+# value x by at most 2^-8 |x|, which alone exceeds FWD_MAX_ABS once |x| > 2.56.
+BF16_ROUND_REL = 2.0 ** -8
+
+
+def compare_fwd_excess(o_gpu: torch.Tensor, O_ref: np.ndarray, units, block: int):
+    """Like compare_fwd, but the element bound adds the bf16 output rounding:
+    |o_gpu - o_ref| <= FWD_MAX_ABS + BF16_ROUND_REL |o_ref|.  Returns (largest
+    violation ratio (<= 1 passes), mean_abs)."""
+    og = o_gpu.float().cpu().numpy()
+    worst, tot, cnt = 0.0, 0.0, 0
+    for u, (h, i) in enumerate(units):
+        ref = O_ref[u]
+        e = np.abs(og[i * block:(i + 1) * block, h, :] - ref)
+        worst = max(worst, float(np.max(e / (FWD_MAX_ABS + BF16_ROUND_REL * np.abs(ref)))))
+        tot += float(e.sum())
+        cnt += e.size
+    return worst, tot / cnt
+
+
 def score_err_excess(gpu_I, ref_I, gpu_m, ref_m, R: float):
     """Largest violation ratio of the score tolerances (<= 1 passes):
       |dI_b| <= SCORE_REL * I_b + 1e-5 * m_b * R
@@ -100,4 +120,95 @@ def lists_agree_at_cut(gpu_rows, ref_rows, Ihat_ref, mhat_ref, n_q_heads, n_tile
                         ok_slack = True
             if not ok_slack:
                 bad.append((h, i, sorted(a - b), sorted(b - a)))
+    return differ, bad
+
+
+# ---------------------------------------------------------------------------
+# Practical (pooled-estimate) selector
+# ---------------------------------------------------------------------------
+
+# Pooled estimates m~, d~ are formed in fp32 from fp32 tile/block means:
+#   |dm| <= POOL_REL * m + 1e-9,   |dd| <= POOL_REL * d + 1e-5 * max ||v~||
+# (the absolute term covers d~ near 0, where fp32 cancellation leaves ~1e-6 |v~|).
+POOL_REL = 1e-4
+
+
+def pooled_err_excess(gpu_m, ref_m, gpu_d, ref_d, vbar_norm: float):
+    gm, rm = np.asarray(gpu_m, np.float64), np.asarray(ref_m, np.float64)
+    gd, rd = np.asarray(gpu_d, np.float64), np.asarray(ref_d, np.float64)
+    tolm = POOL_REL * rm + 1e-9
+    told = POOL_REL * rd + 1e-5 * vbar_norm + 1e-30
+    return float(max(np.max(np.abs(gm - rm) / tolm), np.max(np.abs(gd - rd) / told)))
+
+
+def _practical_keys(m, d, w):
+    with np.errstate(divide="ignore"):
+        lm = np.where(m > 0, np.log(np.where(m > 0, m, 1.0)), -np.inf)
+        ld = np.where(d > 0, np.log(np.where(d > 0, d, 1.0)), -np.inf)
+    if w == 0:
+        return lm
+    key = lm + w * np.where(np.isfinite(ld), ld, 0.0)
+    return np.where((lm == -np.inf) | (ld == -np.inf), -np.inf, key)
+
+
+def practical_row_ambiguous(i, m, d, w, gamma, rho, band_m, band_key, band_acc):
+    """True when a perturbation of the row's estimates within the bands could change
+    its kept set: a near-tie at the stage-1 shortlist boundary (relative band_m), a
+    near-tie of the stage-2 keys across the cut (absolute band_key, log domain), or
+    an accumulated mass within band_acc of gamma at the cut."""
+    m = np.asarray(m, np.float64)
+    d = np.asarray(d, np.float64)
+    cand = np.arange(1, max(i - 1, 1), dtype=np.int64) if i >= 3 else np.zeros(0, np.int64)
+    nc = cand.size
+    o1 = cand[np.lexsort((cand, -m[cand]))] if nc else cand
+    n1 = min(nc, max(0, int(np.ceil(rho * nc))))
+    if 0 < n1 < nc and abs(m[o1[n1 - 1]] - m[o1[n1]]) <= band_m * max(m[o1[n1 - 1]], 1e-300):
+        return True
+    sl = o1[:n1]
+    key = _practical_keys(m[sl], d[sl], w)
+    o2 = sl[np.lexsort((sl, -key))]
+    k2 = _practical_keys(m[o2], d[o2], w)
+    acc = m[0]
+    if i >= 2:
+        acc += m[i - 1]
+    if i >= 1:
+        acc += m[i]
+    accs = [acc]
+    for b in o2:
+        acc += m[b]
+        accs.append(acc)
+    kcut = next((k for k, a in enumerate(accs) if a >= gamma), n1)
+    for k in (kcut - 1, kcut):
+        if 0 <= k <= n1 and abs(accs[k] - gamma) <= band_acc:
+            return True
+    if 0 < kcut < n1 and np.isfinite(k2[kcut - 1]) and abs(k2[kcut - 1] - k2[kcut]) <= band_key:
+        return True
+    return False
+
+
+def check_list_valid(rows, n_tiles):
+    """Every row ascending, unique, within 0..i and holding the mandatory blocks."""
+    for r, row in enumerate(rows):
+        i = r % n_tiles
+        assert row == sorted(set(row)), r
+        assert all(0 <= b <= i for b in row), r
+        mand = {0, i} | ({i - 1} if i >= 1 else set())
+        assert mand <= set(row), r
+
+
+def practical_lists_agree(gpu_rows, ref_rows, m_ref, d_ref, n_q_heads, n_tiles, w, gamma, rho, band_m, band_key,
+                          band_acc, rows=None):
+    """Rows must match exactly unless practical_row_ambiguous flags them on the
+    reference estimates.  Returns (n_rows_differing, violations)."""
+    bad, differ = [], 0
+    rows = range(n_q_heads * n_tiles) if rows is None else rows
+    for r in rows:
+        if list(gpu_rows[r]) == list(ref_rows[r]):
+            continue
+        differ += 1
+        h, i = divmod(r, n_tiles)
+        off = oracle.tri_offset(n_tiles, h, i)
+        if not practical_row_ambiguous(i, m_ref[off:off + i + 1], d_ref[off:off + i + 1], w, gamma, rho, band_m,
+                                       band_key, band_acc):
+            bad.append((h, i, sorted(set(gpu_rows[r]) - set(ref_rows[r])), sorted(set(ref_rows[r]) - set(gpu_rows[r]))))
     return differ, bad

@@ -114,3 +114,41 @@ def test_select_rejects_small_workspace_and_negative_capacity(poem):
 def test_status_strings(poem):
     for code, name in poem.STATUS.items():
         assert poem.poem_status_string(code) == name
+
+
+def test_pooled_workspace_size(poem):
+    sh = _shape(poem)
+    a = ctypes.c_size_t()
+    assert poem._lib.poem_pooled_workspace_size(ctypes.byref(sh), ctypes.byref(a)) == 0
+    T, hq, hkv, d = 8, 4, 2, 128
+    assert a.value >= 256 + (hq + 2 * hkv) * T * d * 4
+    assert poem._lib.poem_pooled_workspace_size(ctypes.byref(_shape(poem, head_dim=96)), ctypes.byref(a)) == 2
+
+
+def test_score_pooled_rejects_bad_pointers_and_workspace(poem):
+    sh = _shape(poem)
+    ok = ctypes.c_void_p(1 << 20)
+    mis = ctypes.c_void_p((1 << 20) + 4)
+    assert poem._lib.poem_score_pooled(ctypes.byref(sh), ok, ok, ok, None, ok, ok, 1 << 30, None) == 1
+    assert poem._lib.poem_score_pooled(ctypes.byref(sh), ok, mis, ok, ok, ok, ok, 1 << 30, None) == 1
+    assert poem._lib.poem_score_pooled(ctypes.byref(sh), ok, ok, ok, ok, ok, ok, 300, None) == 6
+
+
+@pytest.mark.parametrize("w,gamma,rho", [(-1.0, 0.9, 0.5), (math.inf, 0.9, 0.5), (math.nan, 0.9, 0.5),
+                                         (1.0, math.nan, 0.5), (1.0, 0.9, 1.01), (1.0, 0.9, -0.5),
+                                         (1.0, 0.9, math.nan)])
+def test_select_practical_rejects_bad_parameters(poem, w, gamma, rho):
+    sh = _shape(poem)
+    ok = ctypes.c_void_p(1 << 20)
+    st = poem._lib.poem_select_practical(ctypes.byref(sh), ok, ok, w, gamma, rho, ok, ok, 100, None, ok, 1 << 30,
+                                         None)
+    assert st == 1
+
+
+def test_select_practical_rejects_null_deviation_and_small_workspace(poem):
+    sh = _shape(poem)
+    ok = ctypes.c_void_p(1 << 20)
+    assert poem._lib.poem_select_practical(ctypes.byref(sh), ok, None, 1.0, 0.9, 0.5, ok, ok, 100, None, ok, 1 << 30,
+                                           None) == 1
+    assert poem._lib.poem_select_practical(ctypes.byref(sh), ok, ok, 1.0, 0.9, 0.5, ok, ok, 100, None, ok, 8,
+                                           None) == 6
