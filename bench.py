@@ -8,6 +8,11 @@ synthetic Q/K/V from seed 0, tau = 0.05).  One step = poem_score + poem_select
 than L2, so no flush is needed between steps).  Prints one JSON line.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--selector exact|practical [--w W --gamma G --rho R]]
+
+--selector practical times the practical selector instead (poem_score_pooled +
+poem_select_practical + bsa_fwd; pooled estimates, mass shortlist rho, rerank
+log m~ + w log d~, pooled-mass threshold gamma).
 
 With N > 1 (torchrun, one rank per GPU) every rank runs an independent replica
 of the layer (the path needs no exchange step); the reported ms/layer is the
@@ -90,7 +95,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
         except (OSError, FileNotFoundError):
@@ -188,17 +193,26 @@ def run_ours(args):
     T = n // B
     x = poem_synth.heavy_block_layer(n, hq, hkv, d, block=B, rope_base=base, seed=args.seed)
     q, k, v = x["q"].to(dev), x["k"].to(dev), x["v"].to(dev)
-    layer = poem.alloc_layer(q, k, block=B)
+    practical = args.selector == "practical"
+    layer = poem.alloc_layer(q, k, block=B, practical=practical)
     stream = torch.cuda.current_stream(dev)
+    ws_first = layer.ws_pooled if practical else layer.ws_score
 
     def step(ev=None):
         if ev:
             ev[0].record(stream)
-        poem.poem_score(q, k, v, layer.I_hat, layer.m_hat, layer.ws_score, shape=layer.shape)
+        if practical:
+            poem.poem_score_pooled(q, k, v, layer.m_pool, layer.d_pool, layer.ws_pooled, shape=layer.shape)
+        else:
+            poem.poem_score(q, k, v, layer.I_hat, layer.m_hat, layer.ws_score, shape=layer.shape)
         if ev:
             ev[1].record(stream)
-        poem.poem_select(layer.shape, layer.I_hat, layer.m_hat, tau, layer.row_ptr, layer.col_idx, layer.ws_select,
-                         order=layer.order)
+        if practical:
+            poem.poem_select_practical(layer.shape, layer.m_pool, layer.d_pool, args.w, args.gamma, args.rho,
+                                       layer.row_ptr, layer.col_idx, layer.ws_select, order=layer.order)
+        else:
+            poem.poem_select(layer.shape, layer.I_hat, layer.m_hat, tau, layer.row_ptr, layer.col_idx,
+                             layer.ws_select, order=layer.order)
         if ev:
             ev[2].record(stream)
         poem.bsa_fwd(q, k, v, layer.row_ptr, layer.col_idx, layer.o, layer.ws_fwd, order=layer.order,
@@ -209,7 +223,7 @@ def run_ours(args):
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
-    for ws in (layer.ws_score, layer.ws_select, layer.ws_fwd):
+    for ws in (ws_first, layer.ws_select, layer.ws_fwd):
         poem.poem_check(ws)
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
@@ -236,12 +250,15 @@ def run_ours(args):
     ms_per_step = total_ms / args.steps
     ms_per_layer = whole_job_ms_per_layer(total_ms, args.steps, world)
 
-    for ws in (layer.ws_score, layer.ws_select, layer.ws_fwd):
+    for ws in (ws_first, layer.ws_select, layer.ws_fwd):
         poem.poem_check(ws)
     rp = layer.row_ptr.cpu().numpy()
     ci = layer.col_idx[: int(rp[-1])].cpu().numpy()
     kept = int(rp[-1])
     visible = hq * T * (T + 1) // 2
+    if practical:  # exact masses (untimed) for the heavy-mass figure and the mass-only comparison
+        poem.poem_score(q, k, v, layer.I_hat, layer.m_hat, layer.ws_score, shape=layer.shape)
+        poem.poem_check(layer.ws_score)
     # realised heavy-mass fraction: visible (head, tile, block) with m_hat > 10 / (i + 1)
     mh = layer.m_hat.cpu().numpy()
     tile_of = np.tile(np.repeat(np.arange(T), np.arange(1, T + 1)), hq)
@@ -250,7 +267,10 @@ def run_ours(args):
     dflops = dense_flops(n, hq, d)
     peaks, peak_src = load_peaks()
     fwd_tflops = rflops / (fwd_ms * 1e-3) / 1e12
-    traffic, traffic_note = bsa_fwd_traffic() if args.workload == "llama3.1-8b-layer-128k" else (None, "no capture")
+    if args.workload == "llama3.1-8b-layer-128k" and not practical:
+        traffic, traffic_note = bsa_fwd_traffic()
+    else:
+        traffic, traffic_note = None, "no ncu capture of bsa_fwd on these lists"
 
     # end-to-end through the public API with host buffers: H2D of Q/K/V from pinned
     # memory, the three calls, D2H of O, every step.
@@ -282,12 +302,18 @@ def run_ours(args):
     extra = {}
     if not args.no_quality and rank == 0:
         extra = quality_report(poem, q, k, v, layer, tau, n, hq, T, B, dev)
+        if practical:
+            extra["err_vs_dense"]["practical"] = extra["err_vs_dense"].pop("poem")
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(x, n, hq, hkv, d, B, tau, args.cpu_budget_s)
+        cpu = (cpu_baseline_practical(x, n, hq, hkv, d, B, args.w, args.gamma, args.rho, args.cpu_budget_s)
+               if practical else cpu_baseline(x, n, hq, hkv, d, B, tau, args.cpu_budget_s))
+    sel_cfg = ({"selector": "practical", "w": args.w, "gamma": args.gamma, "rho": args.rho} if practical
+               else {"selector": "exact", "tau": tau})
+    names = (("poem_score_pooled", "poem_select_practical") if practical else ("poem_score", "poem_select"))
 
-    launches_per_step = 2 + 3 + 1 + 1  # score(2) + select(3 + order) + bsa_fwd
+    launches_per_step = 2 + 3 + 1 + 1  # score(2 passes | pool + pooled scores) + select(3 + order) + bsa_fwd
     line = {
         "metric": METRIC,
         "value": round(ms_per_layer, 4),
@@ -302,10 +328,10 @@ def run_ours(args):
         "dtype": "bf16",
         "data": "synthetic (seeded heavy-block generator; no model weights or datasets)",
         "config": {"workload": args.workload, "n_tokens": n, "n_q_heads": hq, "n_kv_heads": hkv, "head_dim": d,
-                   "block": B, "n_sample": 16, "tau": tau, "seed": args.seed,
+                   "block": B, "n_sample": 16, **sel_cfg, "seed": args.seed,
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "l2": "inputs larger than L2 (no flush needed)"},
-        "breakdown_ms": {"poem_score": round(score_ms, 4), "poem_select": round(select_ms, 4),
+        "breakdown_ms": {names[0]: round(score_ms, 4), names[1]: round(select_ms, 4),
                          "bsa_fwd": round(fwd_ms, 4)},
         "density": round(kept / visible, 5),
         "heavy_mass_block_fraction": round(heavy_frac, 4),
@@ -406,6 +432,40 @@ def cpu_baseline(x, n, hq, hkv, d, B, tau, budget_s):
             "extrapolated": True}
 
 
+def cpu_baseline_practical(x, n, hq, hkv, d, B, w, gamma, rho, budget_s):
+    """Oracle (fp64, host cores) of the practical path on a bounded sample of
+    (head, tile) units -- pooled estimates, practical selection, masked attention
+    -- scaled to a whole layer by visible blocks per unit."""
+    import oracle
+
+    oracle.build()
+    T = n // B
+    prob = oracle.Problem(q=poem_synth.bf16_bits(x["q"]), k=poem_synth.bf16_bits(x["k"]),
+                          v=poem_synth.bf16_bits(x["v"]), block=B, n_sample=16)
+    units, per_unit, t_total, h = [], [], 0.0, 0
+    for f in (1 / 16, 1 / 8, 1 / 4, 1 / 2, 1.0):
+        if t_total > budget_s:
+            break
+        i = max(0, int(T * f) - 1)
+        t0 = time.perf_counter()
+        mp, dp = prob.pooled_units([(h, i)])
+        off = oracle.tri_offset(T, h, i)
+        keep, _ = oracle.select_practical_row(i, mp[off:off + i + 1], dp[off:off + i + 1], w, gamma, rho)
+        rp = np.zeros(hq * T + 1, dtype=np.int32)
+        rp[h * T + i + 1:] = len(keep)
+        prob.masked_units([(h, i)], rp, np.asarray(keep, dtype=np.int32))
+        dt = time.perf_counter() - t0
+        t_total += dt
+        units.append((h, i))
+        per_unit.append(dt / (i + 1))
+        h = (h + 1) % hq
+    est_ms = float(np.mean(per_unit)) * hq * T * (T + 1) / 2 * 1e3
+    return {"value": round(est_ms, 1), "unit": "ms/layer", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{len(units)} (head, tile) units at tiles {[u[1] for u in units]} (pooled estimates + "
+                      f"practical selection + masked attention), {t_total:.1f} s, scaled by visible blocks per "
+                      f"unit to the whole layer", "extrapolated": True}
+
+
 def run_reference(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -416,8 +476,10 @@ def run_reference(args):
     budget = max(2.0, args.ref_step_budget_s)
     vals = []
     cb = None
+    practical = args.selector == "practical"
     for s in range(args.warmup + args.steps):
-        cb = cpu_baseline(x, n, hq, hkv, d, B, tau, budget)
+        cb = (cpu_baseline_practical(x, n, hq, hkv, d, B, args.w, args.gamma, args.rho, budget) if practical
+              else cpu_baseline(x, n, hq, hkv, d, B, tau, budget))
         if s >= args.warmup:
             vals.append(cb["value"])
     v = float(np.mean(vals))
@@ -426,7 +488,9 @@ def run_reference(args):
         "warmup": args.warmup, "ms_per_step": round(v, 1), "higher_is_better": False, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded heavy-block generator)",
         "config": {"workload": args.workload, "n_tokens": n, "n_q_heads": hq, "n_kv_heads": hkv, "head_dim": d,
-                   "block": B, "n_sample": 16, "tau": tau, "seed": args.seed},
+                   "block": B, "n_sample": 16,
+                   **({"selector": "practical", "w": args.w, "gamma": args.gamma, "rho": args.rho} if practical
+                      else {"selector": "exact", "tau": tau}), "seed": args.seed},
         "impl": "reference",
         "cpu_baseline": {"value": round(v, 1), "unit": "ms/layer", "cores": cb["cores"], "kind": "oracle",
                          "sample": cb["sample"]},
@@ -555,18 +619,143 @@ def _report_sweep(poem, steps, warmup):
     return out
 
 
+PRACTICAL_REPORT = [
+    # (workload, [(w, gamma, rho), ...])
+    ("llama3.1-8b-layer-32k", [(1.0, 0.9, 0.5), (1.0, 0.95, 0.5), (1.0, 0.99, 0.5), (0.0, 0.95, 0.5)]),
+    ("llama3.1-8b-layer-128k", [(1.0, 0.9, 0.5), (1.0, 0.95, 0.5), (1.0, 0.99, 0.5), (0.0, 0.95, 0.5)]),
+]
+
+
+def _stage_diagnostics(m_pool, I_hat, row_ptr, col_idx, rho, hq, T, heads):
+    """For the rows of `heads`: the candidates POEM's exact ranking keeps at the
+    practical list's budget but the practical list drops, split into those the
+    stage-1 mass shortlist excluded and those stage 2 ranked below the cut."""
+    mp = m_pool.cpu().numpy()
+    Ih = I_hat.cpu().numpy()
+    rp = row_ptr.cpu().numpy()
+    ci = col_idx[: int(rp[-1])].cpu().numpy()
+    excl = misrank = kept_free = 0
+    for h in heads:
+        for i in range(3, T):
+            r = h * T + i
+            keep = set(ci[rp[r]:rp[r + 1]].tolist())
+            off = h * (T * (T + 1) // 2) + i * (i + 1) // 2
+            cand = np.arange(1, i - 1)
+            free = len(keep) - 3
+            kept_free += free
+            if free <= 0:
+                continue
+            top_I = cand[np.lexsort((cand, -Ih[off + cand]))][:free]
+            n1 = min(cand.size, int(math.ceil(rho * cand.size)))
+            short = set(cand[np.lexsort((cand, -mp[off + cand]))][:n1].tolist())
+            for b in top_I.tolist():
+                if b not in keep:
+                    if b in short:
+                        misrank += 1
+                    else:
+                        excl += 1
+    return {"rows": len(heads) * max(T - 3, 0), "free_blocks_kept": kept_free,
+            "exact_topk_missed_stage1_excluded": excl, "exact_topk_missed_stage2_misranked": misrank}
+
+
+def _report_practical(poem, wl, params, steps, warmup):
+    n, hq, hkv, d, B, base, _ = WORKLOADS[wl]
+    x = poem_synth.heavy_block_layer(n, hq, hkv, d, block=B, rope_base=base, seed=0)
+    T = n // B
+    q, k, v = x["q"].cuda(), x["k"].cuda(), x["v"].cuda()
+    layer = poem.alloc_layer(q, k, block=B, practical=True)
+    poem.poem_score(q, k, v, layer.I_hat, layer.m_hat, layer.ws_score, shape=layer.shape)  # exact, for comparisons
+    poem.poem_check(layer.ws_score)
+    peaks, _ = load_peaks()
+    visible = hq * T * (T + 1) // 2
+    out = []
+    for w, gamma, rho in params:
+        ph = {"poem_score_pooled": [], "poem_select_practical": [], "bsa_fwd": []}
+        for it in range(warmup + steps):
+            ev = _events(4)
+            ev[0].record()
+            poem.poem_score_pooled(q, k, v, layer.m_pool, layer.d_pool, layer.ws_pooled, shape=layer.shape)
+            ev[1].record()
+            poem.poem_select_practical(layer.shape, layer.m_pool, layer.d_pool, w, gamma, rho, layer.row_ptr,
+                                       layer.col_idx, layer.ws_select, order=layer.order)
+            ev[2].record()
+            poem.bsa_fwd(q, k, v, layer.row_ptr, layer.col_idx, layer.o, layer.ws_fwd, order=layer.order,
+                         shape=layer.shape)
+            ev[3].record()
+            torch.cuda.synchronize()
+            if it >= warmup:
+                for j, key in enumerate(ph):
+                    ph[key].append(ev[j].elapsed_time(ev[j + 1]))
+        for ws in (layer.ws_pooled, layer.ws_select, layer.ws_fwd):
+            poem.poem_check(ws)
+        ms = {key: float(np.median(val)) for key, val in ph.items()}
+        rp = layer.row_ptr.cpu().numpy()
+        ci = layer.col_idx[: int(rp[-1])].cpu().numpy()
+        rfl = retained_flops(rp, ci, T, d, B)
+        fwd_tf = rfl / (ms["bsa_fwd"] * 1e-3) / 1e12
+        # pooled scoring reads Q, K, V once (bf16) and writes m~, d~ (fp32)
+        pooled_bytes = 2.0 * n * (hq + 2 * hkv) * d + 8.0 * visible
+        rec = {"config": f"practical-{wl}", "w": w, "gamma": gamma, "rho": rho, "n_tokens": n,
+               "ms": {key: round(val, 4) for key, val in ms.items()}, "ms_per_layer": round(sum(ms.values()), 4),
+               "density": round(int(rp[-1]) / visible, 5),
+               "bsa_fwd_retained_tflops": round(fwd_tf, 2),
+               "bsa_fwd_frac_sustained": round(fwd_tf / peaks["bf16_tflops_sustained"], 4),
+               "pooled_gbs": round(pooled_bytes / (ms["poem_score_pooled"] * 1e-3) / 1e9, 1)}
+        q_err = quality_report(poem, q, k, v, layer, 0.0, n, hq, T, B, q.device)["err_vs_dense"]
+        rec["err_vs_dense"] = {"practical": q_err["poem"], "mass_only_same_budget": q_err["mass_only_same_budget"]}
+        # exact-score ranking at the same per-row budget
+        rp_i = torch.empty_like(layer.row_ptr)
+        ci_i = torch.empty_like(layer.col_idx)
+        poem.poem_select_ranked_budget(layer.shape, layer.I_hat, layer.row_ptr, rp_i, ci_i, layer.ws_select)
+        o_i = torch.empty_like(q)
+        poem.bsa_fwd(q, k, v, rp_i, ci_i, o_i, layer.ws_fwd, shape=layer.shape)
+        torch.cuda.synchronize()
+        poem.poem_check(layer.ws_select)
+        o_dense = _dense_output(poem, q, k, v, layer, hq, T)
+        diff = o_i.float() - o_dense.float()
+        rec["err_vs_dense"]["exact_I_same_budget"] = {
+            "max_abs": float(diff.abs().max()), "mean_abs": float(diff.abs().mean()),
+            "rel_fro": float(diff.norm() / o_dense.float().norm()), "max_row_l2": float(diff.norm(dim=-1).max())}
+        del o_i, o_dense, diff
+        rec["stage_diagnostics"] = _stage_diagnostics(layer.m_pool, layer.I_hat, layer.row_ptr, layer.col_idx, rho,
+                                                      hq, T, heads=[0, hq // 2])
+        out.append(rec)
+    del layer, q, k, v
+    torch.cuda.empty_cache()
+    return out
+
+
+def _dense_output(poem, q, k, v, layer, hq, T):
+    rp_all, ci_all = poem_synth.random_block_lists(1, T, 1.0, seed=0)
+    counts = np.diff(rp_all)
+    rpd = torch.from_numpy(np.concatenate([[0], np.cumsum(np.tile(counts, hq))]).astype(np.int32)).to(q.device)
+    cid = torch.from_numpy(np.tile(ci_all, hq).astype(np.int32)).to(q.device)
+    o = torch.empty_like(q)
+    poem.bsa_fwd(q, k, v, rpd, cid, o, layer.ws_fwd, shape=layer.shape)
+    torch.cuda.synchronize()
+    poem.poem_check(layer.ws_fwd)
+    return o
+
+
 def run_report(args):
     import block_sparse_attention_poem_b200 as poem
 
     torch.cuda.set_device(0)
     clocks = ClockSampler(0)
     clocks.start()
-    for name, wl, taus, mass_only in REPORT_LAYERS:
-        for tau in taus:
-            rec = _report_layer(poem, name, wl, tau, args.steps, args.warmup, mass_only, args.cpu_budget_s)
+    part = args.report_only
+    if part in (None, "exact"):
+        for name, wl, taus, mass_only in REPORT_LAYERS:
+            for tau in taus:
+                rec = _report_layer(poem, name, wl, tau, args.steps, args.warmup, mass_only, args.cpu_budget_s)
+                print(json.dumps(rec), flush=True)
+    if part in (None, "practical"):
+        for wl, params in PRACTICAL_REPORT:
+            for rec in _report_practical(poem, wl, params, args.steps, args.warmup):
+                print(json.dumps(rec), flush=True)
+    if part in (None, "sweep"):
+        for rec in _report_sweep(poem, args.steps, args.warmup):
             print(json.dumps(rec), flush=True)
-    for rec in _report_sweep(poem, args.steps, args.warmup):
-        print(json.dumps(rec), flush=True)
     print(json.dumps({"config": "clocks", "clocks": clocks.stop()}), flush=True)
 
 
@@ -584,8 +773,14 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget-s", type=float, default=15.0)
     ap.add_argument("--ref-step-budget-s", type=float, default=8.0)
+    ap.add_argument("--selector", choices=["exact", "practical"], default="exact")
+    ap.add_argument("--w", type=float, default=1.0, help="practical: weight of log d~ in the rerank key")
+    ap.add_argument("--gamma", type=float, default=0.95, help="practical: pooled-mass retention threshold")
+    ap.add_argument("--rho", type=float, default=0.5, help="practical: stage-1 shortlist fraction")
     ap.add_argument("--report", action="store_true",
                     help="measure every configuration (one JSON record each) instead of the benchmark line")
+    ap.add_argument("--report-only", choices=["exact", "practical", "sweep"], default=None,
+                    help="with --report: only this part")
     args = ap.parse_args()
     if args.report:
         run_report(args)

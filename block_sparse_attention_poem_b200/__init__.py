@@ -11,6 +11,7 @@ Functions carry the C names:
     poem_score(q, k, v, I_hat, m_hat, ws, block=128, n_sample=16, scale=0.0)
     poem_select(I_hat, m_hat, tau, row_ptr, col_idx, ws, shape..., order=None)
     poem_select_mass_only(m_hat, ref_row_ptr, row_ptr, col_idx, ws, ...)
+    poem_select_ranked_budget(shape, score, ref_row_ptr, row_ptr, col_idx, ws, ...)
     bsa_fwd(q, k, v, row_ptr, col_idx, o, ws, lse=None, order=None, block=128)
     poem_check(ws) -> raises on a device-side error
     poem_pooled_workspace_size(shape) -> bytes
@@ -39,7 +40,7 @@ STATUS = {
 EXPORTED = (
     "poem_workspace_size", "poem_score", "poem_select", "poem_select_mass_only", "bsa_fwd",
     "poem_check", "poem_set_wait_limit_ns", "poem_status_string", "poem_last_error", "poem_select_noalloc",
-    "poem_pooled_workspace_size", "poem_score_pooled", "poem_select_practical",
+    "poem_pooled_workspace_size", "poem_score_pooled", "poem_select_practical", "poem_select_ranked_budget",
 )
 
 
@@ -74,6 +75,8 @@ def _load():
     lib.poem_select.restype = st
     lib.poem_select_mass_only.argtypes = [sp, vp, vp, vp, vp, i64, vp, vp, sz, vp]
     lib.poem_select_mass_only.restype = st
+    lib.poem_select_ranked_budget.argtypes = [sp, vp, vp, vp, vp, i64, vp, vp, sz, vp]
+    lib.poem_select_ranked_budget.restype = st
     lib.poem_select_noalloc.argtypes = [sp, vp, vp, ctypes.c_float, vp, vp, i64, vp, vp]
     lib.poem_select_noalloc.restype = st
     lib.poem_pooled_workspace_size.argtypes = [sp, ctypes.POINTER(sz)]
@@ -166,6 +169,14 @@ def poem_select_mass_only(shape: Shape, m_hat, ref_row_ptr, row_ptr, col_idx, ws
     _raise(_lib.poem_select_mass_only(ctypes.byref(shape), _ptr(m_hat), _ptr(ref_row_ptr), _ptr(row_ptr),
                                       _ptr(col_idx), col_idx.numel(), _ptr(order), _ptr(ws),
                                       ws.numel() * ws.element_size(), _stream(stream)), "poem_select_mass_only")
+
+
+def poem_select_ranked_budget(shape: Shape, score, ref_row_ptr, row_ptr, col_idx, ws, order=None, stream=None):
+    """Mandatory blocks + the top candidates by `score` at the per-row budget of ref_row_ptr."""
+    _raise(_lib.poem_select_ranked_budget(ctypes.byref(shape), _ptr(score), _ptr(ref_row_ptr), _ptr(row_ptr),
+                                          _ptr(col_idx), col_idx.numel(), _ptr(order), _ptr(ws),
+                                          ws.numel() * ws.element_size(), _stream(stream)),
+           "poem_select_ranked_budget")
 
 
 def poem_select_noalloc(shape: Shape, I_hat, m_hat, tau: float, row_ptr, col_idx, order=None, stream=None):

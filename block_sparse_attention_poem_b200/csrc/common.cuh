@@ -90,18 +90,20 @@ struct PoolParams {
   const __nv_bfloat16* v;
   int64_t q_stride_tok, q_stride_head;
   int64_t kv_stride_tok, kv_stride_head;
-  float* q_bar;   // [Hq, T, D] fp32 tile means of the queries
-  float* k_bar;   // [Hkv, T, D] fp32 block means of the keys
-  float* v_bar;   // [Hkv, T, D] fp32 block means of the values
-  float* m_pool;  // packed lower-triangular [Hq, T(T+1)/2]: m~
-  float* d_pool;  //                                          d~
+  float* q_bar;    // [Hq, T, D] fp32 tile means of the queries
+  float* k_bar_t;  // [Hkv, D, T] fp32 block means of the keys, channel-major
+  float* v_bar;    // [Hkv, T, D] fp32 block means of the values
+  float* v_bar_t;  // [Hkv, D, T] the same, channel-major
+  float* m_pool;   // packed lower-triangular [Hq, T(T+1)/2]: m~
+  float* d_pool;   //                                          d~
   int n_q_heads;
   int n_kv_heads;
   int n_tiles;
   int block;
   int group;
-  int rows_per_cta;  // R: query heads of one KV head handled by one CTA (divides group, <= 8)
-  float scale;       // softmax scale (natural-log domain)
+  int heads_per_cta;  // query heads of one KV head per CTA (divides group)
+  int tiles_per_cta;  // adjacent query tiles per CTA; heads * tiles <= 8
+  float scale;        // softmax scale (natural-log domain)
   DevErr err;
 };
 
@@ -111,7 +113,6 @@ cudaError_t launch_bsa_fwd(int head_dim, int block, const CUtensorMap& tmQ, cons
 cudaError_t launch_score(int head_dim, int block, const CUtensorMap& tmQs, const CUtensorMap& tmK,
                          const CUtensorMap& tmV, const ScoreParams& p, cudaStream_t stream);
 cudaError_t launch_select(const SelectParams& p, cudaStream_t stream);
-cudaError_t launch_pooled(int head_dim, const PoolParams& p, cudaStream_t stream);
-int pooled_rows_per_cta(int group, int n_tiles, int head_dim);
+cudaError_t launch_pooled(int head_dim, PoolParams p, cudaStream_t stream);
 
 }  // namespace poem

@@ -74,10 +74,11 @@ size_t select_ws_bytes(const poem_shape* s, int T) {
 
 size_t fwd_ws_bytes(const poem_shape*, int) { return poem::kWsHeader; }
 
-// Pooled means q~ [Hq, T, D], k~ and v~ [Hkv, T, D] (fp32) after the header.
+// Pooled means (fp32) after the header: q~ [Hq, T, D], then k~ channel-major
+// [Hkv, D, T], v~ [Hkv, T, D] and v~ channel-major [Hkv, D, T].
 size_t pooled_ws_bytes(const poem_shape* s, int T) {
   const size_t qn = (size_t)s->n_q_heads * T * s->head_dim, kn = (size_t)s->n_kv_heads * T * s->head_dim;
-  return poem::kWsHeader + round_up(qn * sizeof(float), 256) + 2 * round_up(kn * sizeof(float), 256);
+  return poem::kWsHeader + round_up(qn * sizeof(float), 256) + 3 * round_up(kn * sizeof(float), 256);
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -260,6 +261,13 @@ poem_status poem_select_mass_only(const poem_shape* shape, const float* m_hat, c
                        ws_bytes, stream);
 }
 
+poem_status poem_select_ranked_budget(const poem_shape* shape, const float* score, const int32_t* ref_row_ptr,
+                                      int32_t* row_ptr, int32_t* col_idx, int64_t col_capacity, int32_t* order,
+                                      void* ws, size_t ws_bytes, void* stream) {
+  return select_common(shape, nullptr, score, ref_row_ptr, 0.0, 1, row_ptr, col_idx, col_capacity, order, ws,
+                       ws_bytes, stream);
+}
+
 poem_status poem_pooled_workspace_size(const poem_shape* shape, size_t* pooled_bytes) {
   Layout L;
   poem_status st = check_shape(shape, &L);
@@ -287,9 +295,11 @@ poem_status poem_score_pooled(const poem_shape* shape, const poem_bf16* q, const
   p.q_stride_head = shape->q_stride_head;
   p.kv_stride_tok = shape->kv_stride_tok;
   p.kv_stride_head = shape->kv_stride_head;
+  const size_t qb = round_up(qn * sizeof(float), 256), kb = round_up(kn * sizeof(float), 256);
   p.q_bar = reinterpret_cast<float*>(base);
-  p.k_bar = reinterpret_cast<float*>(base + round_up(qn * sizeof(float), 256));
-  p.v_bar = reinterpret_cast<float*>(base + round_up(qn * sizeof(float), 256) + round_up(kn * sizeof(float), 256));
+  p.k_bar_t = reinterpret_cast<float*>(base + qb);
+  p.v_bar = reinterpret_cast<float*>(base + qb + kb);
+  p.v_bar_t = reinterpret_cast<float*>(base + qb + 2 * kb);
   p.m_pool = m_pool;
   p.d_pool = d_pool;
   p.n_q_heads = shape->n_q_heads;
@@ -297,7 +307,6 @@ poem_status poem_score_pooled(const poem_shape* shape, const poem_bf16* q, const
   p.n_tiles = L.T;
   p.block = shape->block;
   p.group = L.G;
-  p.rows_per_cta = poem::pooled_rows_per_cta(L.G, L.T, shape->head_dim);
   p.scale = L.scale;
   p.err = dev_err(ws);
   cudaError_t e = poem::launch_pooled(shape->head_dim, p, (cudaStream_t)stream);

@@ -15,13 +15,19 @@
 // Kernels (caller's stream):
 //   pool_mean      grid (tile, channel groups, tensor): each thread sums the B
 //                  rows of one (head, 8-channel group) of one tile with 16-byte
-//                  streaming loads, in fp32, and writes the mean.  HBM-bound:
+//                  streaming loads, in fp32, and writes the mean -- row-major for
+//                  q~ and v~, channel-major ([D][T]) for k~ and v~.  HBM-bound:
 //                  reads Q, K and V once.
-//   pooled_scores  one CTA per (tile i, R query heads sharing a KV head), large
-//                  tiles first: logits by warp-per-block dot products (lane slices
-//                  of the channels, butterfly reduction), softmax per row, o~ with
-//                  threads over channels, then d~ like the logits.  k~ and v~ of a
-//                  KV head (T * D * 4 bytes each) stay in L2 across its CTAs.
+//   pooled_scores  one CTA per (R_t adjacent tiles x R_h query heads of one KV
+//                  head), largest tiles first; its R = R_h * R_t <= 8 rows share
+//                  every k~ / v~ value they load:
+//                    logits  lane per block, channel-major k~ (coalesced), q~
+//                            broadcast from shared memory, packed f32x2 FMAs
+//                    softmax warp per row -> m~ (shared memory and m_pool)
+//                    o~      thread per (channel, block slice), 4 blocks a step
+//                    d~      lane per block like the logits, v~ - o~ squared
+//                  The k~ / v~ of a KV head (T * D * 4 bytes each) stay in L2
+//                  across its CTAs; no warp shuffles on the per-block paths.
 #include "common.cuh"
 
 namespace poem {
@@ -29,6 +35,7 @@ namespace {
 
 constexpr int kPoolThreads = 256;
 constexpr int kScoreThreads = 256;
+constexpr int kScoreWarps = kScoreThreads / 32;
 constexpr int kMaxRows = 8;
 constexpr size_t kPooledSmemCap = 200 * 1024;
 
@@ -46,6 +53,7 @@ __global__ void __launch_bounds__(kPoolThreads) pool_mean_kernel(const PoolParam
   const int h = u / C8;
   const int c8 = u - h * C8;
   const int i = blockIdx.x;
+  const int T = p.n_tiles;
   const __nv_bfloat16* src = which == 0 ? p.q : (which == 1 ? p.k : p.v);
   const int64_t st_tok = which == 0 ? p.q_stride_tok : p.kv_stride_tok;
   const int64_t st_head = which == 0 ? p.q_stride_head : p.kv_stride_head;
@@ -59,33 +67,23 @@ __global__ void __launch_bounds__(kPoolThreads) pool_mean_kernel(const PoolParam
     const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      acc[2 * e] += __uint_as_float(ws[e] << 16);
-      acc[2 * e + 1] += __uint_as_float(ws[e] & 0xffff0000u);
+      acc[2 * e] += bf16lo_to_f32(ws[e]);
+      acc[2 * e + 1] += bf16hi_to_f32(ws[e]);
     }
   }
   const float inv = 1.0f / (float)p.block;
-  float* dst = (which == 0 ? p.q_bar : (which == 1 ? p.k_bar : p.v_bar)) + ((int64_t)h * p.n_tiles + i) * D + c8 * 8;
-  reinterpret_cast<float4*>(dst)[0] = make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
-  reinterpret_cast<float4*>(dst)[1] = make_float4(acc[4] * inv, acc[5] * inv, acc[6] * inv, acc[7] * inv);
-}
-
-// Lane slice of a D-channel fp32 row: E = D / 32 consecutive channels per lane.
-template <int E>
-struct Slice {
-  float x[E];
-};
-
-template <int E>
-__device__ __forceinline__ Slice<E> load_slice(const float* row, int lane) {
-  Slice<E> s;
-  if constexpr (E == 4) {
-    const float4 v = *reinterpret_cast<const float4*>(row + lane * 4);
-    s.x[0] = v.x; s.x[1] = v.y; s.x[2] = v.z; s.x[3] = v.w;
-  } else {
-    const float2 v = *reinterpret_cast<const float2*>(row + lane * 2);
-    s.x[0] = v.x; s.x[1] = v.y;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) acc[e] *= inv;
+  if (which != 1) {  // row-major [H, T, D]
+    float* dst = (which == 0 ? p.q_bar : p.v_bar) + ((int64_t)h * T + i) * D + c8 * 8;
+    reinterpret_cast<float4*>(dst)[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+    reinterpret_cast<float4*>(dst)[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
   }
-  return s;
+  if (which != 0) {  // channel-major [H, D, T]
+    float* dst = (which == 1 ? p.k_bar_t : p.v_bar_t) + ((int64_t)h * D + c8 * 8) * T + i;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) dst[(int64_t)e * T] = acc[e];
+  }
 }
 
 __device__ __forceinline__ float warp_sum(float x) {
@@ -102,89 +100,127 @@ __device__ __forceinline__ float warp_max(float x) {
 
 template <int D, int R>
 __global__ void __launch_bounds__(kScoreThreads) pooled_scores_kernel(const PoolParams p) {
-  constexpr int E = D / 32;
-  constexpr int S = kScoreThreads / D;  // channel-parallel slices of the o~ pass
-  constexpr int W = kScoreThreads / 32;
+  constexpr int S = kScoreThreads / D;  // block slices of the o~ pass
   extern __shared__ __align__(16) float smf[];
   const int T = p.n_tiles;
   const int ld = (T + 3) & ~3;
-  float* qb = smf;             // [R][D]
-  float* ob = qb + R * D;      // [R][D]
-  float* part = ob + R * D;    // [S][R][D]
+  float* qb = smf;                // [R][D]
+  float* ob = qb + R * D;         // [R][D]
+  float* part = ob + R * D;       // [S][R][D]
   float* buf = part + S * R * D;  // [R][ld]: logits -> m~ -> d~
+  __shared__ int s_head[R], s_tile[R];
 
-  const int n_chunks = p.n_q_heads / R;
-  const int u = blockIdx.x;
-  const int i = T - 1 - u / n_chunks;
-  const int h0 = (u - (u / n_chunks) * n_chunks) * R;
+  const int Rh = p.heads_per_cta, Rt = p.tiles_per_cta;
+  const int n_hchunks = p.n_q_heads / Rh;
+  const int tg = blockIdx.x / n_hchunks;
+  const int h0 = (blockIdx.x - tg * n_hchunks) * Rh;
+  const int i_top = T - 1 - tg * Rt;  // tiles i_top, i_top - 1, ..., i_top - Rt + 1 (those >= 0)
   const int g = h0 / p.group;
-  const int nb = i + 1;
+  const int nbmax = i_top + 1;
+  const int nb4 = (nbmax + 3) & ~3;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const float* kbar = p.k_bar + (int64_t)g * T * D;
-  const float* vbar = p.v_bar + (int64_t)g * T * D;
+  const float* kT = p.k_bar_t + (int64_t)g * D * T;
+  const float* vT = p.v_bar_t + (int64_t)g * D * T;
+  const float* vb = p.v_bar + (int64_t)g * T * D;
 
+  // Row r: head h0 + r % Rh, tile i_top - r / Rh (invalid when the tile is < 0
+  // or r >= Rh * Rt); nb_r = tile + 1 visible blocks, 0 for invalid rows.
+  int nb[R];
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    const int tile = (r < Rh * Rt) ? i_top - r / Rh : -1;
+    nb[r] = tile >= 0 ? tile + 1 : 0;
+  }
+  if (threadIdx.x < R) {
+    const int r = threadIdx.x;
+    s_head[r] = h0 + r % Rh;
+    s_tile[r] = (r < Rh * Rt) ? i_top - r / Rh : -1;
+  }
   for (int x = threadIdx.x; x < R * D; x += kScoreThreads) {
     const int r = x / D, c = x - r * D;
-    qb[x] = p.q_bar[((int64_t)(h0 + r) * T + i) * D + c];
+    const int tile = (r < Rh * Rt) ? i_top - r / Rh : -1;
+    qb[x] = tile >= 0 ? p.q_bar[((int64_t)(h0 + r % Rh) * T + tile) * D + c] : 0.f;
   }
   __syncthreads();
 
-  // Logits: warp per block, lane slices of the channels.
-  {
-    Slice<E> qs[R];
+  // Logits: lane per block; channel-major k~ makes each channel one coalesced load.
+  for (int b0 = warp * 32; b0 < nbmax; b0 += kScoreThreads) {
+    const int b = b0 + lane;
+    const bool ok = b < nbmax;
+    uint64_t acc[R];
 #pragma unroll
-    for (int r = 0; r < R; ++r) qs[r] = load_slice<E>(qb + r * D, lane);
-    for (int b = warp; b < nb; b += W) {
-      const Slice<E> ks = load_slice<E>(kbar + (int64_t)b * D, lane);
-      float s[R];
+    for (int r = 0; r < R; ++r) acc[r] = 0ull;
+#pragma unroll 4
+    for (int c = 0; c < D; c += 4) {
+      float kv[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) kv[e] = ok ? kT[(int64_t)(c + e) * T + b] : 0.f;
+      const uint64_t k01 = f2_pack(kv[0], kv[1]), k23 = f2_pack(kv[2], kv[3]);
 #pragma unroll
       for (int r = 0; r < R; ++r) {
-        float a = 0.f;
-#pragma unroll
-        for (int e = 0; e < E; ++e) a = fmaf(qs[r].x[e], ks.x[e], a);
-        s[r] = warp_sum(a);
+        const float4 qv = *reinterpret_cast<const float4*>(qb + r * D + c);
+        acc[r] = f2_fma(f2_pack(qv.x, qv.y), k01, acc[r]);
+        acc[r] = f2_fma(f2_pack(qv.z, qv.w), k23, acc[r]);
       }
+    }
 #pragma unroll
-      for (int r = 0; r < R; ++r)
-        if (lane == r) buf[r * ld + b] = s[r] * p.scale;
+    for (int r = 0; r < R; ++r) {
+      if (b < nb[r]) {
+        float lo, hi;
+        f2_unpack(acc[r], lo, hi);
+        buf[r * ld + b] = (lo + hi) * p.scale;
+      }
     }
   }
   __syncthreads();
 
-  // Softmax per row (warp per row): m~ to shared memory and to m_pool.
-  for (int r = warp; r < R; r += W) {
+  // Softmax per row (warp per row): m~ to shared memory and to m_pool; entries
+  // from nb_r up to the 4-block boundary of the longest row are zeroed.
+  for (int r = warp; r < R; r += kScoreWarps) {
     float* row = buf + r * ld;
-    float mx = -INFINITY;
-    for (int b = lane; b < nb; b += 32) mx = fmaxf(mx, row[b]);
-    mx = warp_max(mx);
-    float den = 0.f;
-    for (int b = lane; b < nb; b += 32) {
-      const float e = expf(row[b] - mx);
-      row[b] = e;
-      den += e;
+    const int n = (s_tile[r] >= 0) ? s_tile[r] + 1 : 0;
+    if (n > 0) {
+      float mx = -INFINITY;
+      for (int b = lane; b < n; b += 32) mx = fmaxf(mx, row[b]);
+      mx = warp_max(mx);
+      float den = 0.f;
+      for (int b = lane; b < n; b += 32) {
+        const float e = expf(row[b] - mx);
+        row[b] = e;
+        den += e;
+      }
+      den = warp_sum(den);
+      const float inv = 1.0f / den;
+      float* dst = p.m_pool + tri_off(T, s_head[r], s_tile[r]);
+      for (int b = lane; b < n; b += 32) {
+        const float m = row[b] * inv;
+        row[b] = m;
+        dst[b] = m;
+      }
     }
-    den = warp_sum(den);
-    const float inv = 1.0f / den;
-    float* dst = p.m_pool + tri_off(T, h0 + r, i);
-    for (int b = lane; b < nb; b += 32) {
-      const float m = row[b] * inv;
-      row[b] = m;
-      dst[b] = m;
-    }
+    for (int b = n + lane; b < nb4; b += 32) row[b] = 0.f;
   }
   __syncthreads();
 
-  // o~ = sum_b m~_b v~_b: thread per (slice, channel), slices interleave blocks.
+  // o~ = sum_b m~_b v~_b: thread per (slice, channel), four blocks per step.
   {
     const int c = threadIdx.x % D;
     const int sl = threadIdx.x / D;
     float acc[R];
 #pragma unroll
     for (int r = 0; r < R; ++r) acc[r] = 0.f;
-    for (int b = sl; b < nb; b += S) {
-      const float vv = vbar[(int64_t)b * D + c];
+    for (int b4 = sl * 4; b4 < nb4; b4 += 4 * S) {
+      float vv[4];
 #pragma unroll
-      for (int r = 0; r < R; ++r) acc[r] = fmaf(buf[r * ld + b], vv, acc[r]);
+      for (int e = 0; e < 4; ++e) vv[e] = (b4 + e < nbmax) ? vb[(int64_t)(b4 + e) * D + c] : 0.f;
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        const float4 m = *reinterpret_cast<const float4*>(buf + r * ld + b4);
+        acc[r] = fmaf(m.x, vv[0], acc[r]);
+        acc[r] = fmaf(m.y, vv[1], acc[r]);
+        acc[r] = fmaf(m.z, vv[2], acc[r]);
+        acc[r] = fmaf(m.w, vv[3], acc[r]);
+      }
     }
 #pragma unroll
     for (int r = 0; r < R; ++r) part[(sl * R + r) * D + c] = acc[r];
@@ -198,33 +234,44 @@ __global__ void __launch_bounds__(kScoreThreads) pooled_scores_kernel(const Pool
   }
   __syncthreads();
 
-  // d~_b = || v~_b - o~ ||, like the logits; overwrites m~ in shared memory.
-  {
-    Slice<E> os[R];
+  // d~_b = || v~_b - o~ ||: lane per block like the logits; overwrites m~.
+  const uint64_t neg1 = f2_pack(-1.f, -1.f);
+  for (int b0 = warp * 32; b0 < nbmax; b0 += kScoreThreads) {
+    const int b = b0 + lane;
+    const bool ok = b < nbmax;
+    uint64_t acc[R];
 #pragma unroll
-    for (int r = 0; r < R; ++r) os[r] = load_slice<E>(ob + r * D, lane);
-    for (int b = warp; b < nb; b += W) {
-      const Slice<E> vs = load_slice<E>(vbar + (int64_t)b * D, lane);
-      float s[R];
+    for (int r = 0; r < R; ++r) acc[r] = 0ull;
+#pragma unroll 4
+    for (int c = 0; c < D; c += 4) {
+      float vv[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) vv[e] = ok ? vT[(int64_t)(c + e) * T + b] : 0.f;
+      const uint64_t v01 = f2_pack(vv[0], vv[1]), v23 = f2_pack(vv[2], vv[3]);
 #pragma unroll
       for (int r = 0; r < R; ++r) {
-        float a = 0.f;
-#pragma unroll
-        for (int e = 0; e < E; ++e) {
-          const float df = vs.x[e] - os[r].x[e];
-          a = fmaf(df, df, a);
-        }
-        s[r] = warp_sum(a);
+        const float4 ov = *reinterpret_cast<const float4*>(ob + r * D + c);
+        const uint64_t d01 = f2_fma(f2_pack(ov.x, ov.y), neg1, v01);  // v~ - o~, exactly rounded
+        const uint64_t d23 = f2_fma(f2_pack(ov.z, ov.w), neg1, v23);
+        acc[r] = f2_fma(d01, d01, acc[r]);
+        acc[r] = f2_fma(d23, d23, acc[r]);
       }
+    }
 #pragma unroll
-      for (int r = 0; r < R; ++r)
-        if (lane == r) buf[r * ld + b] = sqrtf(s[r]);
+    for (int r = 0; r < R; ++r) {
+      if (b < nb[r]) {
+        float lo, hi;
+        f2_unpack(acc[r], lo, hi);
+        buf[r * ld + b] = sqrtf(lo + hi);
+      }
     }
   }
   __syncthreads();
   for (int r = 0; r < R; ++r) {
-    float* dst = p.d_pool + tri_off(T, h0 + r, i);
-    for (int b = threadIdx.x; b < nb; b += kScoreThreads) dst[b] = buf[r * ld + b];
+    if (s_tile[r] < 0) continue;
+    const int n = s_tile[r] + 1;
+    float* dst = p.d_pool + tri_off(T, s_head[r], s_tile[r]);
+    for (int b = threadIdx.x; b < n; b += kScoreThreads) dst[b] = buf[r * ld + b];
   }
 }
 
@@ -243,14 +290,15 @@ cudaError_t launch_scores_r(const PoolParams& p, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
     configured = true;
   }
-  const int grid = p.n_tiles * (p.n_q_heads / R);
+  const int n_tgroups = (p.n_tiles + p.tiles_per_cta - 1) / p.tiles_per_cta;
+  const int grid = n_tgroups * (p.n_q_heads / p.heads_per_cta);
   pooled_scores_kernel<D, R><<<grid, kScoreThreads, pooled_smem(R, p.n_tiles, D), stream>>>(p);
   return cudaGetLastError();
 }
 
 template <int D>
 cudaError_t launch_scores(const PoolParams& p, cudaStream_t stream) {
-  switch (p.rows_per_cta) {
+  switch (p.heads_per_cta * p.tiles_per_cta) {
     case 1: return launch_scores_r<D, 1>(p, stream);
     case 2: return launch_scores_r<D, 2>(p, stream);
     case 3: return launch_scores_r<D, 3>(p, stream);
@@ -265,16 +313,25 @@ cudaError_t launch_scores(const PoolParams& p, cudaStream_t stream) {
 
 }  // namespace
 
-// Rows per CTA: the largest divisor of the group size that is <= 8 and whose
-// shared-memory footprint fits the cap (R = 1 always fits up to 8192 tiles).
-int pooled_rows_per_cta(int group, int n_tiles, int head_dim) {
-  for (int r = kMaxRows; r >= 1; --r)
-    if (group % r == 0 && pooled_smem(r, n_tiles, head_dim) <= kPooledSmemCap) return r;
-  return 1;
-}
-
-cudaError_t launch_pooled(int head_dim, const PoolParams& p, cudaStream_t stream) {
+// Work unit of pooled_scores: the largest divisor R_h <= 8 of the group size,
+// then the most adjacent tiles R_t with R_h * R_t <= 8, both within the shared
+// memory cap (R_h = R_t = 1 fits up to 8192 tiles).
+cudaError_t launch_pooled(int head_dim, PoolParams p, cudaStream_t stream) {
   if (p.n_tiles <= 0) return cudaSuccess;
+  int rh = 1;
+  for (int r = kMaxRows; r >= 1; --r)
+    if (p.group % r == 0 && pooled_smem(r, p.n_tiles, head_dim) <= kPooledSmemCap) {
+      rh = r;
+      break;
+    }
+  int rt = 1;
+  for (int t = kMaxRows / rh; t >= 1; --t)
+    if (pooled_smem(rh * t, p.n_tiles, head_dim) <= kPooledSmemCap) {
+      rt = t;
+      break;
+    }
+  p.heads_per_cta = rh;
+  p.tiles_per_cta = rt;
   const dim3 pg(p.n_tiles, (p.n_q_heads * (head_dim / 8) + kPoolThreads - 1) / kPoolThreads, 3);
   if (head_dim == 128) {
     pool_mean_kernel<128><<<pg, kPoolThreads, 0, stream>>>(p);

@@ -142,6 +142,20 @@ poem_status poem_select_mass_only(const poem_shape* shape, const float* m_hat, c
                                   void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * poem_select_ranked_budget -- fixed-budget ranking by any per-block score: row r
+ * keeps the mandatory blocks and the (ref_row_ptr[r+1] - ref_row_ptr[r] -
+ * |mandatory|) candidates of largest score (ties: smaller id).  With score =
+ * m_hat this is poem_select_mass_only; with score = I_hat it is POEM's ranking
+ * at a given block count, which compares selectors at matched budgets (the
+ * evaluation the reading note's last section proposes).  score is packed
+ * lower-triangular like poem_score's outputs.  Same outputs and workspace as
+ * poem_select.
+ */
+poem_status poem_select_ranked_budget(const poem_shape* shape, const float* score, const int32_t* ref_row_ptr,
+                                      int32_t* row_ptr, int32_t* col_idx, int64_t col_capacity, int32_t* order,
+                                      void* ws, size_t ws_bytes, void* stream);
+
+/*
  * poem_select_noalloc -- poem_select for callers that cannot allocate device
  * memory.  (An addition of this library; the method description has no
  * counterpart.)  Some callers own no allocator: a serving runtime that reserves
@@ -180,7 +194,8 @@ poem_status poem_select_noalloc(const poem_shape* shape, const float* I_hat, con
  * ||v_b - o||).
  */
 
-/* Workspace bytes of poem_score_pooled (256-byte header, then fp32 q~, k~, v~). */
+/* Workspace bytes of poem_score_pooled: a 256-byte header, then the fp32 means
+ * q~ (row-major), k~ (channel-major), v~ (row- and channel-major). */
 poem_status poem_pooled_workspace_size(const poem_shape* shape, size_t* pooled_bytes);
 
 /*

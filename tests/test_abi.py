@@ -121,7 +121,7 @@ def test_pooled_workspace_size(poem):
     a = ctypes.c_size_t()
     assert poem._lib.poem_pooled_workspace_size(ctypes.byref(sh), ctypes.byref(a)) == 0
     T, hq, hkv, d = 8, 4, 2, 128
-    assert a.value >= 256 + (hq + 2 * hkv) * T * d * 4
+    assert a.value >= 256 + (hq + 3 * hkv) * T * d * 4
     assert poem._lib.poem_pooled_workspace_size(ctypes.byref(_shape(poem, head_dim=96)), ctypes.byref(a)) == 2
 
 

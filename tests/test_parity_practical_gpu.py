@@ -82,6 +82,8 @@ LAYERS = [
     (1280, 5, 1, 128, 128, 1),   # 5-way GQA, ragged tile count
     (1024, 2, 2, 64, 64, 2),
     (1024, 4, 2, 128, 64, 3),
+    (1152, 2, 2, 64, 64, 7),     # 18 tiles: a partial group of 8 tiles per CTA
+    (128, 4, 1, 128, 128, 8),    # a single tile
 ]
 
 
@@ -214,3 +216,35 @@ def test_prefill_layer_practical_128k_sampled(poem):
     O_ref, _ = prob.masked_units(units, rp, ci)
     exc, mean = compare_fwd_excess(layer.o, O_ref, units, B)
     assert exc <= 1.0 and mean <= FWD_MEAN_ABS, (exc, mean)
+
+
+def test_ranked_budget_matches_oracle(poem):
+    """poem_select_ranked_budget with score = exact I_hat at the practical lists'
+    budgets: identical to the oracle's fixed-budget ranking on the same scores."""
+    n, hq, hkv, d, B = 4096, 4, 1, 128, 128
+    T = n // B
+    x = poem_synth.heavy_block_layer(n, hq, hkv, d, block=B, seed=6)
+    shape, m_pool, d_pool = _pooled(poem, x, B)
+    rpn, _, rp, _ = _select(poem, shape, m_pool, d_pool, 1.0, 0.9, 0.5, hq, T)
+    q, k, v = to_dev(x)
+    ne = poem.n_score_entries(hq, T)
+    I_hat = torch.empty(ne, device="cuda")
+    m_hat = torch.empty(ne, device="cuda")
+    s_b, sel_b, _ = poem.poem_workspace_size(shape)
+    ws_s = poem.alloc_workspace(s_b)
+    poem.poem_score(q, k, v, I_hat, m_hat, ws_s, shape=shape)
+    poem.poem_check(ws_s)
+    ws = poem.alloc_workspace(sel_b)
+    rp2 = torch.empty_like(rp)
+    ci2 = torch.empty(ne, dtype=torch.int32, device="cuda")
+    poem.poem_select_ranked_budget(shape, I_hat, rp, rp2, ci2, ws)
+    poem.poem_check(ws)
+    rows = csr_rows(rp2.cpu().numpy(), ci2[: int(rp2[-1])].cpu().numpy())
+    Ig = I_hat.cpu().numpy().astype(np.float64)
+    for h in range(hq):
+        for i in range(T):
+            r = h * T + i
+            n_mand = 1 if i == 0 else (2 if i == 1 else 3)
+            budget = int(rpn[r + 1] - rpn[r]) - n_mand
+            off = oracle.tri_offset(T, h, i)
+            assert rows[r] == oracle.select_mass_only_row(i, Ig[off:off + i + 1], budget).tolist(), (h, i)
