@@ -737,6 +737,71 @@ def _dense_output(poem, q, k, v, layer, hq, T):
     return o
 
 
+EVAL_LAYERS = [
+    ("heavy-block-32k", "heavy"),
+    ("contrast-32k", "contrast"),
+]
+
+
+def _err_vs(o, o_dense):
+    diff = o.float() - o_dense.float()
+    return {"rel_fro": round(float(diff.norm() / o_dense.float().norm()), 5),
+            "mean_abs": round(float(diff.abs().mean()), 6), "max_row_l2": round(float(diff.norm(dim=-1).max()), 4)}
+
+
+def _report_evaluation(poem):
+    """Selectors compared on output error against dense attention (the evaluation
+    the reading note proposes): POEM's threshold rule with mass-only at the same
+    block count; exact-I order vs exact-mass order at the same retained mass
+    (keep blocks in that order until the max-aggregated mass reaches gamma); the
+    practical selector.  Heavy-block layer and the mass/deviation contrast layer
+    (cancelling heavy pairs, flat heavy blocks, deviant light blocks), 32K tokens."""
+    n, hq, hkv, d, B, base, _ = WORKLOADS["llama3.1-8b-layer-32k"]
+    T = n // B
+    visible = hq * T * (T + 1) // 2
+    out = []
+    for name, kind in EVAL_LAYERS:
+        gen = poem_synth.contrast_layer if kind == "contrast" else poem_synth.heavy_block_layer
+        x = gen(n, hq, hkv, d, block=B, rope_base=base, seed=0)
+        q, k, v = x["q"].cuda(), x["k"].cuda(), x["v"].cuda()
+        layer = poem.alloc_layer(q, k, block=B, practical=True)
+        poem.poem_score(q, k, v, layer.I_hat, layer.m_hat, layer.ws_score, shape=layer.shape)
+        poem.poem_check(layer.ws_score)
+        o_dense = _dense_output(poem, q, k, v, layer, hq, T)
+        rp2 = torch.empty_like(layer.row_ptr)
+        ci2 = torch.empty_like(layer.col_idx)
+        o2 = torch.empty_like(q)
+
+        def run(rp, ci):
+            poem.bsa_fwd(q, k, v, rp, ci, o2, layer.ws_fwd, shape=layer.shape)
+            torch.cuda.synchronize()
+            poem.poem_check(layer.ws_fwd)
+            return {"density": round(int(rp[-1]) / visible, 5), "err": _err_vs(o2, o_dense)}
+
+        for tau in (0.05, 0.2, 0.5):
+            poem.poem_select(layer.shape, layer.I_hat, layer.m_hat, tau, layer.row_ptr, layer.col_idx,
+                             layer.ws_select)
+            rec = {"config": "evaluation", "layer": name, "rule": "poem-threshold", "tau": tau,
+                   **run(layer.row_ptr, layer.col_idx)}
+            poem.poem_select_mass_only(layer.shape, layer.m_hat, layer.row_ptr, rp2, ci2, layer.ws_select)
+            rec["mass_only_same_count"] = run(rp2, ci2)
+            out.append(rec)
+        d_ex = layer.I_hat / layer.m_hat.clamp_min(1e-30)  # harness-side: Î / m̂ turns the rerank key into log Î
+        for gamma in (0.9, 0.95, 0.99):
+            rec = {"config": "evaluation", "layer": name, "rule": "same-retained-mass", "gamma": gamma}
+            for label, w in (("exact_I_order", 1.0), ("mass_order", 0.0)):
+                poem.poem_select_practical(layer.shape, layer.m_hat, d_ex, w, gamma, 1.0, rp2, ci2, layer.ws_select)
+                rec[label] = run(rp2, ci2)
+            poem.poem_score_pooled(q, k, v, layer.m_pool, layer.d_pool, layer.ws_pooled, shape=layer.shape)
+            poem.poem_select_practical(layer.shape, layer.m_pool, layer.d_pool, 1.0, gamma, 0.5, rp2, ci2,
+                                       layer.ws_select)
+            rec["practical_w1_rho0.5"] = run(rp2, ci2)
+            out.append(rec)
+        del layer, q, k, v, o_dense, o2, d_ex
+        torch.cuda.empty_cache()
+    return out
+
+
 def run_report(args):
     import block_sparse_attention_poem_b200 as poem
 
@@ -753,6 +818,9 @@ def run_report(args):
         for wl, params in PRACTICAL_REPORT:
             for rec in _report_practical(poem, wl, params, args.steps, args.warmup):
                 print(json.dumps(rec), flush=True)
+    if part in (None, "evaluation"):
+        for rec in _report_evaluation(poem):
+            print(json.dumps(rec), flush=True)
     if part in (None, "sweep"):
         for rec in _report_sweep(poem, args.steps, args.warmup):
             print(json.dumps(rec), flush=True)
@@ -779,7 +847,7 @@ def main():
     ap.add_argument("--rho", type=float, default=0.5, help="practical: stage-1 shortlist fraction")
     ap.add_argument("--report", action="store_true",
                     help="measure every configuration (one JSON record each) instead of the benchmark line")
-    ap.add_argument("--report-only", choices=["exact", "practical", "sweep"], default=None,
+    ap.add_argument("--report-only", choices=["exact", "practical", "evaluation", "sweep"], default=None,
                     help="with --report: only this part")
     args = ap.parse_args()
     if args.report:

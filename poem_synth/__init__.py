@@ -23,6 +23,14 @@ which need model weights and datasets that are not used here):
   keys.  Rotary embedding (rotate-half pairing, given base, no frequency
   rescaling) is applied to Q and K.  V = Z_v + mu[g, block], with
   mu ~ N(0, 0.5^2) per (KV head, block, dim).  Converted to bf16.
+* ``contrast_layer``: the heavy-block layer's Q and K (same draws), but
+  value offsets chosen so that block mass and block deviation disagree: no
+  offset on ordinary blocks; a fraction ``flat_frac`` of the heavy blocks keep
+  no offset (high mass, value near the dense output); the other heavy blocks,
+  taken in id order, form pairs with opposite offsets +c w, -c w (w a random
+  unit vector per pair, c = ``pair_offset``), whose deviations cancel in the
+  output; ordinary blocks are "deviant" with probability ``deviant_prob`` and
+  get an offset of norm ``deviant_offset`` along a random unit vector.
 * ``iid_layer``: Q, K, V i.i.d. N(0, 1), converted to bf16.
 * ``random_block_lists``: per (head, tile i) the mandatory sink and diagonal
   blocks {0, i}, then blocks drawn uniformly without replacement from
@@ -129,6 +137,46 @@ def heavy_block_layer(n_tokens: int, n_q_heads: int = 32, n_kv_heads: int = 8, h
         "heavy": heavy,
         "beta": beta,
     }
+
+
+def contrast_layer(n_tokens: int, n_q_heads: int = 32, n_kv_heads: int = 8, head_dim: int = 128,
+                   block: int = 128, rope_base: float = 500000.0, seed: int = 0, heavy_prob: float = 0.1,
+                   beta_range=(4.0, 6.0), flat_frac: float = 0.5, pair_offset: float = 3.0,
+                   deviant_prob: float = 0.05, deviant_offset: float = 6.0):
+    """Mass/deviation contrast recipe (module docstring).  Q and K are those of
+    heavy_block_layer with the same arguments; returns dict with bf16 q, k, v and
+    the drawn structure (heavy, flat, pair_sign, deviant masks)."""
+    x = heavy_block_layer(n_tokens, n_q_heads, n_kv_heads, head_dim, block=block, rope_base=rope_base, seed=seed,
+                          heavy_prob=heavy_prob, beta_range=beta_range)
+    g = torch.Generator().manual_seed(seed + 7919)
+    T = n_tokens // block
+    heavy = x["heavy"]
+    v = torch.randn(n_tokens, n_kv_heads, head_dim, generator=g, dtype=torch.float32)
+    flat = torch.zeros(n_kv_heads, T, dtype=torch.bool)
+    sign = torch.zeros(n_kv_heads, T, dtype=torch.int8)
+    deviant = torch.zeros(n_kv_heads, T, dtype=torch.bool)
+    mu = torch.zeros(n_kv_heads, T, head_dim, dtype=torch.float32)
+    for gi in range(n_kv_heads):
+        hb = torch.nonzero(heavy[gi]).flatten()
+        keep_flat = torch.rand(hb.numel(), generator=g) < flat_frac
+        flat[gi, hb[keep_flat]] = True
+        paired = hb[~keep_flat]
+        for a in range(0, paired.numel() - 1, 2):
+            w = torch.randn(head_dim, generator=g)
+            w = w / w.norm()
+            mu[gi, paired[a]] = pair_offset * w
+            mu[gi, paired[a + 1]] = -pair_offset * w
+            sign[gi, paired[a]] = 1
+            sign[gi, paired[a + 1]] = -1
+        light = torch.nonzero(~heavy[gi]).flatten()
+        dv = light[torch.rand(light.numel(), generator=g) < deviant_prob]
+        for b in dv.tolist():
+            w = torch.randn(head_dim, generator=g)
+            mu[gi, b] = deviant_offset * w / w.norm()
+        deviant[gi, dv] = True
+        v[:, gi, :] += mu[gi].repeat_interleave(block, dim=0)
+    return {"q": x["q"], "k": x["k"], "v": v.to(torch.bfloat16), "heavy": heavy, "flat": flat,
+            "pair_sign": sign, "deviant": deviant}
 
 
 def iid_layer(n_tokens: int, n_q_heads: int = 32, n_kv_heads: int = 8, head_dim: int = 128, seed: int = 0):

@@ -43,3 +43,21 @@ def test_random_block_lists_structure():
         assert len(row) == max(len({0, i}), int(round(0.25 * (i + 1))))
     rp1, ci1 = poem_synth.random_block_lists(2, 20, 1.0, seed=5)
     assert rp1[-1] == 2 * 20 * 21 // 2
+
+
+def test_contrast_layer_structure():
+    x = poem_synth.contrast_layer(4096, 4, 2, 64, block=128, seed=2, heavy_prob=0.3)
+    y = poem_synth.heavy_block_layer(4096, 4, 2, 64, block=128, seed=2, heavy_prob=0.3)
+    assert torch.equal(x["q"], y["q"]) and torch.equal(x["k"], y["k"])
+    v = x["v"].float().view(32, 128, 2, 64).mean(1)  # block means [T, Hkv, d]
+    for g in range(2):
+        heavy, flat, sign, dev = x["heavy"][g], x["flat"][g], x["pair_sign"][g], x["deviant"][g]
+        assert not (flat & ~heavy).any() and not (dev & heavy).any()
+        assert int((sign == 1).sum()) == int((sign == -1).sum())
+        pos = torch.nonzero(sign == 1).flatten()
+        neg = torch.nonzero(sign == -1).flatten()
+        for a, b in zip(pos.tolist(), neg.tolist()):
+            # opposite offsets: the pair's block means nearly cancel
+            assert float((v[a, g] + v[b, g]).norm()) < 1.6 < float(v[a, g].norm())
+        if dev.any():
+            assert float(v[dev, g].norm(dim=-1).min()) > 4.0
