@@ -54,7 +54,7 @@ class Shape(ctypes.Structure):
     _fields_ = [
         ("n_tokens", ctypes.c_int32), ("n_q_heads", ctypes.c_int32), ("n_kv_heads", ctypes.c_int32),
         ("head_dim", ctypes.c_int32), ("block", ctypes.c_int32), ("n_sample", ctypes.c_int32),
-        ("softmax_scale", ctypes.c_float), ("reserved0", ctypes.c_int32),
+        ("softmax_scale", ctypes.c_float), ("q_offset", ctypes.c_int32),
         ("q_stride_tok", ctypes.c_int64), ("q_stride_head", ctypes.c_int64),
         ("kv_stride_tok", ctypes.c_int64), ("kv_stride_head", ctypes.c_int64),
         ("o_stride_tok", ctypes.c_int64), ("o_stride_head", ctypes.c_int64),
@@ -119,14 +119,17 @@ def _stream(stream):
 
 def make_shape(q: torch.Tensor, k: torch.Tensor, block: int = 128, n_sample: int = 16, scale: float = 0.0,
                o: torch.Tensor | None = None) -> Shape:
-    """Shape of a layer from q [N, Hq, d] and k/v [N, Hkv, d] (any strides with a
-    contiguous head dimension); o defaults to q's strides."""
+    """Shape of a layer from q [Nq, Hq, d] and k/v [Nk, Hkv, d] (any strides with a
+    contiguous head dimension); o defaults to q's strides.  Nk > Nq is a chunked
+    prefill: the queries are the last Nq of the Nk tokens (q_offset = Nk - Nq)."""
     n, hq, d = q.shape
-    hkv = k.shape[1]
+    nk, hkv = k.shape[0], k.shape[1]
     if q.stride(2) != 1 or k.stride(2) != 1:
         raise ValueError("the head dimension must be contiguous")
+    if nk < n:
+        raise ValueError("k/v must hold at least as many tokens as q")
     o_st = (o.stride(0), o.stride(1)) if o is not None else (q.stride(0), q.stride(1))
-    return Shape(n, hq, hkv, d, block, n_sample, float(scale), 0, q.stride(0), q.stride(1), k.stride(0),
+    return Shape(n, hq, hkv, d, block, n_sample, float(scale), nk - n, q.stride(0), q.stride(1), k.stride(0),
                  k.stride(1), o_st[0], o_st[1])
 
 
@@ -142,8 +145,15 @@ def alloc_workspace(nbytes: int, device="cuda") -> torch.Tensor:
     return torch.zeros(max(int(nbytes), 256), dtype=torch.uint8, device=device)
 
 
-def n_score_entries(n_q_heads: int, n_tiles: int) -> int:
-    return n_q_heads * n_tiles * (n_tiles + 1) // 2
+def n_score_entries(n_q_heads: int, n_tiles: int, q_tile0: int = 0) -> int:
+    """Entries of the per-(head, query tile, visible block) arrays: row (h, i) holds
+    q_tile0 + i + 1 entries at h*E + i*q_tile0 + i*(i+1)/2."""
+    return n_q_heads * (n_tiles * q_tile0 + n_tiles * (n_tiles + 1) // 2)
+
+
+def score_row_offset(n_tiles: int, q_tile0: int, h: int, i: int) -> int:
+    """Offset of row (head h, query tile i) in the per-(head, tile, block) arrays."""
+    return h * (n_tiles * q_tile0 + n_tiles * (n_tiles + 1) // 2) + i * q_tile0 + i * (i + 1) // 2
 
 
 def _check_bf16(*ts):
@@ -267,7 +277,7 @@ def alloc_layer(q, k, block: int = 128, n_sample: int = 16, with_lse: bool = Fal
     T = n // block
     s_b, sel_b, f_b = poem_workspace_size(shape)
     dev = q.device
-    ne = n_score_entries(hq, T)
+    ne = n_score_entries(hq, T, shape.q_offset // block)
     extra = {}
     if practical:
         extra = dict(m_pool=torch.empty(ne, dtype=torch.float32, device=dev),

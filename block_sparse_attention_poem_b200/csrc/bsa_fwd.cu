@@ -6,7 +6,9 @@
 // diagonal block, only keys at or before the query).
 //
 // One CTA per (head, tile) row, 128 query rows (M = 128; with 64-token blocks the
-// upper 64 rows are padding and are not stored).  Roles:
+// upper 64 rows are padding and are not stored).  With a query offset (chunked
+// prefill) local query tile i is global tile q_tile0 + i: it sees key blocks
+// 0 .. q_tile0 + i and its diagonal block is q_tile0 + i.  Roles:
 //   warps 0-3  softmax: one query row per thread; reads S from TMEM, keeps the
 //              running max / sum, writes P (bf16) back into the S columns, rescales
 //              O in TMEM only when the max grows by more than 2^8, and runs the
@@ -141,7 +143,8 @@ __global__ void __launch_bounds__(kThreadsFwd, 2)
     return;
   }
   const int h = row / p.n_tiles;
-  const int tile = row - h * p.n_tiles;
+  const int tile = row - h * p.n_tiles;   // local query tile (row of Q / O)
+  const int gtile = tile + p.q_tile0;     // its global index: key blocks 0 .. gtile are visible
   const int hk = h / p.group;
   const int beg = p.row_ptr[row];
   int end = p.row_ptr[row + 1];
@@ -179,7 +182,7 @@ __global__ void __launch_bounds__(kThreadsFwd, 2)
       int q_issued = 0, k_issued = 0, v_issued = 0;
       bool have_any = false;
       for (int e = beg; e < end; ++e) {
-        if (block_ok(p.col_idx[e], tile)) { have_any = true; break; }
+        if (block_ok(p.col_idx[e], gtile)) { have_any = true; break; }
       }
       if (have_any) {
         mbar_arrive_expect_tx(&sb->q_full, C::kQBytes);
@@ -189,7 +192,7 @@ __global__ void __launch_bounds__(kThreadsFwd, 2)
       }
       for (int e = beg; e < end && !sb->abort_flag; ++e) {
         const int id = p.col_idx[e];
-        if (!block_ok(id, tile)) {
+        if (!block_ok(id, gtile)) {
           raise_err(p.err, kErrBadList);
           continue;
         }
@@ -239,7 +242,7 @@ __global__ void __launch_bounds__(kThreadsFwd, 2)
         return true;
       };
       for (int e = beg; e < end && ok; ++e) {
-        if (!block_ok(p.col_idx[e], tile)) continue;
+        if (!block_ok(p.col_idx[e], gtile)) continue;
         if (!q_ready) {
           if (!wait_or_abort(&sb->q_full, 0, sb, p.err)) { ok = false; break; }
           q_ready = true;
@@ -270,7 +273,8 @@ __global__ void __launch_bounds__(kThreadsFwd, 2)
   } else {
     // ============================ softmax warps ============================
     const int r = tid;                       // query row within the tile (TMEM lane)
-    const int qpos = tile * BN + r;          // token index of this row
+    const int qpos = tile * BN + r;          // query token index of this row (row of O / lse)
+    const int kpos = gtile * BN + r;         // its position among the keys
     const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
     const uint32_t tS = lane_base + C::kColS;
     const uint32_t tO = lane_base + C::kColO;
@@ -282,12 +286,12 @@ __global__ void __launch_bounds__(kThreadsFwd, 2)
     int id = (beg < end) ? p.col_idx[beg] : -1;
     for (int e = beg; e < end; ++e) {
       const int id_next = (e + 1 < end) ? p.col_idx[e + 1] : -1;  // prefetched a block ahead
-      if (block_ok(id, tile)) {
+      if (block_ok(id, gtile)) {
         // tcgen05.ld is warp-collective: every lane of the warp takes the same branch.
         if (!__all_sync(0xffffffffu, wait_or_abort(&sb->s_full, it & 1, sb, p.err))) { ok = false; break; }
         tc_fence_after();
-        const bool diag = (id == tile);
-        const int lim = qpos - id * BN;  // on the diagonal block, columns <= lim are visible
+        const bool diag = (id == gtile);
+        const int lim = kpos - id * BN;  // on the diagonal block, columns <= lim are visible
         // row max of S_j (all column chunks, one wait)
         float mx = -INFINITY;
         {

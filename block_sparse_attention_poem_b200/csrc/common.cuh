@@ -27,6 +27,18 @@ __host__ __device__ __forceinline__ int default_row_of_unit(int u, int n_tiles, 
   return h * n_tiles + i;
 }
 
+// Offset of row (head h, local query tile i) in the packed per-(head, tile, block)
+// arrays (scores, estimates, per-row scratch lists).  Local tile i is global tile
+// t0 + i (t0 = query offset / block) and has t0 + i + 1 visible key blocks, so
+// each head holds E = Tq t0 + Tq (Tq + 1) / 2 entries; t0 = 0 gives the plain
+// lower-triangular layout h T (T + 1) / 2 + i (i + 1) / 2.
+__host__ __device__ __forceinline__ int64_t row_entries(int n_q_tiles, int t0) {
+  return (int64_t)n_q_tiles * t0 + (int64_t)n_q_tiles * (n_q_tiles + 1) / 2;
+}
+__host__ __device__ __forceinline__ int64_t row_off(int n_q_tiles, int t0, int h, int i) {
+  return (int64_t)h * row_entries(n_q_tiles, t0) + (int64_t)i * t0 + (int64_t)i * (i + 1) / 2;
+}
+
 struct FwdParams {
   const int32_t* row_ptr;
   const int32_t* col_idx;
@@ -35,9 +47,10 @@ struct FwdParams {
   float* lse;
   int64_t o_stride_tok;
   int64_t o_stride_head;
-  int n_tokens;
+  int n_tokens;       // query tokens (rows of q, o and lse)
   int n_q_heads;
-  int n_tiles;
+  int n_tiles;        // query tiles
+  int q_tile0;        // global tile of the first query tile (query offset / block)
   int group;          // query heads per KV head
   float scale_log2;   // softmax_scale * log2(e)
   DevErr err;
@@ -51,7 +64,8 @@ struct ScoreParams {
   int n_tokens;
   int n_q_heads;
   int n_kv_heads;
-  int n_tiles;
+  int n_tiles;         // query tiles
+  int q_tile0;         // global tile of the first query tile
   int group;
   int n_sample;        // S
   int sample_stride;   // B / S
@@ -70,7 +84,8 @@ struct SelectParams {
   int32_t* order;
   int64_t col_capacity;
   int n_q_heads;
-  int n_tiles;
+  int n_tiles;   // query tiles
+  int q_tile0;   // global tile of the first query tile
   int group;
   double tau;
   int mass_only;
@@ -90,15 +105,17 @@ struct PoolParams {
   const __nv_bfloat16* v;
   int64_t q_stride_tok, q_stride_head;
   int64_t kv_stride_tok, kv_stride_head;
-  float* q_bar;    // [Hq, T, D] fp32 tile means of the queries
-  float* k_bar_t;  // [Hkv, D, T] fp32 block means of the keys, channel-major
-  float* v_bar;    // [Hkv, T, D] fp32 block means of the values
-  float* v_bar_t;  // [Hkv, D, T] the same, channel-major
-  float* m_pool;   // packed lower-triangular [Hq, T(T+1)/2]: m~
-  float* d_pool;   //                                          d~
+  float* q_bar;    // [Hq, Tq, D] fp32 tile means of the queries
+  float* k_bar_t;  // [Hkv, D, Tk] fp32 block means of the keys, channel-major
+  float* v_bar;    // [Hkv, Tk, D] fp32 block means of the values
+  float* v_bar_t;  // [Hkv, D, Tk] the same, channel-major
+  float* m_pool;   // packed per (head, query tile) rows (row_off): m~
+  float* d_pool;   //                                                d~
   int n_q_heads;
   int n_kv_heads;
-  int n_tiles;
+  int n_tiles;     // query tiles Tq
+  int n_kv_tiles;  // key blocks Tk = q_tile0 + Tq
+  int q_tile0;
   int block;
   int group;
   int heads_per_cta;  // query heads of one KV head per CTA (divides group)

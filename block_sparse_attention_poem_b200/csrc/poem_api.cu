@@ -30,7 +30,10 @@ bool aligned16(const void* p) { return p != nullptr && (reinterpret_cast<uintptr
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 struct Layout {
-  int T;       // tiles
+  int T;       // query tiles
+  int t0;      // global tile of the first query tile (q_offset / block)
+  int Tk;      // key blocks (t0 + T)
+  int n_kv;    // key / value tokens (q_offset + n_tokens)
   int G;       // query heads per KV head
   float scale; // softmax scale
 };
@@ -44,40 +47,51 @@ poem_status check_shape(const poem_shape* s, Layout* out) {
     return arg_fail(POEM_ERR_INVALID_ARG, "sizes must be positive");
   if (s->n_q_heads % s->n_kv_heads) return arg_fail(POEM_ERR_INVALID_ARG, "n_q_heads % n_kv_heads != 0");
   if (s->n_tokens % s->block) return arg_fail(POEM_ERR_INVALID_ARG, "n_tokens % block != 0");
+  if (s->q_offset < 0 || s->q_offset % s->block)
+    return arg_fail(POEM_ERR_INVALID_ARG, "q_offset must be >= 0 and a multiple of block");
+  if ((int64_t)s->q_offset + s->n_tokens > (int64_t)INT32_MAX)
+    return arg_fail(POEM_ERR_INVALID_ARG, "q_offset + n_tokens overflows int32");
   if (!(s->softmax_scale >= 0.f) || !std::isfinite(s->softmax_scale))
     return arg_fail(POEM_ERR_INVALID_ARG, "softmax_scale must be finite and >= 0");
   if (s->head_dim != 64 && s->head_dim != 128) return arg_fail(POEM_ERR_UNSUPPORTED, "head_dim must be 64 or 128");
   if (s->block != 64 && s->block != 128) return arg_fail(POEM_ERR_UNSUPPORTED, "block must be 64 or 128");
-  if (s->n_tokens / s->block > kMaxTiles) return arg_fail(POEM_ERR_UNSUPPORTED, "more than 8192 tiles");
+  if ((s->q_offset + s->n_tokens) / s->block > kMaxTiles)
+    return arg_fail(POEM_ERR_UNSUPPORTED, "more than 8192 key blocks");
   const int64_t strides[6] = {s->q_stride_tok, s->q_stride_head, s->kv_stride_tok,
                               s->kv_stride_head, s->o_stride_tok, s->o_stride_head};
   for (int64_t st : strides)
     if (st <= 0 || (st % 8) != 0 || st >= (int64_t(1) << 38))
       return arg_fail(POEM_ERR_INVALID_ARG, "strides must be positive multiples of 8 elements");
   out->T = s->n_tokens / s->block;
+  out->t0 = s->q_offset / s->block;
+  out->Tk = out->t0 + out->T;
+  out->n_kv = s->q_offset + s->n_tokens;
   out->G = s->n_q_heads / s->n_kv_heads;
   out->scale = s->softmax_scale > 0.f ? s->softmax_scale : 1.0f / std::sqrt((float)s->head_dim);
   return POEM_OK;
 }
 
-size_t tri_entries(const poem_shape* s, int T) { return (size_t)s->n_q_heads * (size_t)T * (size_t)(T + 1) / 2; }
+// Entries of the per-(head, query tile, visible block) arrays (row_off layout).
+size_t tri_entries(const poem_shape* s, const Layout& L) {
+  return (size_t)s->n_q_heads * (size_t)poem::row_entries(L.T, L.t0);
+}
 
 size_t score_ws_bytes(const poem_shape* s, int T) {
   const size_t rows = (size_t)s->n_q_heads * T * s->n_sample;
   return poem::kWsHeader + round_up(rows * s->head_dim * sizeof(float), 256) + round_up(rows * sizeof(float), 256);
 }
 
-size_t select_ws_bytes(const poem_shape* s, int T) {
-  const size_t rows = (size_t)s->n_q_heads * T;
-  return poem::kWsHeader + round_up(rows * sizeof(int32_t), 256) + round_up(tri_entries(s, T) * sizeof(int32_t), 256);
+size_t select_ws_bytes(const poem_shape* s, const Layout& L) {
+  const size_t rows = (size_t)s->n_q_heads * L.T;
+  return poem::kWsHeader + round_up(rows * sizeof(int32_t), 256) + round_up(tri_entries(s, L) * sizeof(int32_t), 256);
 }
 
 size_t fwd_ws_bytes(const poem_shape*, int) { return poem::kWsHeader; }
 
-// Pooled means (fp32) after the header: q~ [Hq, T, D], then k~ channel-major
-// [Hkv, D, T], v~ [Hkv, T, D] and v~ channel-major [Hkv, D, T].
-size_t pooled_ws_bytes(const poem_shape* s, int T) {
-  const size_t qn = (size_t)s->n_q_heads * T * s->head_dim, kn = (size_t)s->n_kv_heads * T * s->head_dim;
+// Pooled means (fp32) after the header: q~ [Hq, Tq, D], then k~ channel-major
+// [Hkv, D, Tk], v~ [Hkv, Tk, D] and v~ channel-major [Hkv, D, Tk].
+size_t pooled_ws_bytes(const poem_shape* s, const Layout& L) {
+  const size_t qn = (size_t)s->n_q_heads * L.T * s->head_dim, kn = (size_t)s->n_kv_heads * L.Tk * s->head_dim;
   return poem::kWsHeader + round_up(qn * sizeof(float), 256) + 3 * round_up(kn * sizeof(float), 256);
 }
 
@@ -150,7 +164,7 @@ poem_status poem_workspace_size(const poem_shape* shape, size_t* score_bytes, si
   poem_status st = check_shape(shape, &L);
   if (st != POEM_OK) return st;
   if (score_bytes) *score_bytes = score_ws_bytes(shape, L.T);
-  if (select_bytes) *select_bytes = select_ws_bytes(shape, L.T);
+  if (select_bytes) *select_bytes = select_ws_bytes(shape, L);
   if (fwd_bytes) *fwd_bytes = fwd_ws_bytes(shape, L.T);
   return POEM_OK;
 }
@@ -167,10 +181,10 @@ poem_status poem_score(const poem_shape* shape, const poem_bf16* q, const poem_b
   if (ws_bytes < score_ws_bytes(shape, L.T)) return arg_fail(POEM_ERR_WORKSPACE, "score workspace too small");
   CUtensorMap tmQs, tmK, tmV;
   if ((st = make_map_sampled(&tmQs, q, shape, L.T)) != POEM_OK) return st;
-  if ((st = make_map_3d(&tmK, k, shape->head_dim, shape->n_kv_heads, shape->n_tokens, shape->kv_stride_head,
+  if ((st = make_map_3d(&tmK, k, shape->head_dim, shape->n_kv_heads, L.n_kv, shape->kv_stride_head,
                         shape->kv_stride_tok, shape->block)) != POEM_OK)
     return st;
-  if ((st = make_map_3d(&tmV, v, shape->head_dim, shape->n_kv_heads, shape->n_tokens, shape->kv_stride_head,
+  if ((st = make_map_3d(&tmV, v, shape->head_dim, shape->n_kv_heads, L.n_kv, shape->kv_stride_head,
                         shape->kv_stride_tok, shape->block)) != POEM_OK)
     return st;
   const size_t rows = (size_t)shape->n_q_heads * L.T * shape->n_sample;
@@ -184,6 +198,7 @@ poem_status poem_score(const poem_shape* shape, const poem_bf16* q, const poem_b
   p.n_q_heads = shape->n_q_heads;
   p.n_kv_heads = shape->n_kv_heads;
   p.n_tiles = L.T;
+  p.q_tile0 = L.t0;
   p.group = L.G;
   p.n_sample = shape->n_sample;
   p.sample_stride = shape->block / shape->n_sample;
@@ -214,7 +229,7 @@ static poem_status select_common(const poem_shape* shape, const float* I_hat, co
     return arg_fail(POEM_ERR_INVALID_ARG, "pointers must be non-NULL and 16-byte aligned");
   if (col_capacity < 0) return arg_fail(POEM_ERR_INVALID_ARG, "col_capacity < 0");
   if (!mass_only && (!std::isfinite(tau) || tau < 0.0)) return arg_fail(POEM_ERR_INVALID_ARG, "tau must be finite and >= 0");
-  if (ws_bytes < select_ws_bytes(shape, L.T)) return arg_fail(POEM_ERR_WORKSPACE, "select workspace too small");
+  if (ws_bytes < select_ws_bytes(shape, L)) return arg_fail(POEM_ERR_WORKSPACE, "select workspace too small");
   if (order && L.G * L.T > (1 << 14)) return arg_fail(POEM_ERR_UNSUPPORTED, "work order needs group*tiles <= 16384");
   const size_t rows = (size_t)shape->n_q_heads * L.T;
   uint8_t* base = reinterpret_cast<uint8_t*>(ws);
@@ -230,6 +245,7 @@ static poem_status select_common(const poem_shape* shape, const float* I_hat, co
   p.col_capacity = col_capacity;
   p.n_q_heads = shape->n_q_heads;
   p.n_tiles = L.T;
+  p.q_tile0 = L.t0;
   p.group = L.G;
   p.tau = tau;
   p.mass_only = mass_only;
@@ -272,7 +288,7 @@ poem_status poem_pooled_workspace_size(const poem_shape* shape, size_t* pooled_b
   Layout L;
   poem_status st = check_shape(shape, &L);
   if (st != POEM_OK) return st;
-  if (pooled_bytes) *pooled_bytes = pooled_ws_bytes(shape, L.T);
+  if (pooled_bytes) *pooled_bytes = pooled_ws_bytes(shape, L);
   return POEM_OK;
 }
 
@@ -283,9 +299,9 @@ poem_status poem_score_pooled(const poem_shape* shape, const poem_bf16* q, const
   if (st != POEM_OK) return st;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(m_pool) || !aligned16(d_pool) || !aligned16(ws))
     return arg_fail(POEM_ERR_INVALID_ARG, "pointers must be non-NULL and 16-byte aligned");
-  if (ws_bytes < pooled_ws_bytes(shape, L.T)) return arg_fail(POEM_ERR_WORKSPACE, "pooled workspace too small");
+  if (ws_bytes < pooled_ws_bytes(shape, L)) return arg_fail(POEM_ERR_WORKSPACE, "pooled workspace too small");
   const size_t qn = (size_t)shape->n_q_heads * L.T * shape->head_dim;
-  const size_t kn = (size_t)shape->n_kv_heads * L.T * shape->head_dim;
+  const size_t kn = (size_t)shape->n_kv_heads * L.Tk * shape->head_dim;
   uint8_t* base = reinterpret_cast<uint8_t*>(ws) + poem::kWsHeader;
   poem::PoolParams p{};
   p.q = reinterpret_cast<const __nv_bfloat16*>(q);
@@ -305,6 +321,8 @@ poem_status poem_score_pooled(const poem_shape* shape, const poem_bf16* q, const
   p.n_q_heads = shape->n_q_heads;
   p.n_kv_heads = shape->n_kv_heads;
   p.n_tiles = L.T;
+  p.n_kv_tiles = L.Tk;
+  p.q_tile0 = L.t0;
   p.block = shape->block;
   p.group = L.G;
   p.scale = L.scale;
@@ -339,10 +357,10 @@ poem_status bsa_fwd(const poem_shape* shape, const poem_bf16* q, const poem_bf16
   if ((st = make_map_3d(&tmQ, q, shape->head_dim, shape->n_q_heads, shape->n_tokens, shape->q_stride_head,
                         shape->q_stride_tok, 128)) != POEM_OK)
     return st;
-  if ((st = make_map_3d(&tmK, k, shape->head_dim, shape->n_kv_heads, shape->n_tokens, shape->kv_stride_head,
+  if ((st = make_map_3d(&tmK, k, shape->head_dim, shape->n_kv_heads, L.n_kv, shape->kv_stride_head,
                         shape->kv_stride_tok, shape->block)) != POEM_OK)
     return st;
-  if ((st = make_map_3d(&tmV, v, shape->head_dim, shape->n_kv_heads, shape->n_tokens, shape->kv_stride_head,
+  if ((st = make_map_3d(&tmV, v, shape->head_dim, shape->n_kv_heads, L.n_kv, shape->kv_stride_head,
                         shape->kv_stride_tok, shape->block)) != POEM_OK)
     return st;
   poem::FwdParams p{};
@@ -356,6 +374,7 @@ poem_status bsa_fwd(const poem_shape* shape, const poem_bf16* q, const poem_bf16
   p.n_tokens = shape->n_tokens;
   p.n_q_heads = shape->n_q_heads;
   p.n_tiles = L.T;
+  p.q_tile0 = L.t0;
   p.group = L.G;
   p.scale_log2 = L.scale * poem::kLog2e;
   p.err = dev_err(ws);

@@ -28,6 +28,8 @@
 //                    d~      lane per block like the logits, v~ - o~ squared
 //                  The k~ / v~ of a KV head (T * D * 4 bytes each) stay in L2
 //                  across its CTAs; no warp shuffles on the per-block paths.
+// With a query offset (chunked prefill) q~ covers the Tq query tiles, k~ / v~
+// all q_tile0 + Tq key blocks, and local tile i sees blocks 0 .. q_tile0 + i.
 #include "common.cuh"
 
 namespace poem {
@@ -39,21 +41,17 @@ constexpr int kScoreWarps = kScoreThreads / 32;
 constexpr int kMaxRows = 8;
 constexpr size_t kPooledSmemCap = 200 * 1024;
 
-__device__ __forceinline__ int64_t tri_off(int n_tiles, int h, int i) {
-  return (int64_t)h * ((int64_t)n_tiles * (n_tiles + 1) / 2) + (int64_t)i * (i + 1) / 2;
-}
-
 template <int D>
 __global__ void __launch_bounds__(kPoolThreads) pool_mean_kernel(const PoolParams p) {
   constexpr int C8 = D / 8;
   const int which = blockIdx.z;  // 0: q, 1: k, 2: v
   const int heads = which == 0 ? p.n_q_heads : p.n_kv_heads;
   const int u = blockIdx.y * kPoolThreads + threadIdx.x;
-  if (u >= heads * C8) return;
+  const int i = blockIdx.x;                            // query tile (q) or key block (k, v)
+  const int T = which == 0 ? p.n_tiles : p.n_kv_tiles;
+  if (u >= heads * C8 || i >= T) return;
   const int h = u / C8;
   const int c8 = u - h * C8;
-  const int i = blockIdx.x;
-  const int T = p.n_tiles;
   const __nv_bfloat16* src = which == 0 ? p.q : (which == 1 ? p.k : p.v);
   const int64_t st_tok = which == 0 ? p.q_stride_tok : p.kv_stride_tok;
   const int64_t st_head = which == 0 ? p.q_stride_head : p.kv_stride_head;
@@ -102,8 +100,10 @@ template <int D, int R>
 __global__ void __launch_bounds__(kScoreThreads) pooled_scores_kernel(const PoolParams p) {
   constexpr int S = kScoreThreads / D;  // block slices of the o~ pass
   extern __shared__ __align__(16) float smf[];
-  const int T = p.n_tiles;
-  const int ld = (T + 3) & ~3;
+  const int T = p.n_tiles;      // query tiles
+  const int Tk = p.n_kv_tiles;  // key blocks
+  const int t0 = p.q_tile0;
+  const int ld = (Tk + 3) & ~3;
   float* qb = smf;                // [R][D]
   float* ob = qb + R * D;         // [R][D]
   float* part = ob + R * D;       // [S][R][D]
@@ -114,22 +114,22 @@ __global__ void __launch_bounds__(kScoreThreads) pooled_scores_kernel(const Pool
   const int n_hchunks = p.n_q_heads / Rh;
   const int tg = blockIdx.x / n_hchunks;
   const int h0 = (blockIdx.x - tg * n_hchunks) * Rh;
-  const int i_top = T - 1 - tg * Rt;  // tiles i_top, i_top - 1, ..., i_top - Rt + 1 (those >= 0)
+  const int i_top = T - 1 - tg * Rt;  // local tiles i_top, i_top - 1, ..., i_top - Rt + 1 (those >= 0)
   const int g = h0 / p.group;
-  const int nbmax = i_top + 1;
+  const int nbmax = i_top + t0 + 1;   // key blocks of the longest row
   const int nb4 = (nbmax + 3) & ~3;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const float* kT = p.k_bar_t + (int64_t)g * D * T;
-  const float* vT = p.v_bar_t + (int64_t)g * D * T;
-  const float* vb = p.v_bar + (int64_t)g * T * D;
+  const float* kT = p.k_bar_t + (int64_t)g * D * Tk;
+  const float* vT = p.v_bar_t + (int64_t)g * D * Tk;
+  const float* vb = p.v_bar + (int64_t)g * Tk * D;
 
-  // Row r: head h0 + r % Rh, tile i_top - r / Rh (invalid when the tile is < 0
-  // or r >= Rh * Rt); nb_r = tile + 1 visible blocks, 0 for invalid rows.
+  // Row r: head h0 + r % Rh, local tile i_top - r / Rh (invalid when the tile is
+  // < 0 or r >= Rh * Rt); nb_r = t0 + tile + 1 visible blocks, 0 for invalid rows.
   int nb[R];
 #pragma unroll
   for (int r = 0; r < R; ++r) {
     const int tile = (r < Rh * Rt) ? i_top - r / Rh : -1;
-    nb[r] = tile >= 0 ? tile + 1 : 0;
+    nb[r] = tile >= 0 ? t0 + tile + 1 : 0;
   }
   if (threadIdx.x < R) {
     const int r = threadIdx.x;
@@ -154,7 +154,7 @@ __global__ void __launch_bounds__(kScoreThreads) pooled_scores_kernel(const Pool
     for (int c = 0; c < D; c += 4) {
       float kv[4];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) kv[e] = ok ? kT[(int64_t)(c + e) * T + b] : 0.f;
+      for (int e = 0; e < 4; ++e) kv[e] = ok ? kT[(int64_t)(c + e) * Tk + b] : 0.f;
       const uint64_t k01 = f2_pack(kv[0], kv[1]), k23 = f2_pack(kv[2], kv[3]);
 #pragma unroll
       for (int r = 0; r < R; ++r) {
@@ -178,7 +178,7 @@ __global__ void __launch_bounds__(kScoreThreads) pooled_scores_kernel(const Pool
   // from nb_r up to the 4-block boundary of the longest row are zeroed.
   for (int r = warp; r < R; r += kScoreWarps) {
     float* row = buf + r * ld;
-    const int n = (s_tile[r] >= 0) ? s_tile[r] + 1 : 0;
+    const int n = (s_tile[r] >= 0) ? t0 + s_tile[r] + 1 : 0;
     if (n > 0) {
       float mx = -INFINITY;
       for (int b = lane; b < n; b += 32) mx = fmaxf(mx, row[b]);
@@ -191,7 +191,7 @@ __global__ void __launch_bounds__(kScoreThreads) pooled_scores_kernel(const Pool
       }
       den = warp_sum(den);
       const float inv = 1.0f / den;
-      float* dst = p.m_pool + tri_off(T, s_head[r], s_tile[r]);
+      float* dst = p.m_pool + row_off(T, t0, s_head[r], s_tile[r]);
       for (int b = lane; b < n; b += 32) {
         const float m = row[b] * inv;
         row[b] = m;
@@ -246,7 +246,7 @@ __global__ void __launch_bounds__(kScoreThreads) pooled_scores_kernel(const Pool
     for (int c = 0; c < D; c += 4) {
       float vv[4];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) vv[e] = ok ? vT[(int64_t)(c + e) * T + b] : 0.f;
+      for (int e = 0; e < 4; ++e) vv[e] = ok ? vT[(int64_t)(c + e) * Tk + b] : 0.f;
       const uint64_t v01 = f2_pack(vv[0], vv[1]), v23 = f2_pack(vv[2], vv[3]);
 #pragma unroll
       for (int r = 0; r < R; ++r) {
@@ -269,8 +269,8 @@ __global__ void __launch_bounds__(kScoreThreads) pooled_scores_kernel(const Pool
   __syncthreads();
   for (int r = 0; r < R; ++r) {
     if (s_tile[r] < 0) continue;
-    const int n = s_tile[r] + 1;
-    float* dst = p.d_pool + tri_off(T, s_head[r], s_tile[r]);
+    const int n = t0 + s_tile[r] + 1;
+    float* dst = p.d_pool + row_off(T, t0, s_head[r], s_tile[r]);
     for (int b = threadIdx.x; b < n; b += kScoreThreads) dst[b] = buf[r * ld + b];
   }
 }
@@ -292,7 +292,7 @@ cudaError_t launch_scores_r(const PoolParams& p, cudaStream_t stream) {
   }
   const int n_tgroups = (p.n_tiles + p.tiles_per_cta - 1) / p.tiles_per_cta;
   const int grid = n_tgroups * (p.n_q_heads / p.heads_per_cta);
-  pooled_scores_kernel<D, R><<<grid, kScoreThreads, pooled_smem(R, p.n_tiles, D), stream>>>(p);
+  pooled_scores_kernel<D, R><<<grid, kScoreThreads, pooled_smem(R, p.n_kv_tiles, D), stream>>>(p);
   return cudaGetLastError();
 }
 
@@ -320,19 +320,19 @@ cudaError_t launch_pooled(int head_dim, PoolParams p, cudaStream_t stream) {
   if (p.n_tiles <= 0) return cudaSuccess;
   int rh = 1;
   for (int r = kMaxRows; r >= 1; --r)
-    if (p.group % r == 0 && pooled_smem(r, p.n_tiles, head_dim) <= kPooledSmemCap) {
+    if (p.group % r == 0 && pooled_smem(r, p.n_kv_tiles, head_dim) <= kPooledSmemCap) {
       rh = r;
       break;
     }
   int rt = 1;
   for (int t = kMaxRows / rh; t >= 1; --t)
-    if (pooled_smem(rh * t, p.n_tiles, head_dim) <= kPooledSmemCap) {
+    if (pooled_smem(rh * t, p.n_kv_tiles, head_dim) <= kPooledSmemCap) {
       rt = t;
       break;
     }
   p.heads_per_cta = rh;
   p.tiles_per_cta = rt;
-  const dim3 pg(p.n_tiles, (p.n_q_heads * (head_dim / 8) + kPoolThreads - 1) / kPoolThreads, 3);
+  const dim3 pg(p.n_kv_tiles, (p.n_q_heads * (head_dim / 8) + kPoolThreads - 1) / kPoolThreads, 3);
   if (head_dim == 128) {
     pool_mean_kernel<128><<<pg, kPoolThreads, 0, stream>>>(p);
     cudaError_t e = cudaGetLastError();

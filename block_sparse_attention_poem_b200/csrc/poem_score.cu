@@ -19,6 +19,9 @@
 // 2 adjacent tiles x 4 heads for 4-way GQA.  The 16 rows of a group are gathered
 // by one 4-D TMA box (dims: head_dim, head, sample j, tile i).  A CTA sweeps key
 // blocks 0 .. (largest tile among its groups); a query masks keys after itself.
+// With a query offset (chunked prefill) local query tile i is global tile
+// q_tile0 + i: its sampled queries sit at key positions (q_tile0 + i) B + j (B / S)
+// and its score row has q_tile0 + i + 1 entries (row_off layout).
 //
 // Pipeline (one CTA per SM, TMEM fully allocated):
 //   TMEM  S0 [0,128)  S1 [128,256)  -- S double-buffered: S_{b+1} is computed while
@@ -179,8 +182,9 @@ __global__ void __launch_bounds__(ScoreCfg<D, BN, PASS>::kThreads, 1)
   int g, z0;
   score_cta_coords(blockIdx.x, ctas_per_g, g, z0);
   const int z_last = min(z0 + 7, n_groups - 1);
-  const int nb = z_last / G + 1;  // key blocks 0 .. largest tile of the CTA
-  const int i_lo = z0 / G;        // smallest tile of the CTA: blocks < i_lo need no mask
+  const int t0 = p.q_tile0;            // global index of local query tile 0
+  const int nb = z_last / G + 1 + t0;  // key blocks 0 .. largest (global) tile of the CTA
+  const int i_lo = z0 / G + t0;        // smallest global tile of the CTA: blocks < i_lo need no mask
 
   if (tid == 0) {
     mbar_init(&sb->q_full, 1);
@@ -300,7 +304,7 @@ __global__ void __launch_bounds__(ScoreCfg<D, BN, PASS>::kThreads, 1)
     const bool valid = (z < n_groups);
     const int i = valid ? z / G : 0;
     const int hq = g * G + (valid ? z - i * G : 0);
-    const int qpos = valid ? i * BN + j * p.sample_stride : -1;  // -1: padding row, sees nothing
+    const int qpos = valid ? (i + t0) * BN + j * p.sample_stride : -1;  // key position; -1: padding row
     const int64_t srow = ((int64_t)hq * p.n_tiles + i) * p.n_sample + j;  // sampled-row index
     const uint32_t lane_off = ((uint32_t)(warp * 32) << 16);
     const uint32_t tO = tmem + lane_off + C::kColO;
@@ -439,7 +443,7 @@ __global__ void __launch_bounds__(ScoreCfg<D, BN, PASS>::kThreads, 1)
       }
       tmem_st_wait();
     }
-    const int64_t tri = (int64_t)hq * ((int64_t)p.n_tiles * (p.n_tiles + 1) / 2) + (int64_t)i * (i + 1) / 2;
+    const int64_t tri = row_off(p.n_tiles, t0, hq, i);
     for (int b = 0; b < nb; ++b) {
       const int s = b & 1;
       if (!warp_wait(&sb->pv_full, b & 1, sb, p.err)) break;
@@ -481,7 +485,7 @@ __global__ void __launch_bounds__(ScoreCfg<D, BN, PASS>::kThreads, 1)
         Ib = fmaxf(Ib, __shfl_xor_sync(0xffffffffu, Ib, off));
         mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, off));
       }
-      if (j == 0 && valid && b <= i) {
+      if (j == 0 && valid && b <= i + t0) {
         p.I_hat[tri + b] = Ib;
         p.m_hat[tri + b] = mb;
       }

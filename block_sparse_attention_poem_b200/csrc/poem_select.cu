@@ -37,9 +37,6 @@ namespace {
 
 constexpr int kSelThreads = 256;
 
-__device__ __forceinline__ int64_t tri_off(int n_tiles, int h, int i) {
-  return (int64_t)h * ((int64_t)n_tiles * (n_tiles + 1) / 2) + (int64_t)i * (i + 1) / 2;
-}
 
 // Ascending bitonic sort of n (power of two) 64-bit keys in shared memory.
 __device__ void bitonic_sort_u64(uint64_t* a, int n) {
@@ -210,8 +207,8 @@ __device__ void block_suffix_scan_d2(double a, double b, double* tmpa, double* t
   __syncthreads();
 }
 
-// Ascending compaction of the kept flags of block ids 0..i into the row's
-// triangular scratch slot; the list length goes to counts[row].
+// Ascending compaction of the kept flags of block ids 0..i (i: the row's global
+// tile) into the row's scratch slot at offset off; the length goes to counts[row].
 __device__ void emit_row(const SelectParams& p, const int* keep, int row, int i, int64_t off, int* tmpi) {
   const int n = i + 1;
   const int E2 = (n + kSelThreads - 1) / kSelThreads;
@@ -232,17 +229,18 @@ __global__ void __launch_bounds__(kSelThreads) select_rows_kernel(const SelectPa
   const int row = blockIdx.x;
   const int T = p.n_tiles;
   const int h = row / T;
-  const int i = row - h * T;
+  const int il = row - h * T;       // local query tile
+  const int i = il + p.q_tile0;     // global tile: blocks 0..i visible
   const int nc = max(0, i - 2);
   int P = 1;
   while (P < nc) P <<= 1;
   uint64_t* keys = reinterpret_cast<uint64_t*>(sm);                      // [P]
-  int* keep = reinterpret_cast<int*>(sm + sizeof(uint64_t) * (size_t)max(P, 1));  // [T]
+  int* keep = reinterpret_cast<int*>(sm + sizeof(uint64_t) * (size_t)max(P, 1));  // [i + 1]
   __shared__ double tmpa[kSelThreads / 32], tmpb[kSelThreads / 32];
   __shared__ int tmpi[kSelThreads / 32];
   __shared__ int s_kcut;
 
-  const int64_t off = tri_off(T, h, i);
+  const int64_t off = row_off(T, p.q_tile0, h, il);
   const float* Ih = p.I_hat + off;
   const float* mh = p.m_hat + off;
   const float* rank_src = p.mass_only ? mh : Ih;
@@ -309,18 +307,19 @@ __global__ void __launch_bounds__(kSelThreads) select_practical_rows_kernel(cons
   const int row = blockIdx.x;
   const int T = p.n_tiles;
   const int h = row / T;
-  const int i = row - h * T;
+  const int il = row - h * T;       // local query tile
+  const int i = il + p.q_tile0;     // global tile: blocks 0..i visible
   const int nc = max(0, i - 2);
   int P = 1;
   while (P < nc) P <<= 1;
   uint64_t* keys = reinterpret_cast<uint64_t*>(sm);                    // [P]
   uint32_t* ids = reinterpret_cast<uint32_t*>(sm + sizeof(uint64_t) * (size_t)P);  // [P]
-  int* keep = reinterpret_cast<int*>(sm + (sizeof(uint64_t) + sizeof(uint32_t)) * (size_t)P);  // [T]
+  int* keep = reinterpret_cast<int*>(sm + (sizeof(uint64_t) + sizeof(uint32_t)) * (size_t)P);  // [i + 1]
   __shared__ double tmpd[kSelThreads / 32];
   __shared__ int tmpi[kSelThreads / 32];
   __shared__ int s_kcut;
 
-  const int64_t off = tri_off(T, h, i);
+  const int64_t off = row_off(T, p.q_tile0, h, il);
   const float* mp = p.m_hat + off;
   const float* dp = p.d_pool + off;
 
@@ -427,7 +426,7 @@ __global__ void __launch_bounds__(128) gather_lists_kernel(const SelectParams p)
   const int i = row - h * T;
   const int64_t start = p.row_ptr[row];
   const int n = p.counts[row];
-  const int32_t* src = p.scratch + tri_off(T, h, i);
+  const int32_t* src = p.scratch + row_off(T, p.q_tile0, h, i);
   const int64_t cap = p.col_capacity;
   for (int x = threadIdx.x; x < n; x += blockDim.x) {
     const int64_t d = start + x;
@@ -460,10 +459,11 @@ __global__ void __launch_bounds__(1024) work_order_kernel(const SelectParams p, 
 cudaError_t launch_select(const SelectParams& p, cudaStream_t stream) {
   const int rows = p.n_q_heads * p.n_tiles;
   if (rows <= 0) return cudaSuccess;
+  const int n_blocks = p.n_tiles + p.q_tile0;  // key blocks of the longest row
   int P = 1;
-  while (P < p.n_tiles) P <<= 1;
+  while (P < n_blocks) P <<= 1;
   if (p.practical) {
-    const size_t smem = (sizeof(uint64_t) + sizeof(uint32_t)) * (size_t)P + sizeof(int) * (size_t)p.n_tiles + 16;
+    const size_t smem = (sizeof(uint64_t) + sizeof(uint32_t)) * (size_t)P + sizeof(int) * (size_t)n_blocks + 16;
     static size_t pconf = 0;
     if (smem > 48 * 1024 && smem > pconf) {
       cudaError_t e =
@@ -473,7 +473,7 @@ cudaError_t launch_select(const SelectParams& p, cudaStream_t stream) {
     }
     select_practical_rows_kernel<<<rows, kSelThreads, smem, stream>>>(p);
   } else {
-    const size_t smem = sizeof(uint64_t) * (size_t)P + sizeof(int) * (size_t)p.n_tiles + 16;
+    const size_t smem = sizeof(uint64_t) * (size_t)P + sizeof(int) * (size_t)n_blocks + 16;
     static size_t configured = 0;
     if (smem > 48 * 1024 && smem > configured) {
       cudaError_t e =

@@ -105,6 +105,7 @@ extern "C" poem_status poem_select_noalloc(const poem_shape* shape, const float*
   p.col_capacity = col_capacity;
   p.n_q_heads = shape->n_q_heads;
   p.n_tiles = T;
+  p.q_tile0 = shape->q_offset / shape->block;
   p.group = G;
   p.tau = (double)tau;
   p.mass_only = 0;

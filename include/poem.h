@@ -62,13 +62,21 @@ typedef enum poem_status {
 /*
  * Problem shape of one attention layer.
  *   q: [n_tokens, n_q_heads, head_dim], element (t, h, c) at
- *      q[t*q_stride_tok + h*q_stride_head + c]; k, v: [n_tokens, n_kv_heads,
- *      head_dim] with kv_stride_*; o like q with o_stride_*.
+ *      q[t*q_stride_tok + h*q_stride_head + c]; o like q with o_stride_*.
+ *   k, v: [q_offset + n_tokens, n_kv_heads, head_dim] with kv_stride_*.
  *   Query head h reads KV head h / (n_q_heads / n_kv_heads) (GQA).
- *   block: key block size = query tile size B; T = n_tokens / B tiles; tile i
- *      holds queries iB..iB+B-1 and sees key blocks 0..i (causal).
+ *   block: key block size = query tile size B; T = n_tokens / B query tiles.
+ *   q_offset: position of the first query among the keys (chunked prefill: the
+ *      queries are the last n_tokens of the q_offset + n_tokens visible tokens;
+ *      0 for a whole prefill).  Must be a multiple of block.  Query tile i holds
+ *      the queries at key positions q_offset + iB .. q_offset + iB + B - 1, is
+ *      global tile t0 + i (t0 = q_offset / B) and sees key blocks 0..t0+i
+ *      (causal).
  *   n_sample: S sampled queries per tile for scoring, rows iB + j*(B/S).
  *   softmax_scale: logit scale; 0 selects 1/sqrt(head_dim).
+ * Per-(head, query tile, visible block) arrays (scores, estimates) hold row
+ * (h, i) at h*E + i*t0 + i*(i+1)/2, E = T*t0 + T*(T+1)/2 entries per head
+ * (t0 = 0: the packed lower triangle h*T*(T+1)/2 + i*(i+1)/2).
  */
 typedef struct poem_shape {
   int32_t n_tokens;
@@ -78,7 +86,7 @@ typedef struct poem_shape {
   int32_t block;
   int32_t n_sample;
   float softmax_scale;
-  int32_t reserved0;
+  int32_t q_offset;
   int64_t q_stride_tok, q_stride_head;
   int64_t kv_stride_tok, kv_stride_head;
   int64_t o_stride_tok, o_stride_head;
@@ -96,12 +104,13 @@ poem_status poem_workspace_size(const poem_shape* shape, size_t* score_bytes, si
  * Section 4.1 (m_b, v_b, o) and Equation (4) (I_b = m_b ||v_b - o||) of the
  * reading note; sampling (S strided queries per tile) and max-aggregation are
  * the hot-path contract's choices.
- * For each query head h, tile i and visible block b <= i:
+ * For each query head h, query tile i (global tile g = t0 + i) and visible
+ * block b <= g:
  *   I_hat[h, i, b] = max_j I_b(q_j),  m_hat[h, i, b] = max_j m_b(q_j)
  * over the sampled queries q_j = iB + j*(B/S), j = 0..S-1, with dense causal
  * softmax attention of q_j over keys 0..q_j.
- * Outputs (fp32, packed lower-triangular): entry (h, i, b) at
- *   h*T*(T+1)/2 + i*(i+1)/2 + b; n_q_heads*T*(T+1)/2 entries each.
+ * Outputs (fp32, packed per (head, query tile) row, see poem_shape): entry
+ *   (h, i, b) at h*E + i*t0 + i*(i+1)/2 + b; n_q_heads*E entries each.
  * ws: at least score_bytes (holds per-sampled-query dense outputs and
  *   log-sum-exps between the two passes).
  */
@@ -110,7 +119,8 @@ poem_status poem_score(const poem_shape* shape, const poem_bf16* q, const poem_b
 
 /*
  * poem_select -- threshold selection per (head, tile), Equation (4).
- * Row r = h*T + i.  Mandatory: sink block 0, local block i-1 (i >= 1) and the
+ * Row r = h*T + i; below, i stands for the row's global tile t0 + i (block ids
+ * are global).  Mandatory: sink block 0, local block i-1 (i >= 1) and the
  * diagonal block i.  Candidates 1..i-2 are ranked by (I_hat desc, id asc) --
  * equal scores favour the smaller id, the convention of the "Block-Filtered
  * Long-Context Attention" page, Appendix "Block ordering".  With D_k the
@@ -121,7 +131,7 @@ poem_status poem_score(const poem_shape* shape, const poem_bf16* q, const poem_b
  *   and col_idx[row_ptr[r] .. row_ptr[r+1]) the kept ids of row r in
  *   ascending order.  col_capacity: entries available in col_idx; when the
  *   lists need more, col_idx holds a truncated prefix and POEM_ERR_CAPACITY is
- *   reported by poem_check (n_q_heads*T*(T+1)/2 always suffices).
+ *   reported by poem_check (n_q_heads*E always suffices).
  * order (nullable): int32[n_q_heads*T], a work order for bsa_fwd -- rows grouped
  *   by KV head, longest list first, ties by row id.
  * tau: absolute bound on the per-query head-output error in V's units; must be
@@ -200,8 +210,8 @@ poem_status poem_pooled_workspace_size(const poem_shape* shape, size_t* pooled_b
 
 /*
  * poem_score_pooled -- m~ and d~ for every (head, tile, visible block).
- * Outputs (fp32, packed lower-triangular like poem_score's): entry (h, i, b) at
- *   h*T*(T+1)/2 + i*(i+1)/2 + b.  fp32 arithmetic throughout.
+ * Outputs (fp32, in poem_score's row layout): entry (h, i, b) at
+ *   h*E + i*t0 + i*(i+1)/2 + b.  fp32 arithmetic throughout.
  * ws: at least pooled_bytes; holds the pooled means after the call.
  * n_sample is ignored.
  */
@@ -210,8 +220,8 @@ poem_status poem_score_pooled(const poem_shape* shape, const poem_bf16* q, const
 
 /*
  * poem_select_practical -- two-stage selection per (head, tile) from m~, d~.
- * Row r = h*T + i.  Mandatory: blocks 0, i-1 (i >= 1) and i.  Candidates
- * 1..i-2:
+ * Row r = h*T + i (i below: the row's global tile t0 + i).  Mandatory: blocks
+ * 0, i-1 (i >= 1) and i.  Candidates 1..i-2:
  *   stage 1: ranked by (m~ desc, id asc); the first ceil(rho * |Cand|) form the
  *            shortlist (rho in [0, 1]);
  *   stage 2: the shortlist ranked by (log m~ + w * log d~ desc, id asc), in
@@ -228,10 +238,11 @@ poem_status poem_select_practical(const poem_shape* shape, const float* m_pool, 
 
 /*
  * bsa_fwd -- causal GQA block-sparse attention forward.
- * Query t of head h in tile i attends, with softmax, to the keys u <= t whose
+ * Query t of head h in query tile i (key position q_offset + t, global tile
+ * g = t0 + i) attends, with softmax, to the keys u <= q_offset + t whose
  * block is listed in col_idx[row_ptr[r] .. row_ptr[r+1]), r = h*T + i
  * (the renormalised output o~ of Section 4.1).  Lists must be ascending and
- * hold ids in 0..i; an id outside that range is skipped and reported as
+ * hold ids in 0..g; an id outside that range is skipped and reported as
  * POEM_ERR_BAD_LIST by poem_check.  A row with no visible key outputs 0 and
  * lse = -inf.
  * o: bf16 output with o_stride_*; lse (nullable): fp32 [n_q_heads, n_tokens],

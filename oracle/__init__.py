@@ -59,6 +59,7 @@ class _Shape(ctypes.Structure):
         ("n_sample", ctypes.c_int),
         ("scale", ctypes.c_double),
         ("in_kind", ctypes.c_int),
+        ("q_offset", ctypes.c_int),
     ]
 
 
@@ -122,9 +123,12 @@ def _ip(a):
 class Problem:
     """Q, K, V of one attention layer, as seen by the oracle.
 
-    q: [n_tokens, n_q_heads, head_dim]; k, v: [n_tokens, n_kv_heads, head_dim].
-    Either all float64 or all uint16 (bf16 bit patterns).  ``scale`` defaults
-    to 1/sqrt(head_dim).
+    k, v: [n_tokens, n_kv_heads, head_dim]; q: [n_tokens - q_offset, n_q_heads,
+    head_dim], the queries at positions q_offset .. n_tokens-1 (q_offset =
+    len(k) - len(q), 0 for a whole prefill, a multiple of block otherwise: a
+    chunked prefill).  Tiles and token positions are global; only tiles >=
+    q_offset / block hold queries.  Either all float64 or all uint16 (bf16 bit
+    patterns).  ``scale`` defaults to 1/sqrt(head_dim).
     """
 
     q: np.ndarray
@@ -145,10 +149,12 @@ class Problem:
         self.q = np.ascontiguousarray(self.q)
         self.k = np.ascontiguousarray(self.k)
         self.v = np.ascontiguousarray(self.v)
-        n, hq, d = self.q.shape
-        nk, hkv, dk = self.k.shape
-        if self.v.shape != self.k.shape or nk != n or dk != d:
+        nq, hq, d = self.q.shape
+        n, hkv, dk = self.k.shape
+        if self.v.shape != self.k.shape or nq > n or dk != d:
             raise ValueError("shape mismatch between q, k and v")
+        if (n - nq) % self.block:
+            raise ValueError("q_offset = len(k) - len(q) must be a multiple of block")
         if hq % hkv:
             raise ValueError("n_q_heads must be a multiple of n_kv_heads")
         if n % self.block:
@@ -157,11 +163,19 @@ class Problem:
             raise ValueError("n_sample must divide block")
         if self.scale is None:
             self.scale = 1.0 / np.sqrt(d)
-        self._shape = _Shape(n, hq, hkv, d, self.block, self.n_sample, float(self.scale), self._kind)
+        self._shape = _Shape(n, hq, hkv, d, self.block, self.n_sample, float(self.scale), self._kind, n - nq)
 
     @property
     def n_tokens(self):
-        return self.q.shape[0]
+        return self.k.shape[0]
+
+    @property
+    def q_offset(self):
+        return self.k.shape[0] - self.q.shape[0]
+
+    @property
+    def q_tile0(self):
+        return self.q_offset // self.block
 
     @property
     def n_q_heads(self):

@@ -31,6 +31,9 @@
  *
  * Inputs are [n_tokens, n_heads, head_dim] row-major arrays, either fp64
  * (in_kind 0) or raw bf16 bit patterns (in_kind 1), widened exactly to fp64.
+ * For a chunked prefill (q_offset > 0) q holds only the rows of the positions
+ * q_offset .. n_tokens-1; every function takes global token positions and
+ * global tiles and must only be asked about query positions >= q_offset.
  * All arithmetic is fp64.  Parallelism is OpenMP over independent
  * (head, query tile) units only; each unit is computed by the plain loops
  * below with no blocking or reordering.
@@ -49,6 +52,8 @@ typedef struct oracle_shape {
     int n_sample;  /* sampled queries per tile; must divide block */
     double scale;  /* softmax scale applied to q.k */
     int in_kind;   /* 0: double arrays, 1: bf16 bit patterns (uint16) */
+    int q_offset;  /* position of the first query among the keys (chunked prefill):
+                      q holds rows for positions q_offset .. n_tokens-1 only */
 } oracle_shape;
 
 /* ---- element access ------------------------------------------------------ */
@@ -68,6 +73,11 @@ static double elem(const oracle_shape* s, const void* x, int n_heads, int t, int
     return ((const double*)x)[idx];
 }
 
+/* Query row at key position t (t >= q_offset). */
+static double qelem(const oracle_shape* s, const void* q, int t, int h, int c) {
+    return elem(s, q, s->n_q_heads, t - s->q_offset, h, c);
+}
+
 static int kv_head_of(const oracle_shape* s, int h) {
     int g = s->n_q_heads / s->n_kv_heads; /* query heads per KV head (GQA) */
     return h / g;
@@ -78,7 +88,7 @@ static double logit(const oracle_shape* s, const void* q, const void* k, int h, 
     int hk = kv_head_of(s, h);
     double acc = 0.0;
     for (int c = 0; c < s->head_dim; ++c)
-        acc += elem(s, q, s->n_q_heads, t, h, c) * elem(s, k, s->n_kv_heads, u, hk, c);
+        acc += qelem(s, q, t, h, c) * elem(s, k, s->n_kv_heads, u, hk, c);
     return s->scale * acc;
 }
 
@@ -407,7 +417,7 @@ void oracle_pooled_units(const oracle_shape* s, const void* q, const void* k, co
         double* lg = (double*)malloc(sizeof(double) * (size_t)nb);
         double* om = (double*)calloc((size_t)d, sizeof(double));
         for (int t = i * B; t < (i + 1) * B; ++t)
-            for (int c = 0; c < d; ++c) qm[c] += elem(s, q, s->n_q_heads, t, h, c) / B;
+            for (int c = 0; c < d; ++c) qm[c] += qelem(s, q, t, h, c) / B;
         for (int b = 0; b < nb; ++b)
             for (int t = b * B; t < (b + 1) * B; ++t)
                 for (int c = 0; c < d; ++c) {

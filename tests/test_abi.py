@@ -44,7 +44,7 @@ def test_library_exports_every_declared_symbol(poem):
 
 def _shape(poem, **kw):
     base = dict(n_tokens=1024, n_q_heads=4, n_kv_heads=2, head_dim=128, block=128, n_sample=16, softmax_scale=0.0,
-                reserved0=0, q_stride_tok=512, q_stride_head=128, kv_stride_tok=256, kv_stride_head=128,
+                q_offset=0, q_stride_tok=512, q_stride_head=128, kv_stride_tok=256, kv_stride_head=128,
                 o_stride_tok=512, o_stride_head=128)
     base.update(kw)
     return poem.Shape(**base)
@@ -152,3 +152,24 @@ def test_select_practical_rejects_null_deviation_and_small_workspace(poem):
                                            None) == 1
     assert poem._lib.poem_select_practical(ctypes.byref(sh), ok, ok, 1.0, 0.9, 0.5, ok, ok, 100, None, ok, 8,
                                            None) == 6
+
+
+def test_query_offset_shape(poem):
+    import torch
+
+    q = torch.zeros(256, 2, 128, dtype=torch.bfloat16)
+    k = torch.zeros(256 + 384, 1, 128, dtype=torch.bfloat16)
+    sh = poem.make_shape(q, k, block=128)
+    assert sh.q_offset == 384 and sh.n_tokens == 256
+    st, s, sel, f = _ws(poem, sh)
+    assert st == 0
+    Tq, t0, hq = 2, 3, 2
+    entries = hq * (Tq * t0 + Tq * (Tq + 1) // 2)
+    assert entries == poem.n_score_entries(hq, Tq, t0) == 18  # per head: rows of 4 and 5 blocks
+    assert sel >= 256 + hq * Tq * 4 + entries * 4
+    assert poem.score_row_offset(Tq, t0, 1, 1) == 9 + 4
+    for bad in (64, -128):  # not a multiple of block / negative
+        st, *_ = _ws(poem, _shape(poem, q_offset=bad))
+        assert st == 1
+    with pytest.raises(ValueError):
+        poem.make_shape(k, q)  # fewer keys than queries
