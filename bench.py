@@ -134,11 +134,12 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
-def retained_flops(row_ptr: np.ndarray, col_idx: np.ndarray, n_tiles: int, d: int, B: int) -> float:
-    """4 d (kept query-key pairs): full blocks B^2 pairs, the diagonal block B(B+1)/2."""
+def retained_flops(row_ptr: np.ndarray, col_idx: np.ndarray, n_tiles: int, d: int, B: int, q_tile0: int = 0) -> float:
+    """4 d (kept query-key pairs): full blocks B^2 pairs, the diagonal block B(B+1)/2.
+    Row r is query tile r % n_tiles, global tile q_tile0 + r % n_tiles."""
     rows = len(row_ptr) - 1
     counts = np.diff(row_ptr).astype(np.int64)
-    tiles = np.arange(rows) % n_tiles
+    tiles = np.arange(rows) % n_tiles + q_tile0
     # diagonal present? (lists are ascending: last entry == tile)
     last = np.where(counts > 0, col_idx[np.maximum(row_ptr[1:] - 1, 0)], -1)
     diag = (last == tiles).astype(np.int64)
@@ -163,10 +164,23 @@ def reduce_max(value: float) -> float:
     return float(t.item())
 
 
-def whole_job_ms_per_layer(max_rank_ms: float, steps: int, world: int) -> float:
-    """Every rank runs `steps` layers (independent replicas); the job's ms per layer is
-    the slowest rank's time over all layers the job processed."""
-    return max_rank_ms / (steps * world)
+def whole_job_ms_per_layer(max_rank_ms: float, steps: int, world: int, sharded: bool = False) -> float:
+    """Replicas: every rank runs `steps` whole layers, so the job's ms per layer is the
+    slowest rank's time over all steps * world layers.  Head-sharded: the ranks
+    together run one layer per step, so it is the slowest rank's time per step."""
+    return max_rank_ms / (steps if sharded else steps * world)
+
+
+def shard_heads(n_q_heads: int, n_kv_heads: int, world: int, rank: int):
+    """Head sharding of one layer (as in tensor-parallel attention): rank r owns KV
+    heads [r Hkv/N, (r+1) Hkv/N) and the query heads that read them.  Every
+    (head, tile) unit is independent, so no collective is needed.  Returns
+    ((q_head_lo, q_head_hi), (kv_head_lo, kv_head_hi))."""
+    if n_kv_heads % world:
+        raise ValueError(f"{n_kv_heads} KV heads do not split over {world} ranks")
+    per = n_kv_heads // world
+    group = n_q_heads // n_kv_heads
+    return (rank * per * group, (rank + 1) * per * group), (rank * per, (rank + 1) * per)
 
 
 def dist_setup():
@@ -192,6 +206,13 @@ def run_ours(args):
     n, hq, hkv, d, B, base, tau = WORKLOADS[args.workload]
     T = n // B
     x = poem_synth.heavy_block_layer(n, hq, hkv, d, block=B, rope_base=base, seed=args.seed)
+    sharded = args.shard == "heads" and world > 1
+    hq_all, hkv_all = hq, hkv
+    if sharded:  # this rank's heads only, as a tensor-parallel attention layer holds them
+        (qa, qb), (ka, kb) = shard_heads(hq, hkv, world, rank)
+        x = {"q": x["q"][:, qa:qb].contiguous(), "k": x["k"][:, ka:kb].contiguous(),
+             "v": x["v"][:, ka:kb].contiguous()}
+        hq, hkv = qb - qa, kb - ka
     q, k, v = x["q"].to(dev), x["k"].to(dev), x["v"].to(dev)
     practical = args.selector == "practical"
     layer = poem.alloc_layer(q, k, block=B, practical=practical)
@@ -248,7 +269,7 @@ def run_ours(args):
     fwd_ms = float(np.mean([e[2].elapsed_time(e[3]) for e in evs]))
     total_ms = reduce_max(total_ms)
     ms_per_step = total_ms / args.steps
-    ms_per_layer = whole_job_ms_per_layer(total_ms, args.steps, world)
+    ms_per_layer = whole_job_ms_per_layer(total_ms, args.steps, world, sharded)
 
     for ws in (ws_first, layer.ws_select, layer.ws_fwd):
         poem.poem_check(ws)
@@ -295,7 +316,7 @@ def run_ours(args):
         e1.record(stream)
         torch.cuda.synchronize()
         e2e_ms = reduce_max(e0.elapsed_time(e1))
-        e2e = {"value": whole_job_ms_per_layer(e2e_ms, args.e2e_steps, world), "unit": "ms/layer",
+        e2e = {"value": whole_job_ms_per_layer(e2e_ms, args.e2e_steps, world, sharded), "unit": "ms/layer",
                "h2d_bytes_per_step": int(hq_h.numel() * 2 + hk_h.numel() * 2 + hv_h.numel() * 2),
                "d2h_bytes_per_step": int(ho.numel() * 2)}
 
@@ -323,13 +344,14 @@ def run_ours(args):
         "warmup": args.warmup,
         "ms_per_step": round(ms_per_step, 4),
         "higher_is_better": False,
-        "scaling": "weak",
+        "scaling": "strong" if sharded else "weak",
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (seeded heavy-block generator; no model weights or datasets)",
-        "config": {"workload": args.workload, "n_tokens": n, "n_q_heads": hq, "n_kv_heads": hkv, "head_dim": d,
-                   "block": B, "n_sample": 16, **sel_cfg, "seed": args.seed,
-                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+        "config": {"workload": args.workload, "n_tokens": n, "n_q_heads": hq_all, "n_kv_heads": hkv_all,
+                   "head_dim": d, "block": B, "n_sample": 16, **sel_cfg, "seed": args.seed,
+                   "parallelism": (f"head-sharded x{world} ({hq} query / {hkv} KV heads per rank)" if sharded
+                                   else f"replicas x{world}" if world > 1 else "single GPU"),
                    "l2": "inputs larger than L2 (no flush needed)"},
         "breakdown_ms": {names[0]: round(score_ms, 4), names[1]: round(select_ms, 4),
                          "bsa_fwd": round(fwd_ms, 4)},
@@ -737,6 +759,74 @@ def _dense_output(poem, q, k, v, layer, hq, T):
     return o
 
 
+CHUNK_REPORT = [
+    # (context tokens, query-chunk tokens): the last chunk of a long prefill
+    (131072, 16384),
+    (131072, 32768),
+    (65536, 16384),
+]
+
+
+def _report_chunked(poem, steps, warmup):
+    """The last query chunk of a long prefill (queries are the final Nq of N
+    tokens): exact POEM (tau = 0.05) and the practical selector (w = 1,
+    gamma = 0.95, rho = 0.5) on the Llama-shaped heavy-block layer."""
+    out = []
+    peaks, _ = load_peaks()
+    hq, hkv, d, B = 32, 8, 128, 128
+    for n, nq in CHUNK_REPORT:
+        x = poem_synth.heavy_block_layer(n, hq, hkv, d, block=B, rope_base=500000.0, seed=0)
+        q = x["q"][n - nq:].cuda()
+        k, v = x["k"].cuda(), x["v"].cuda()
+        T, t0 = n // B, (n - nq) // B
+        Tq = T - t0
+        visible = hq * (Tq * t0 + Tq * (Tq + 1) // 2)
+        for selector in ("exact", "practical"):
+            layer = poem.alloc_layer(q, k, block=B, practical=(selector == "practical"))
+            ph = {"score": [], "select": [], "bsa_fwd": []}
+            for it in range(warmup + steps):
+                ev = _events(4)
+                ev[0].record()
+                if selector == "exact":
+                    poem.poem_score(q, k, v, layer.I_hat, layer.m_hat, layer.ws_score, shape=layer.shape)
+                else:
+                    poem.poem_score_pooled(q, k, v, layer.m_pool, layer.d_pool, layer.ws_pooled, shape=layer.shape)
+                ev[1].record()
+                if selector == "exact":
+                    poem.poem_select(layer.shape, layer.I_hat, layer.m_hat, 0.05, layer.row_ptr, layer.col_idx,
+                                     layer.ws_select, order=layer.order)
+                else:
+                    poem.poem_select_practical(layer.shape, layer.m_pool, layer.d_pool, 1.0, 0.95, 0.5,
+                                               layer.row_ptr, layer.col_idx, layer.ws_select, order=layer.order)
+                ev[2].record()
+                poem.bsa_fwd(q, k, v, layer.row_ptr, layer.col_idx, layer.o, layer.ws_fwd, order=layer.order,
+                             shape=layer.shape)
+                ev[3].record()
+                torch.cuda.synchronize()
+                if it >= warmup:
+                    for j, key in enumerate(ph):
+                        ph[key].append(ev[j].elapsed_time(ev[j + 1]))
+            for ws in (layer.ws_pooled if selector == "practical" else layer.ws_score, layer.ws_select, layer.ws_fwd):
+                poem.poem_check(ws)
+            ms = {key: float(np.median(val)) for key, val in ph.items()}
+            rp = layer.row_ptr.cpu().numpy()
+            ci = layer.col_idx[: int(rp[-1])].cpu().numpy()
+            rfl = retained_flops(rp, ci, Tq, d, B, q_tile0=t0)
+            fwd_tf = rfl / (ms["bsa_fwd"] * 1e-3) / 1e12
+            dense_fl = 2.0 * d * hq * nq * (2 * (n - nq) + nq + 1)
+            out.append({"config": "chunked-prefill", "context_tokens": n, "query_tokens": nq, "q_offset": n - nq,
+                        "selector": selector, "ms": {key: round(val, 4) for key, val in ms.items()},
+                        "ms_per_chunk": round(sum(ms.values()), 4), "density": round(int(rp[-1]) / visible, 5),
+                        "bsa_fwd_retained_tflops": round(fwd_tf, 2),
+                        "bsa_fwd_frac_sustained": round(fwd_tf / peaks["bf16_tflops_sustained"], 4),
+                        "dense_equiv_tflops": round(dense_fl / (sum(ms.values()) * 1e-3) / 1e12, 2)})
+            del layer
+            torch.cuda.empty_cache()
+        del q, k, v
+        torch.cuda.empty_cache()
+    return out
+
+
 EVAL_LAYERS = [
     ("heavy-block-32k", "heavy"),
     ("contrast-32k", "contrast"),
@@ -821,6 +911,9 @@ def run_report(args):
     if part in (None, "evaluation"):
         for rec in _report_evaluation(poem):
             print(json.dumps(rec), flush=True)
+    if part in (None, "chunked"):
+        for rec in _report_chunked(poem, args.steps, args.warmup):
+            print(json.dumps(rec), flush=True)
     if part in (None, "sweep"):
         for rec in _report_sweep(poem, args.steps, args.warmup):
             print(json.dumps(rec), flush=True)
@@ -842,12 +935,15 @@ def main():
     ap.add_argument("--cpu-budget-s", type=float, default=15.0)
     ap.add_argument("--ref-step-budget-s", type=float, default=8.0)
     ap.add_argument("--selector", choices=["exact", "practical"], default="exact")
+    ap.add_argument("--shard", choices=["replicas", "heads"], default="replicas",
+                    help="N > 1: independent whole-layer replicas (weak scaling) or one layer split by KV-head "
+                         "groups across the ranks (strong scaling)")
     ap.add_argument("--w", type=float, default=1.0, help="practical: weight of log d~ in the rerank key")
     ap.add_argument("--gamma", type=float, default=0.95, help="practical: pooled-mass retention threshold")
     ap.add_argument("--rho", type=float, default=0.5, help="practical: stage-1 shortlist fraction")
     ap.add_argument("--report", action="store_true",
                     help="measure every configuration (one JSON record each) instead of the benchmark line")
-    ap.add_argument("--report-only", choices=["exact", "practical", "evaluation", "sweep"], default=None,
+    ap.add_argument("--report-only", choices=["exact", "practical", "evaluation", "chunked", "sweep"], default=None,
                     help="with --report: only this part")
     args = ap.parse_args()
     if args.report:
