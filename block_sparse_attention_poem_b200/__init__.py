@@ -12,6 +12,8 @@ Functions carry the C names:
     poem_select(I_hat, m_hat, tau, row_ptr, col_idx, ws, shape..., order=None)
     poem_select_mass_only(m_hat, ref_row_ptr, row_ptr, col_idx, ws, ...)
     poem_select_ranked_budget(shape, score, ref_row_ptr, row_ptr, col_idx, ws, ...)
+    poem_select_per_head(shape, I_hat, m_hat, tau_per_head, row_ptr, col_idx, ws, ...)
+    poem_select_practical_per_head(shape, m_pool, d_pool, w, gamma_per_head, rho, ...)
     bsa_fwd(q, k, v, row_ptr, col_idx, o, ws, lse=None, order=None, block=128)
     poem_check(ws) -> raises on a device-side error
     poem_pooled_workspace_size(shape) -> bytes
@@ -41,6 +43,7 @@ EXPORTED = (
     "poem_workspace_size", "poem_score", "poem_select", "poem_select_mass_only", "bsa_fwd",
     "poem_check", "poem_set_wait_limit_ns", "poem_status_string", "poem_last_error", "poem_select_noalloc",
     "poem_pooled_workspace_size", "poem_score_pooled", "poem_select_practical", "poem_select_ranked_budget",
+    "poem_select_per_head", "poem_select_practical_per_head",
 )
 
 
@@ -75,6 +78,11 @@ def _load():
     lib.poem_select.restype = st
     lib.poem_select_mass_only.argtypes = [sp, vp, vp, vp, vp, i64, vp, vp, sz, vp]
     lib.poem_select_mass_only.restype = st
+    lib.poem_select_per_head.argtypes = [sp, vp, vp, vp, vp, vp, i64, vp, vp, sz, vp]
+    lib.poem_select_per_head.restype = st
+    lib.poem_select_practical_per_head.argtypes = [sp, vp, vp, ctypes.c_double, vp, ctypes.c_double, vp, vp, i64,
+                                                   vp, vp, sz, vp]
+    lib.poem_select_practical_per_head.restype = st
     lib.poem_select_ranked_budget.argtypes = [sp, vp, vp, vp, vp, i64, vp, vp, sz, vp]
     lib.poem_select_ranked_budget.restype = st
     lib.poem_select_noalloc.argtypes = [sp, vp, vp, ctypes.c_float, vp, vp, i64, vp, vp]
@@ -173,6 +181,23 @@ def poem_select(shape: Shape, I_hat, m_hat, tau: float, row_ptr, col_idx, ws, or
     _raise(_lib.poem_select(ctypes.byref(shape), _ptr(I_hat), _ptr(m_hat), ctypes.c_float(tau), _ptr(row_ptr),
                             _ptr(col_idx), col_idx.numel(), _ptr(order), _ptr(ws), ws.numel() * ws.element_size(),
                             _stream(stream)), "poem_select")
+
+
+def poem_select_per_head(shape: Shape, I_hat, m_hat, tau_per_head, row_ptr, col_idx, ws, order=None, stream=None):
+    """poem_select with a device tensor of one tau per query head (float32, [n_q_heads])."""
+    _raise(_lib.poem_select_per_head(ctypes.byref(shape), _ptr(I_hat), _ptr(m_hat), _ptr(tau_per_head),
+                                     _ptr(row_ptr), _ptr(col_idx), col_idx.numel(), _ptr(order), _ptr(ws),
+                                     ws.numel() * ws.element_size(), _stream(stream)), "poem_select_per_head")
+
+
+def poem_select_practical_per_head(shape: Shape, m_pool, d_pool, w: float, gamma_per_head, rho: float, row_ptr,
+                                   col_idx, ws, order=None, stream=None):
+    """poem_select_practical with a device tensor of one gamma per query head."""
+    _raise(_lib.poem_select_practical_per_head(ctypes.byref(shape), _ptr(m_pool), _ptr(d_pool), ctypes.c_double(w),
+                                               _ptr(gamma_per_head), ctypes.c_double(rho), _ptr(row_ptr),
+                                               _ptr(col_idx), col_idx.numel(), _ptr(order), _ptr(ws),
+                                               ws.numel() * ws.element_size(), _stream(stream)),
+           "poem_select_practical_per_head")
 
 
 def poem_select_mass_only(shape: Shape, m_hat, ref_row_ptr, row_ptr, col_idx, ws, order=None, stream=None):

@@ -88,11 +88,13 @@ struct SelectParams {
   int q_tile0;   // global tile of the first query tile
   int group;
   double tau;
+  const float* tau_heads;  // nullable: per-query-head tau (device, [n_q_heads]) instead of tau
   int mass_only;
   // Practical selector (pooled estimates): m_hat holds m~, d_pool holds d~.
   const float* d_pool;
   double w;      // weight of log d~ in the rerank key
   double gamma;  // pooled-mass retention threshold
+  const float* gamma_heads;  // nullable: per-query-head gamma (device, [n_q_heads]) instead of gamma
   double rho;    // stage-1 shortlist fraction of the candidates
   int practical;
   DevErr err;

@@ -212,17 +212,21 @@ poem_status poem_score(const poem_shape* shape, const poem_bf16* q, const poem_b
 struct PracticalArgs {
   const float* d_pool;
   double w, gamma, rho;
+  const float* gamma_heads;  // nullable
 };
 
 static poem_status select_common(const poem_shape* shape, const float* I_hat, const float* m_hat,
                                  const int32_t* ref_row_ptr, double tau, int mass_only, int32_t* row_ptr,
                                  int32_t* col_idx, int64_t col_capacity, int32_t* order, void* ws, size_t ws_bytes,
-                                 void* stream, const PracticalArgs* practical = nullptr) {
+                                 void* stream, const PracticalArgs* practical = nullptr,
+                                 const float* tau_heads = nullptr) {
   Layout L;
   poem_status st = check_shape(shape, &L);
   if (st != POEM_OK) return st;
   if (practical && !aligned16(practical->d_pool))
     return arg_fail(POEM_ERR_INVALID_ARG, "pointers must be non-NULL and 16-byte aligned");
+  if ((practical && practical->gamma_heads && !aligned16(practical->gamma_heads)))
+    return arg_fail(POEM_ERR_INVALID_ARG, "gamma_per_head must be 16-byte aligned");
   if ((!mass_only && !practical && !aligned16(I_hat)) || !aligned16(m_hat) || !aligned16(row_ptr) || !aligned16(ws) ||
       (col_capacity > 0 && !aligned16(col_idx)) || (order && !aligned16(order)) ||
       (mass_only && !aligned16(ref_row_ptr)))
@@ -248,12 +252,14 @@ static poem_status select_common(const poem_shape* shape, const float* I_hat, co
   p.q_tile0 = L.t0;
   p.group = L.G;
   p.tau = tau;
+  p.tau_heads = tau_heads;
   p.mass_only = mass_only;
   if (practical) {
     p.practical = 1;
     p.d_pool = practical->d_pool;
     p.w = practical->w;
     p.gamma = practical->gamma;
+    p.gamma_heads = practical->gamma_heads;
     p.rho = practical->rho;
   }
   p.err = dev_err(ws);
@@ -268,6 +274,14 @@ poem_status poem_select(const poem_shape* shape, const float* I_hat, const float
   if (!std::isfinite(tau) || tau < 0.f) return arg_fail(POEM_ERR_INVALID_ARG, "tau must be finite and >= 0");
   return select_common(shape, I_hat, m_hat, nullptr, (double)tau, 0, row_ptr, col_idx, col_capacity, order, ws,
                        ws_bytes, stream);
+}
+
+poem_status poem_select_per_head(const poem_shape* shape, const float* I_hat, const float* m_hat,
+                                 const float* tau_per_head, int32_t* row_ptr, int32_t* col_idx, int64_t col_capacity,
+                                 int32_t* order, void* ws, size_t ws_bytes, void* stream) {
+  if (!aligned16(tau_per_head)) return arg_fail(POEM_ERR_INVALID_ARG, "tau_per_head must be non-NULL and 16-byte aligned");
+  return select_common(shape, I_hat, m_hat, nullptr, 0.0, 0, row_ptr, col_idx, col_capacity, order, ws, ws_bytes,
+                       stream, nullptr, tau_per_head);
 }
 
 poem_status poem_select_mass_only(const poem_shape* shape, const float* m_hat, const int32_t* ref_row_ptr,
@@ -338,7 +352,20 @@ poem_status poem_select_practical(const poem_shape* shape, const float* m_pool, 
   if (!std::isfinite(w) || w < 0.0) return arg_fail(POEM_ERR_INVALID_ARG, "w must be finite and >= 0");
   if (std::isnan(gamma)) return arg_fail(POEM_ERR_INVALID_ARG, "gamma is NaN");
   if (!(rho >= 0.0 && rho <= 1.0)) return arg_fail(POEM_ERR_INVALID_ARG, "rho must lie in [0, 1]");
-  PracticalArgs pa{d_pool, w, gamma, rho};
+  PracticalArgs pa{d_pool, w, gamma, rho, nullptr};
+  return select_common(shape, nullptr, m_pool, nullptr, 0.0, 0, row_ptr, col_idx, col_capacity, order, ws, ws_bytes,
+                       stream, &pa);
+}
+
+poem_status poem_select_practical_per_head(const poem_shape* shape, const float* m_pool, const float* d_pool, double w,
+                                           const float* gamma_per_head, double rho, int32_t* row_ptr,
+                                           int32_t* col_idx, int64_t col_capacity, int32_t* order, void* ws,
+                                           size_t ws_bytes, void* stream) {
+  if (!std::isfinite(w) || w < 0.0) return arg_fail(POEM_ERR_INVALID_ARG, "w must be finite and >= 0");
+  if (!(rho >= 0.0 && rho <= 1.0)) return arg_fail(POEM_ERR_INVALID_ARG, "rho must lie in [0, 1]");
+  if (!aligned16(gamma_per_head))
+    return arg_fail(POEM_ERR_INVALID_ARG, "gamma_per_head must be non-NULL and 16-byte aligned");
+  PracticalArgs pa{d_pool, w, 0.0, rho, gamma_per_head};
   return select_common(shape, nullptr, m_pool, nullptr, 0.0, 0, row_ptr, col_idx, col_capacity, order, ws, ws_bytes,
                        stream, &pa);
 }
@@ -399,6 +426,7 @@ poem_status poem_check(void* stream, void* ws) {
   if (word & poem::kErrTimeout) return POEM_ERR_TIMEOUT;
   if (word & poem::kErrBadList) return POEM_ERR_BAD_LIST;
   if (word & poem::kErrCapacity) return POEM_ERR_CAPACITY;
+  if (word & poem::kErrBadParam) return POEM_ERR_INVALID_ARG;
   return POEM_OK;
 }
 

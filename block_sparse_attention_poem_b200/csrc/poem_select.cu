@@ -37,7 +37,6 @@ namespace {
 
 constexpr int kSelThreads = 256;
 
-
 // Ascending bitonic sort of n (power of two) 64-bit keys in shared memory.
 __device__ void bitonic_sort_u64(uint64_t* a, int n) {
   for (int k = 2; k <= n; k <<= 1) {
@@ -265,6 +264,19 @@ __global__ void __launch_bounds__(kSelThreads) select_rows_kernel(const SelectPa
     const int n_mand = (i == 0) ? 1 : (i == 1 ? 2 : 3);
     kcut = min(max(ref - n_mand, 0), nc);
   } else if (nc > 0) {
+    // Threshold of this row: the call's tau, or its head's entry of tau_heads (a
+    // NaN, negative or infinite entry keeps every candidate and is reported).
+    double tau = p.tau;
+    bool keep_all = false;  // uniform over the CTA
+    if (p.tau_heads) {
+      const float th = p.tau_heads[h];
+      if (!(th >= 0.f) || isinf(th)) {
+        if (threadIdx.x == 0) raise_err(p.err, kErrBadParam);
+        keep_all = true;
+      } else {
+        tau = (double)th;
+      }
+    }
     // Each thread owns a contiguous run of ranks; suffix sums inside the run, then
     // a block suffix scan of the run totals.
     const int E = (nc + kSelThreads - 1) / kSelThreads;
@@ -285,9 +297,9 @@ __global__ void __launch_bounds__(kSelThreads) select_rows_kernel(const SelectPa
       const int id = (int)(keys[r] & 0xffffffffu);
       sa += (double)Ih[id];
       sb2 += (double)mh[id];
-      if (sb2 < 1.0 && sa <= p.tau * (1.0 - sb2)) best = r;
+      if (sb2 < 1.0 && sa <= tau * (1.0 - sb2)) best = r;
     }
-    if (best < nc) atomicMin(&s_kcut, best);
+    if (best < nc && !keep_all) atomicMin(&s_kcut, best);
     __syncthreads();
     kcut = s_kcut;
   }
@@ -351,6 +363,18 @@ __global__ void __launch_bounds__(kSelThreads) select_practical_rows_kernel(cons
   __syncthreads();
   if (n1 > 1) bitonic_sort_pairs(keys, ids, P2);
 
+  // Threshold of this row: the call's gamma, or its head's entry of gamma_heads
+  // (a NaN or infinite entry keeps the whole shortlist and is reported).
+  double gamma = p.gamma;
+  if (p.gamma_heads) {
+    const float gh = p.gamma_heads[h];
+    if (isnan(gh) || isinf(gh)) {
+      if (threadIdx.x == 0) raise_err(p.err, kErrBadParam);
+      gamma = INFINITY;  // never reached: the whole shortlist is kept
+    } else {
+      gamma = (double)gh;
+    }
+  }
   // Threshold: mandatory mass (ascending ids), then the reranked prefix, in fp64.
   double acc0 = (double)mp[0];
   if (i >= 2) acc0 += (double)mp[i - 1];
@@ -364,12 +388,12 @@ __global__ void __launch_bounds__(kSelThreads) select_practical_rows_kernel(cons
   double run = acc0 + carry;
   for (int r = r0; r < r1; ++r) {
     run += (double)mp[ids[r]];
-    if (run >= p.gamma) {
+    if (run >= gamma) {
       atomicMin(&s_kcut, r + 1);
       break;
     }
   }
-  if (threadIdx.x == 0 && acc0 >= p.gamma) atomicMin(&s_kcut, 0);
+  if (threadIdx.x == 0 && acc0 >= gamma) atomicMin(&s_kcut, 0);
   __syncthreads();
   const int kcut = s_kcut;
   for (int r = threadIdx.x; r < kcut; r += blockDim.x) keep[ids[r]] = 1;

@@ -17,6 +17,7 @@ enum : uint32_t {
   kErrTimeout = 1u,      // a bounded wait gave up
   kErrBadList = 2u,      // a block id outside 0..tile (skipped)
   kErrCapacity = 4u,     // col_idx capacity too small (output truncated)
+  kErrBadParam = 8u,     // a per-head threshold was NaN, negative or infinite (row kept whole)
 };
 
 struct DevErr {

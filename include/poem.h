@@ -142,6 +142,19 @@ poem_status poem_select(const poem_shape* shape, const float* I_hat, const float
                         size_t ws_bytes, void* stream);
 
 /*
+ * poem_select_per_head -- poem_select with one tau per query head: the pages
+ * calibrate retention thresholds offline for each head group; a caller passes
+ * its calibrated values here (a group's value repeated over its heads).
+ * tau_per_head: device array of n_q_heads floats, read by the kernel (so a
+ * captured CUDA graph picks up new values without re-capture).  Entries must be
+ * finite and >= 0; a bad entry makes its head's rows keep every candidate and
+ * poem_check reports POEM_ERR_INVALID_ARG.  Outputs and workspace as poem_select.
+ */
+poem_status poem_select_per_head(const poem_shape* shape, const float* I_hat, const float* m_hat,
+                                 const float* tau_per_head, int32_t* row_ptr, int32_t* col_idx, int64_t col_capacity,
+                                 int32_t* order, void* ws, size_t ws_bytes, void* stream);
+
+/*
  * poem_select_mass_only -- the mass-only baseline at a matched budget: row r
  * keeps the mandatory blocks and the (ref_row_ptr[r+1] - ref_row_ptr[r] -
  * |mandatory|) candidates of largest m_hat (ties: smaller id).  Same outputs
@@ -237,6 +250,17 @@ poem_status poem_select_practical(const poem_shape* shape, const float* m_pool, 
                                   int64_t col_capacity, int32_t* order, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * poem_select_practical_per_head -- poem_select_practical with one gamma per
+ * query head (device array of n_q_heads floats, read by the kernel).  A NaN or
+ * infinite entry keeps its head's whole shortlist and poem_check reports
+ * POEM_ERR_INVALID_ARG.
+ */
+poem_status poem_select_practical_per_head(const poem_shape* shape, const float* m_pool, const float* d_pool, double w,
+                                           const float* gamma_per_head, double rho, int32_t* row_ptr,
+                                           int32_t* col_idx, int64_t col_capacity, int32_t* order, void* ws,
+                                           size_t ws_bytes, void* stream);
+
+/*
  * bsa_fwd -- causal GQA block-sparse attention forward.
  * Query t of head h in query tile i (key position q_offset + t, global tile
  * g = t0 + i) attends, with softmax, to the keys u <= q_offset + t whose
@@ -257,7 +281,8 @@ poem_status bsa_fwd(const poem_shape* shape, const poem_bf16* q, const poem_bf16
 /*
  * Synchronise `stream`, read and clear the error word at the start of `ws`
  * (a workspace passed to one of the calls above) and map it to a status:
- * POEM_ERR_TIMEOUT, POEM_ERR_BAD_LIST, POEM_ERR_CAPACITY, or POEM_OK.
+ * POEM_ERR_TIMEOUT, POEM_ERR_BAD_LIST, POEM_ERR_CAPACITY, POEM_ERR_INVALID_ARG
+ * (a bad per-head threshold), or POEM_OK.
  */
 poem_status poem_check(void* stream, void* ws);
 
