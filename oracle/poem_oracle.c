@@ -391,12 +391,12 @@ int oracle_num_threads(void) {
 /* ---- practical (estimated) scoring: pooled block statistics ----------------- */
 
 /*
- * Practical POEM (reading note, the paragraph on Equation (6) and Appendix B)
- * estimates the dense reference and the block outputs instead of computing
- * them, pre-selects candidates by mass, reranks them by an approximate log mass
- * plus a weighted log deviation, and keeps blocks in that order until the
- * accumulated pooled mass reaches the retention threshold.  The estimators are
- * not printed; the reading taken here is the plainest one:
+ * Practical POEM (reading note, the paragraph on Equation (6) and Appendix B):
+ * cheap estimates stand in for the exact dense output and block outputs; a
+ * shortlist of candidates is taken by mass, re-ordered by log mass plus w times
+ * log deviation, and blocks are kept in the new order until their pooled mass
+ * reaches the threshold.  No estimator is printed; the reading taken here is
+ * the plainest one:
  *   q~_i = mean of the B queries of tile i,   k~_b, v~_b = means of block b,
  *   m~_b = softmax over visible b <= i of scale * <q~_i, k~_b>,
  *   o~_i = sum_b m~_b v~_b,   d~_b = || v~_b - o~_i ||.
