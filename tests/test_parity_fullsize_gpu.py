@@ -121,3 +121,29 @@ def test_bsa_fwd_random_masks_128k(poem, density):
     O_ref, _ = problem_from(x, B).masked_units(units, rp, ci)
     mx, mean = compare_fwd(o, O_ref, units, B)
     assert mx <= FWD_MAX_ABS and mean <= FWD_MEAN_ABS, (mx, mean)
+
+
+def test_maximum_tile_count_single_head(poem):
+    """The largest supported layer length: 8192 key blocks (1,048,576 tokens at
+    B = 128), one head, d = 64 -- the largest shared-memory configurations of the
+    selectors, the pooled estimates and the work order.  Exact and practical paths,
+    checked on sampled units (the last tile sees all 8192 blocks)."""
+    n, hq, hkv, d, B = 8192 * 128, 1, 1, 64, 128
+    T = n // B
+    x = poem_synth.heavy_block_layer(n, hq, hkv, d, block=B, rope_base=500000.0, seed=5, n_dir_pairs=4)
+    units = [(0, 0), (0, 3), (0, T // 2), (0, T - 1)]
+    _check_layer(poem, x, B, 0.05, units)
+    q, k, v = x["q"].cuda(), x["k"].cuda(), x["v"].cuda()
+    layer = poem.prefill_layer_practical(q, k, v, 1.0, 0.95, 0.5, block=B)
+    for ws in (layer.ws_pooled, layer.ws_select, layer.ws_fwd):
+        poem.poem_check(ws)
+    rm, rd = problem_from(x, B).pooled_units(units)
+    idx = np.concatenate([np.arange(oracle.tri_offset(T, h, i), oracle.tri_offset(T, h, i) + i + 1) for h, i in units])
+    vbar = float(x["v"].float().view(T, B, hkv, d).mean(1).norm(dim=-1).max())
+    from _parity import pooled_err_excess
+    assert pooled_err_excess(layer.m_pool.cpu().numpy()[idx], rm[idx], layer.d_pool.cpu().numpy()[idx], rd[idx],
+                             vbar) <= 1.0
+    rp = layer.row_ptr.cpu().numpy()
+    rows = csr_rows(rp, layer.col_idx[: int(rp[-1])].cpu().numpy())
+    for h, i in units:
+        assert rows[h * T + i] == sorted(set(rows[h * T + i])) and {0, i} <= set(rows[h * T + i])
