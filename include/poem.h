@@ -103,7 +103,7 @@ poem_status poem_workspace_size(const poem_shape* shape, size_t* score_bytes, si
  * poem_score -- exact block scores on the sampled queries.
  * Section 4.1 (m_b, v_b, o) and Equation (4) (I_b = m_b ||v_b - o||) of the
  * reading note; sampling (S strided queries per tile) and max-aggregation are
- * the hot-path contract's choices.
+ * this library's choices.
  * For each query head h, query tile i (global tile g = t0 + i) and visible
  * block b <= g:
  *   I_hat[h, i, b] = max_j I_b(q_j),  m_hat[h, i, b] = max_j m_b(q_j)

@@ -13,7 +13,7 @@ Every function cites the passage of the method description it follows:
   block mass m_b, weighted block mean v_b, dense output o, renormalised sparse
   output o~, the deletion-error identity (Equation 3) and the per-block proxy
   I_b = m_b ||v_b - o|| with the triangle bound (Equation 4).
-* The hot-path contract fixes what the note leaves open: 16 strided sampled
+* What the note leaves open is fixed as the CUDA library fixes it: 16 strided sampled
   queries per tile, max-aggregation, mandatory blocks {0, i-1, i} and the
   stopping rule  S_m < 1 and S_I <= tau (1 - S_m)  over the discarded suffix.
 * "Block-Filtered Long-Context Attention", Appendix "Block ordering": equal

@@ -20,7 +20,7 @@
  * and the triangle bound || o - o~ || <= sum_{b in D} I_b / (1 - delta).
  *
  * Choices the note leaves open (tile size, sampled queries, aggregation,
- * mandatory blocks, stopping rule) follow the hot-path contract: 16 strided
+ * mandatory blocks, stopping rule) are fixed as in the CUDA library: 16 strided
  * queries per tile (rows i*B + j*(B/S)), max-aggregation of I_b and of m_b,
  * mandatory blocks {0, i-1, i}, and the stopping rule
  *     S_m < 1  and  S_I <= tau * (1 - S_m)

@@ -8,7 +8,7 @@ import torch
 import oracle
 import poem_synth
 
-# Tolerances (hot-path contract): bsa_fwd on an identical list, unit-scale V.
+# Tolerances: bsa_fwd on an identical list, unit-scale V.
 FWD_MAX_ABS = 1e-2
 FWD_MEAN_ABS = 1e-3
 # I_hat / m_hat relative error, with a floor relative to the row maximum.

@@ -199,7 +199,7 @@ def test_select_bit_exact_on_identical_scores(poem, T, hq, hkv, seed):
             w = rng.random(i + 1) ** 4
             mh[off:off + i + 1] = (w / w.sum() * 1.3).astype(np.float32)
     shape = _fake_shape(poem, hq, hkv, T)
-    for tau in (0.0, 0.002, 0.02, 0.1):
+    for tau in (0.0, 0.002, 0.02, 0.1, 1e6):  # 1e6: only the mandatory blocks survive
         rp, ci, order, status = _gpu_select(poem, shape, Ih, mh, tau, hq * T)
         assert status == 0
         rp_ref, ci_ref, _ = oracle.select_all(hq, T, Ih.astype(np.float64), mh.astype(np.float64), tau)
