@@ -400,13 +400,8 @@ template <int D, int BN>
 cudaError_t launch_fwd_t(const CUtensorMap& tmQ, const CUtensorMap& tmK, const CUtensorMap& tmV,
                          const FwdParams& p, int n_units, cudaStream_t stream) {
   using C = FwdCfg<D, BN>;
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(bsa_fwd_kernel<D, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         C::kSmemBytes);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
+  cudaError_t e = ensure_smem_limit(bsa_fwd_kernel<D, BN>, C::kSmemBytes);
+  if (e != cudaSuccess) return e;
   bsa_fwd_kernel<D, BN><<<n_units, kThreadsFwd, C::kSmemBytes, stream>>>(tmQ, tmK, tmV, p);
   return cudaGetLastError();
 }

@@ -5,9 +5,33 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <map>
+#include <mutex>
+#include <utility>
+
 #include "sm100.cuh"
 
 namespace poem {
+
+// Raise a kernel's dynamic shared-memory limit to at least `bytes` on the current
+// device.  The attribute is per device, so the setting is remembered per (kernel,
+// device); thread-safe.  Sizes up to the 48 KB default need no call.
+template <typename F>
+inline cudaError_t ensure_smem_limit(F* func, size_t bytes) {
+  if (bytes <= 48 * 1024) return cudaSuccess;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  static std::mutex mu;
+  static std::map<std::pair<const void*, int>, size_t> done;
+  std::lock_guard<std::mutex> lock(mu);
+  const auto key = std::make_pair(reinterpret_cast<const void*>(func), dev);
+  const auto it = done.find(key);
+  if (it != done.end() && it->second >= bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e == cudaSuccess) done[key] = bytes;
+  return e;
+}
 
 constexpr int kWsHeader = 256;          // bytes reserved at the start of every workspace
 constexpr int kThreadsFwd = 192;        // 4 softmax warps + 1 TMA warp + 1 MMA warp

@@ -283,13 +283,8 @@ size_t pooled_smem(int R, int T, int D) {
 
 template <int D, int R>
 cudaError_t launch_scores_r(const PoolParams& p, cudaStream_t stream) {
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(pooled_scores_kernel<D, R>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)kPooledSmemCap);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
+  cudaError_t e = ensure_smem_limit(pooled_scores_kernel<D, R>, kPooledSmemCap);
+  if (e != cudaSuccess) return e;
   const int n_tgroups = (p.n_tiles + p.tiles_per_cta - 1) / p.tiles_per_cta;
   const int grid = n_tgroups * (p.n_q_heads / p.heads_per_cta);
   pooled_scores_kernel<D, R><<<grid, kScoreThreads, pooled_smem(R, p.n_kv_tiles, D), stream>>>(p);

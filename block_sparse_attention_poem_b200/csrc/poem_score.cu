@@ -505,13 +505,8 @@ template <int D, int BN, int PASS>
 cudaError_t launch_pass(const CUtensorMap& tmQs, const CUtensorMap& tmK, const CUtensorMap& tmV,
                         const ScoreParams& p, int grid, cudaStream_t stream) {
   using C = ScoreCfg<D, BN, PASS>;
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(poem_score_kernel<D, BN, PASS>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
+  cudaError_t e = ensure_smem_limit(poem_score_kernel<D, BN, PASS>, C::kSmemBytes);
+  if (e != cudaSuccess) return e;
   poem_score_kernel<D, BN, PASS><<<grid, C::kThreads, C::kSmemBytes, stream>>>(tmQs, tmK, tmV, p);
   return cudaGetLastError();
 }

@@ -488,23 +488,13 @@ cudaError_t launch_select(const SelectParams& p, cudaStream_t stream) {
   while (P < n_blocks) P <<= 1;
   if (p.practical) {
     const size_t smem = (sizeof(uint64_t) + sizeof(uint32_t)) * (size_t)P + sizeof(int) * (size_t)n_blocks + 16;
-    static size_t pconf = 0;
-    if (smem > 48 * 1024 && smem > pconf) {
-      cudaError_t e =
-          cudaFuncSetAttribute(select_practical_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      if (e != cudaSuccess) return e;
-      pconf = smem;
-    }
+    cudaError_t e = ensure_smem_limit(select_practical_rows_kernel, smem);
+    if (e != cudaSuccess) return e;
     select_practical_rows_kernel<<<rows, kSelThreads, smem, stream>>>(p);
   } else {
     const size_t smem = sizeof(uint64_t) * (size_t)P + sizeof(int) * (size_t)n_blocks + 16;
-    static size_t configured = 0;
-    if (smem > 48 * 1024 && smem > configured) {
-      cudaError_t e =
-          cudaFuncSetAttribute(select_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      if (e != cudaSuccess) return e;
-      configured = smem;
-    }
+    cudaError_t e = ensure_smem_limit(select_rows_kernel, smem);
+    if (e != cudaSuccess) return e;
     select_rows_kernel<<<rows, kSelThreads, smem, stream>>>(p);
   }
   scan_counts_kernel<<<1, 1024, 0, stream>>>(p.counts, p.row_ptr, rows);
@@ -514,12 +504,8 @@ cudaError_t launch_select(const SelectParams& p, cudaStream_t stream) {
     int sp = 1;
     while (sp < seg) sp <<= 1;
     const size_t osmem = sizeof(uint32_t) * (size_t)sp;
-    static size_t oconf = 0;
-    if (osmem > 48 * 1024 && osmem > oconf) {
-      cudaError_t e = cudaFuncSetAttribute(work_order_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)osmem);
-      if (e != cudaSuccess) return e;
-      oconf = osmem;
-    }
+    cudaError_t e = ensure_smem_limit(work_order_kernel, osmem);
+    if (e != cudaSuccess) return e;
     work_order_kernel<<<p.n_q_heads / p.group, 1024, osmem, stream>>>(p, sp);
   }
   return cudaGetLastError();
