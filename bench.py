@@ -53,9 +53,9 @@ WORKLOADS = {
 # MEASURED_PEAKS.json, when present, takes precedence).
 FALLBACK_PEAKS = {"bf16_tflops": 1667.9, "bf16_tflops_sustained": 1378.8, "hbm_gbs": 6452.5}
 # DRAM bytes per bsa_fwd launch on the 128K layer: the ncu capture of the 32K layer
-# (dram__bytes_read.sum + dram__bytes_write.sum = 407.0 + 233.5 = 640.5 MB per launch)
+# (dram__bytes_read.sum + dram__bytes_write.sum = 407.6 + 233.3 = 640.9 MB per launch)
 # scaled by rows processed (x4).  Valid only for the kernel source it was taken on.
-BSA_FWD_TRAFFIC = {"bytes": 2.562e9, "source_sha256_prefix": "6603b0060543b045",
+BSA_FWD_TRAFFIC = {"bytes": 2.564e9, "source_sha256_prefix": "aede93e9ca9611e3",
                    "note": "ncu dram bytes of the 32K layer launch x4 rows"}
 
 
