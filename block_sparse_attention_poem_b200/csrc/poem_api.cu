@@ -232,6 +232,8 @@ static poem_status select_common(const poem_shape* shape, const float* I_hat, co
       (mass_only && !aligned16(ref_row_ptr)))
     return arg_fail(POEM_ERR_INVALID_ARG, "pointers must be non-NULL and 16-byte aligned");
   if (col_capacity < 0) return arg_fail(POEM_ERR_INVALID_ARG, "col_capacity < 0");
+  if (tri_entries(shape, L) > (size_t)INT32_MAX)
+    return arg_fail(POEM_ERR_UNSUPPORTED, "the block lists could exceed int32 row_ptr offsets (too many heads x tiles)");
   if (!mass_only && (!std::isfinite(tau) || tau < 0.0)) return arg_fail(POEM_ERR_INVALID_ARG, "tau must be finite and >= 0");
   if (ws_bytes < select_ws_bytes(shape, L)) return arg_fail(POEM_ERR_WORKSPACE, "select workspace too small");
   if (order && L.G * L.T > (1 << 14)) return arg_fail(POEM_ERR_UNSUPPORTED, "work order needs group*tiles <= 16384");

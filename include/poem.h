@@ -127,6 +127,8 @@ poem_status poem_score(const poem_shape* shape, const poem_bf16* q, const poem_b
  * candidates ranked k, k+1, ..., S_I = sum_{D_k} I_hat and S_m = sum_{D_k}
  * m_hat (fp64), the row keeps the top k for the smallest k with
  *     S_m < 1  and  S_I <= tau * (1 - S_m).
+ * Shapes whose lists could exceed int32 offsets (n_q_heads*E > 2^31 - 1) are
+ * POEM_ERR_UNSUPPORTED.
  * Outputs: row_ptr[n_q_heads*T + 1] (int32, exclusive scan of list lengths)
  *   and col_idx[row_ptr[r] .. row_ptr[r+1]) the kept ids of row r in
  *   ascending order.  col_capacity: entries available in col_idx; when the

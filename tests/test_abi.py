@@ -173,3 +173,13 @@ def test_query_offset_shape(poem):
         assert st == 1
     with pytest.raises(ValueError):
         poem.make_shape(k, q)  # fewer keys than queries
+
+
+def test_select_rejects_lists_beyond_int32_offsets(poem):
+    # 128 heads x 8192 tiles: 128 * 8192 * 8193 / 2 > 2^31 - 1 entries
+    sh = _shape(poem, n_tokens=8192 * 128, n_q_heads=128, n_kv_heads=8, q_stride_tok=128 * 128,
+                o_stride_tok=128 * 128, kv_stride_tok=8 * 128)
+    ok = ctypes.c_void_p(1 << 20)
+    st = poem._lib.poem_select(ctypes.byref(sh), ok, ok, ctypes.c_float(0.05), ok, ok, 100, None, ok, 1 << 62, None)
+    assert st == 2
+    assert "int32" in poem.poem_last_error()
