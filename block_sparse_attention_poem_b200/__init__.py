@@ -170,8 +170,16 @@ def _check_bf16(*ts):
             raise TypeError("q, k, v, o must be CUDA bfloat16 tensors")
 
 
+def _check_kv(k, v):
+    """The ABI describes K and V with one shape and one stride pair."""
+    if k.shape != v.shape or k.stride() != v.stride():
+        raise ValueError(f"k and v must have the same shape and strides (k {tuple(k.shape)} {k.stride()}, "
+                         f"v {tuple(v.shape)} {v.stride()})")
+
+
 def poem_score(q, k, v, I_hat, m_hat, ws, shape: Shape | None = None, stream=None, **shape_kw):
     _check_bf16(q, k, v)
+    _check_kv(k, v)
     shape = shape or make_shape(q, k, **shape_kw)
     _raise(_lib.poem_score(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(I_hat), _ptr(m_hat), _ptr(ws),
                            ws.numel() * ws.element_size(), _stream(stream)), "poem_score")
@@ -233,6 +241,7 @@ def poem_pooled_workspace_size(shape: Shape) -> int:
 def poem_score_pooled(q, k, v, m_pool, d_pool, ws, shape: Shape | None = None, stream=None, **shape_kw):
     """Pooled estimates m~ and d~ (packed lower-triangular fp32) for the practical selector."""
     _check_bf16(q, k, v)
+    _check_kv(k, v)
     shape = shape or make_shape(q, k, **shape_kw)
     _raise(_lib.poem_score_pooled(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(m_pool), _ptr(d_pool),
                                   _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)), "poem_score_pooled")
@@ -250,6 +259,9 @@ def poem_select_practical(shape: Shape, m_pool, d_pool, w: float, gamma: float, 
 def bsa_fwd(q, k, v, row_ptr, col_idx, o, ws, lse=None, order=None, shape: Shape | None = None, stream=None,
             **shape_kw):
     _check_bf16(q, k, v, o)
+    _check_kv(k, v)
+    if o.shape != q.shape:
+        raise ValueError("o must have q's shape")
     shape = shape or make_shape(q, k, o=o, **shape_kw)
     _raise(_lib.bsa_fwd(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(row_ptr), _ptr(col_idx), _ptr(order),
                         _ptr(o), _ptr(lse), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)), "bsa_fwd")
@@ -297,7 +309,9 @@ class Layer:
 
 
 def alloc_layer(q, k, block: int = 128, n_sample: int = 16, with_lse: bool = False, practical: bool = False) -> Layer:
-    shape = make_shape(q, k, block=block, n_sample=n_sample)
+    # O is allocated contiguous and the shape takes O's own strides (q may be a padded view)
+    o = torch.empty(q.shape, dtype=q.dtype, device=q.device)
+    shape = make_shape(q, k, block=block, n_sample=n_sample, o=o)
     n, hq, d = q.shape
     T = n // block
     s_b, sel_b, f_b = poem_workspace_size(shape)
@@ -315,7 +329,7 @@ def alloc_layer(q, k, block: int = 128, n_sample: int = 16, with_lse: bool = Fal
         row_ptr=torch.empty(hq * T + 1, dtype=torch.int32, device=dev),
         col_idx=torch.empty(ne, dtype=torch.int32, device=dev),
         order=torch.empty(hq * T, dtype=torch.int32, device=dev),
-        o=torch.empty_like(q),
+        o=o,
         lse=torch.empty(hq, n, dtype=torch.float32, device=dev) if with_lse else None,
         ws_score=alloc_workspace(s_b, dev),
         ws_select=alloc_workspace(sel_b, dev),

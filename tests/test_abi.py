@@ -183,3 +183,14 @@ def test_select_rejects_lists_beyond_int32_offsets(poem):
     st = poem._lib.poem_select(ctypes.byref(sh), ok, ok, ctypes.c_float(0.05), ok, ok, 100, None, ok, 1 << 62, None)
     assert st == 2
     assert "int32" in poem.poem_last_error()
+
+
+def test_binding_rejects_k_v_with_different_layouts(poem):
+    import torch
+
+    q = torch.zeros(256, 2, 128, dtype=torch.bfloat16)
+    k = torch.zeros(256, 1, 128, dtype=torch.bfloat16)
+    v = torch.zeros(256, 2, 160, dtype=torch.bfloat16)[:, :1, :128]  # same shape, other strides
+    with pytest.raises(ValueError):
+        poem._check_kv(k, v)
+    poem._check_kv(k, k.clone())

@@ -351,3 +351,42 @@ def test_prefill_layer_end_to_end(poem, tau):
             od, _ = prob.dense_row(h, t)
             ot, _ = prob.masked_row(h, t, keep)
             assert np.linalg.norm(od - ot) <= tau * (1 + 1e-3) + 1e-6
+
+
+def test_strided_views_match_contiguous(poem):
+    """Q, K, V as padded views (head stride and token stride larger than dense) and a
+    padded O: the layer equals the contiguous run bit for bit, and the padding of O
+    is never written."""
+    n, hq, hkv, d, B, tau = 2048, 4, 2, 128, 128, 0.05
+    x = poem_synth.heavy_block_layer(n, hq, hkv, d, block=B, seed=23)
+    q, k, v = to_dev(x)
+    ref = poem.prefill_layer(q, k, v, tau, block=B)
+    for ws in (ref.ws_score, ref.ws_select, ref.ws_fwd):
+        poem.poem_check(ws)
+
+    def padded(t, extra_heads, extra_dim):
+        big = torch.zeros(t.shape[0], t.shape[1] + extra_heads, t.shape[2] + extra_dim, dtype=t.dtype,
+                          device=t.device)
+        big[:, : t.shape[1], : t.shape[2]] = t
+        return big[:, : t.shape[1], : t.shape[2]]
+
+    qv, kv, vv = padded(q, 1, 64), padded(k, 2, 32), padded(v, 2, 32)  # K and V share one layout (ABI)
+    assert qv.stride() != q.stride() and not qv.is_contiguous()
+    lay = poem.prefill_layer(qv, kv, vv, tau, block=B)
+    for ws in (lay.ws_score, lay.ws_select, lay.ws_fwd):
+        poem.poem_check(ws)
+    assert torch.equal(lay.I_hat, ref.I_hat) and torch.equal(lay.row_ptr, ref.row_ptr)
+    assert torch.equal(lay.o, ref.o)
+    # a padded O written through its own strides
+    ob = torch.full((n, hq, d + 32), 7.0, dtype=torch.bfloat16, device="cuda")
+    ov = ob[:, :, :d]
+    poem.bsa_fwd(qv, kv, vv, ref.row_ptr, ref.col_idx, ov, ref.ws_fwd, block=B)
+    poem.poem_check(ref.ws_fwd)
+    assert torch.equal(ov, ref.o)
+    assert bool((ob[:, :, d:] == 7.0).all())
+    # the practical path reads strided inputs too (pooling)
+    p_ref = poem.prefill_layer_practical(q, k, v, 1.0, 0.95, 0.5, block=B)
+    p_str = poem.prefill_layer_practical(qv, kv, vv, 1.0, 0.95, 0.5, block=B)
+    for ws in (p_ref.ws_pooled, p_str.ws_pooled):
+        poem.poem_check(ws)
+    assert torch.equal(p_ref.m_pool, p_str.m_pool) and torch.equal(p_ref.d_pool, p_str.d_pool)
