@@ -170,6 +170,29 @@ def _check_bf16(*ts):
             raise TypeError("q, k, v, o must be CUDA bfloat16 tensors")
 
 
+def _dims(shape: Shape):
+    """(rows, entries) of a shape: rows = n_q_heads * T, entries of the per-(head,
+    tile, block) arrays."""
+    if shape.block <= 0 or shape.n_tokens <= 0 or shape.n_q_heads <= 0:
+        return 0, 0  # an invalid shape: the library rejects it
+    T = shape.n_tokens // shape.block
+    t0 = max(shape.q_offset, 0) // shape.block
+    return shape.n_q_heads * T, n_score_entries(shape.n_q_heads, T, t0)
+
+
+def _need(t, dtype, min_numel: int, name: str, optional: bool = False):
+    """A device buffer handed to the library: CUDA, contiguous, the right dtype and
+    large enough for what the call writes or reads."""
+    if t is None:
+        if optional:
+            return
+        raise TypeError(f"{name} is required")
+    if not t.is_cuda or t.dtype != dtype or not t.is_contiguous():
+        raise TypeError(f"{name} must be a contiguous CUDA {dtype} tensor (got {t.dtype}, cuda={t.is_cuda})")
+    if t.numel() < min_numel:
+        raise ValueError(f"{name} holds {t.numel()} elements; this shape needs {min_numel}")
+
+
 def _check_kv(k, v):
     """The ABI describes K and V with one shape and one stride pair."""
     if k.shape != v.shape or k.stride() != v.stride():
@@ -181,11 +204,22 @@ def poem_score(q, k, v, I_hat, m_hat, ws, shape: Shape | None = None, stream=Non
     _check_bf16(q, k, v)
     _check_kv(k, v)
     shape = shape or make_shape(q, k, **shape_kw)
+    rows, ne = _dims(shape)
+    _need(I_hat, torch.float32, ne, "I_hat")
+    _need(m_hat, torch.float32, ne, "m_hat")
+    _need(ws, torch.uint8, 0, "ws")
     _raise(_lib.poem_score(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(I_hat), _ptr(m_hat), _ptr(ws),
                            ws.numel() * ws.element_size(), _stream(stream)), "poem_score")
 
 
 def poem_select(shape: Shape, I_hat, m_hat, tau: float, row_ptr, col_idx, ws, order=None, stream=None):
+    rows, ne = _dims(shape)
+    _need(row_ptr, torch.int32, rows + 1, "row_ptr")
+    _need(col_idx, torch.int32, 0, "col_idx")
+    _need(order, torch.int32, rows, "order", optional=True)
+    _need(I_hat, torch.float32, ne, "I_hat")
+    _need(m_hat, torch.float32, ne, "m_hat")
+    _need(ws, torch.uint8, 0, "ws")
     _raise(_lib.poem_select(ctypes.byref(shape), _ptr(I_hat), _ptr(m_hat), ctypes.c_float(tau), _ptr(row_ptr),
                             _ptr(col_idx), col_idx.numel(), _ptr(order), _ptr(ws), ws.numel() * ws.element_size(),
                             _stream(stream)), "poem_select")
@@ -193,6 +227,14 @@ def poem_select(shape: Shape, I_hat, m_hat, tau: float, row_ptr, col_idx, ws, or
 
 def poem_select_per_head(shape: Shape, I_hat, m_hat, tau_per_head, row_ptr, col_idx, ws, order=None, stream=None):
     """poem_select with a device tensor of one tau per query head (float32, [n_q_heads])."""
+    rows, ne = _dims(shape)
+    _need(row_ptr, torch.int32, rows + 1, "row_ptr")
+    _need(col_idx, torch.int32, 0, "col_idx")
+    _need(order, torch.int32, rows, "order", optional=True)
+    _need(I_hat, torch.float32, ne, "I_hat")
+    _need(m_hat, torch.float32, ne, "m_hat")
+    _need(tau_per_head, torch.float32, shape.n_q_heads, "tau_per_head")
+    _need(ws, torch.uint8, 0, "ws")
     _raise(_lib.poem_select_per_head(ctypes.byref(shape), _ptr(I_hat), _ptr(m_hat), _ptr(tau_per_head),
                                      _ptr(row_ptr), _ptr(col_idx), col_idx.numel(), _ptr(order), _ptr(ws),
                                      ws.numel() * ws.element_size(), _stream(stream)), "poem_select_per_head")
@@ -201,6 +243,14 @@ def poem_select_per_head(shape: Shape, I_hat, m_hat, tau_per_head, row_ptr, col_
 def poem_select_practical_per_head(shape: Shape, m_pool, d_pool, w: float, gamma_per_head, rho: float, row_ptr,
                                    col_idx, ws, order=None, stream=None):
     """poem_select_practical with a device tensor of one gamma per query head."""
+    rows, ne = _dims(shape)
+    _need(row_ptr, torch.int32, rows + 1, "row_ptr")
+    _need(col_idx, torch.int32, 0, "col_idx")
+    _need(order, torch.int32, rows, "order", optional=True)
+    _need(m_pool, torch.float32, ne, "m_pool")
+    _need(d_pool, torch.float32, ne, "d_pool")
+    _need(gamma_per_head, torch.float32, shape.n_q_heads, "gamma_per_head")
+    _need(ws, torch.uint8, 0, "ws")
     _raise(_lib.poem_select_practical_per_head(ctypes.byref(shape), _ptr(m_pool), _ptr(d_pool), ctypes.c_double(w),
                                                _ptr(gamma_per_head), ctypes.c_double(rho), _ptr(row_ptr),
                                                _ptr(col_idx), col_idx.numel(), _ptr(order), _ptr(ws),
@@ -209,6 +259,13 @@ def poem_select_practical_per_head(shape: Shape, m_pool, d_pool, w: float, gamma
 
 
 def poem_select_mass_only(shape: Shape, m_hat, ref_row_ptr, row_ptr, col_idx, ws, order=None, stream=None):
+    rows, ne = _dims(shape)
+    _need(row_ptr, torch.int32, rows + 1, "row_ptr")
+    _need(col_idx, torch.int32, 0, "col_idx")
+    _need(order, torch.int32, rows, "order", optional=True)
+    _need(m_hat, torch.float32, ne, "m_hat")
+    _need(ref_row_ptr, torch.int32, rows + 1, "ref_row_ptr")
+    _need(ws, torch.uint8, 0, "ws")
     _raise(_lib.poem_select_mass_only(ctypes.byref(shape), _ptr(m_hat), _ptr(ref_row_ptr), _ptr(row_ptr),
                                       _ptr(col_idx), col_idx.numel(), _ptr(order), _ptr(ws),
                                       ws.numel() * ws.element_size(), _stream(stream)), "poem_select_mass_only")
@@ -216,6 +273,13 @@ def poem_select_mass_only(shape: Shape, m_hat, ref_row_ptr, row_ptr, col_idx, ws
 
 def poem_select_ranked_budget(shape: Shape, score, ref_row_ptr, row_ptr, col_idx, ws, order=None, stream=None):
     """Mandatory blocks + the top candidates by `score` at the per-row budget of ref_row_ptr."""
+    rows, ne = _dims(shape)
+    _need(row_ptr, torch.int32, rows + 1, "row_ptr")
+    _need(col_idx, torch.int32, 0, "col_idx")
+    _need(order, torch.int32, rows, "order", optional=True)
+    _need(score, torch.float32, ne, "score")
+    _need(ref_row_ptr, torch.int32, rows + 1, "ref_row_ptr")
+    _need(ws, torch.uint8, 0, "ws")
     _raise(_lib.poem_select_ranked_budget(ctypes.byref(shape), _ptr(score), _ptr(ref_row_ptr), _ptr(row_ptr),
                                           _ptr(col_idx), col_idx.numel(), _ptr(order), _ptr(ws),
                                           ws.numel() * ws.element_size(), _stream(stream)),
@@ -227,6 +291,12 @@ def poem_select_noalloc(shape: Shape, I_hat, m_hat, tau: float, row_ptr, col_idx
     memory: the scratch is a fixed 8 MiB array inside the library (shared by all
     calls -- do not overlap calls on the GPU).  Check row_ptr[-1] against
     col_idx.numel() afterwards; there is no error word to poll."""
+    rows, ne = _dims(shape)
+    _need(row_ptr, torch.int32, rows + 1, "row_ptr")
+    _need(col_idx, torch.int32, 0, "col_idx")
+    _need(order, torch.int32, rows, "order", optional=True)
+    _need(I_hat, torch.float32, ne, "I_hat")
+    _need(m_hat, torch.float32, ne, "m_hat")
     _raise(_lib.poem_select_noalloc(ctypes.byref(shape), _ptr(I_hat), _ptr(m_hat), ctypes.c_float(tau),
                                     _ptr(row_ptr), _ptr(col_idx), col_idx.numel(), _ptr(order), _stream(stream)),
            "poem_select_noalloc")
@@ -243,6 +313,10 @@ def poem_score_pooled(q, k, v, m_pool, d_pool, ws, shape: Shape | None = None, s
     _check_bf16(q, k, v)
     _check_kv(k, v)
     shape = shape or make_shape(q, k, **shape_kw)
+    rows, ne = _dims(shape)
+    _need(m_pool, torch.float32, ne, "m_pool")
+    _need(d_pool, torch.float32, ne, "d_pool")
+    _need(ws, torch.uint8, 0, "ws")
     _raise(_lib.poem_score_pooled(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(m_pool), _ptr(d_pool),
                                   _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)), "poem_score_pooled")
 
@@ -250,6 +324,13 @@ def poem_score_pooled(q, k, v, m_pool, d_pool, ws, shape: Shape | None = None, s
 def poem_select_practical(shape: Shape, m_pool, d_pool, w: float, gamma: float, rho: float, row_ptr, col_idx, ws,
                           order=None, stream=None):
     """Two-stage practical selection (mass shortlist, log m~ + w log d~ rerank, pooled-mass threshold gamma)."""
+    rows, ne = _dims(shape)
+    _need(row_ptr, torch.int32, rows + 1, "row_ptr")
+    _need(col_idx, torch.int32, 0, "col_idx")
+    _need(order, torch.int32, rows, "order", optional=True)
+    _need(m_pool, torch.float32, ne, "m_pool")
+    _need(d_pool, torch.float32, ne, "d_pool")
+    _need(ws, torch.uint8, 0, "ws")
     _raise(_lib.poem_select_practical(ctypes.byref(shape), _ptr(m_pool), _ptr(d_pool), ctypes.c_double(w),
                                       ctypes.c_double(gamma), ctypes.c_double(rho), _ptr(row_ptr), _ptr(col_idx),
                                       col_idx.numel(), _ptr(order), _ptr(ws), ws.numel() * ws.element_size(),
@@ -263,6 +344,12 @@ def bsa_fwd(q, k, v, row_ptr, col_idx, o, ws, lse=None, order=None, shape: Shape
     if o.shape != q.shape:
         raise ValueError("o must have q's shape")
     shape = shape or make_shape(q, k, o=o, **shape_kw)
+    rows, _ = _dims(shape)
+    _need(row_ptr, torch.int32, rows + 1, "row_ptr")
+    _need(col_idx, torch.int32, 0, "col_idx")  # must hold row_ptr[-1] entries (not checked: on the device)
+    _need(order, torch.int32, rows, "order", optional=True)
+    _need(lse, torch.float32, shape.n_q_heads * shape.n_tokens, "lse", optional=True)
+    _need(ws, torch.uint8, 0, "ws")
     _raise(_lib.bsa_fwd(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(row_ptr), _ptr(col_idx), _ptr(order),
                         _ptr(o), _ptr(lse), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)), "bsa_fwd")
 

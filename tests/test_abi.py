@@ -194,3 +194,19 @@ def test_binding_rejects_k_v_with_different_layouts(poem):
     with pytest.raises(ValueError):
         poem._check_kv(k, v)
     poem._check_kv(k, k.clone())
+
+
+def test_binding_checks_buffer_types_and_sizes(poem):
+    import torch
+
+    sh = _shape(poem)  # 4 q heads, 8 tiles: 32 rows, 144 entries
+    rows, ne = poem._dims(sh)
+    assert (rows, ne) == (32, 144)
+    cpu_f = torch.zeros(ne, dtype=torch.float32)
+    with pytest.raises(TypeError):  # not on a CUDA device
+        poem._need(cpu_f, torch.float32, ne, "I_hat")
+    with pytest.raises(TypeError):
+        poem._need(torch.zeros(ne, dtype=torch.float64), torch.float32, ne, "I_hat")
+    with pytest.raises(TypeError):
+        poem._need(None, torch.int32, rows + 1, "row_ptr")
+    poem._need(None, torch.int32, rows, "order", optional=True)
