@@ -35,7 +35,7 @@
 namespace poem {
 namespace {
 
-constexpr int kSelThreads = 256;
+constexpr int kSelThreads = 128;
 
 // Ascending bitonic sort of n (power of two) 64-bit keys in shared memory.
 __device__ void bitonic_sort_u64(uint64_t* a, int n) {
