@@ -888,6 +888,58 @@ def _report_chunked(poem, steps, warmup):
     return out
 
 
+def _report_dense_context(poem, steps, warmup):
+    """Context only (not the product path): dense causal GQA attention from the
+    framework's own library kernel (torch scaled_dot_product_attention on the
+    device) next to bsa_fwd with every causal block listed, on i.i.d. inputs."""
+    import torch.nn.functional as F
+
+    out = []
+    hq, hkv, d, B = 32, 8, 128, 128
+    for n in (32768, 131072):
+        x = poem_synth.iid_layer(n, hq, hkv, d, seed=0)
+        q, k, v = x["q"].cuda(), x["k"].cuda(), x["v"].cuda()
+        qt, kt, vt = q.permute(1, 0, 2).unsqueeze(0), k.permute(1, 0, 2).unsqueeze(0), v.permute(1, 0, 2).unsqueeze(0)
+        qt, kt, vt = qt.contiguous(), kt.contiguous(), vt.contiguous()
+        times = []
+        for it in range(warmup + steps):
+            ev = _events(2)
+            ev[0].record()
+            o_ref = F.scaled_dot_product_attention(qt, kt, vt, is_causal=True, enable_gqa=True)
+            ev[1].record()
+            torch.cuda.synchronize()
+            if it >= warmup:
+                times.append(ev[0].elapsed_time(ev[1]))
+        t_sdpa = float(np.median(times))
+        T = n // B
+        layer = poem.alloc_layer(q, k, block=B)
+        o_all = _dense_output(poem, q, k, v, layer, hq, T)
+        rp_all, ci_all = poem_synth.random_block_lists(1, T, 1.0, seed=0)
+        counts = np.diff(rp_all)
+        rpd = torch.from_numpy(np.concatenate([[0], np.cumsum(np.tile(counts, hq))]).astype(np.int32)).cuda()
+        cid = torch.from_numpy(np.tile(ci_all, hq).astype(np.int32)).cuda()
+        times = []
+        for it in range(warmup + steps):
+            ev = _events(2)
+            ev[0].record()
+            poem.bsa_fwd(q, k, v, rpd, cid, layer.o, layer.ws_fwd, shape=layer.shape)
+            ev[1].record()
+            torch.cuda.synchronize()
+            if it >= warmup:
+                times.append(ev[0].elapsed_time(ev[1]))
+        poem.poem_check(layer.ws_fwd)
+        t_all = float(np.median(times))
+        diff = (o_all.float() - o_ref[0].permute(1, 0, 2).float()).abs()
+        dfl = dense_flops(n, hq, d)
+        out.append({"config": "dense-context", "n_tokens": n, "sdpa_ms": round(t_sdpa, 4),
+                    "sdpa_tflops": round(dfl / (t_sdpa * 1e-3) / 1e12, 1), "bsa_fwd_all_blocks_ms": round(t_all, 4),
+                    "bsa_fwd_all_blocks_tflops": round(dfl / (t_all * 1e-3) / 1e12, 1),
+                    "max_abs_diff_vs_sdpa": float(diff.max())})
+        del q, k, v, qt, kt, vt, o_ref, o_all, layer
+        torch.cuda.empty_cache()
+    return out
+
+
 EVAL_LAYERS = [
     ("heavy-block-32k", "heavy"),
     ("contrast-32k", "contrast"),
@@ -975,6 +1027,9 @@ def run_report(args):
     if part in (None, "chunked"):
         for rec in _report_chunked(poem, args.steps, args.warmup):
             print(json.dumps(rec), flush=True)
+    if part in (None, "dense"):
+        for rec in _report_dense_context(poem, args.steps, args.warmup):
+            print(json.dumps(rec), flush=True)
     if part in (None, "sweep"):
         for rec in _report_sweep(poem, args.steps, args.warmup):
             print(json.dumps(rec), flush=True)
@@ -1004,7 +1059,8 @@ def main():
     ap.add_argument("--rho", type=float, default=0.5, help="practical: stage-1 shortlist fraction")
     ap.add_argument("--report", action="store_true",
                     help="measure every configuration (one JSON record each) instead of the benchmark line")
-    ap.add_argument("--report-only", choices=["exact", "practical", "evaluation", "chunked", "sweep"], default=None,
+    ap.add_argument("--report-only", choices=["exact", "practical", "evaluation", "chunked", "dense", "sweep"],
+                    default=None,
                     help="with --report: only this part")
     args = ap.parse_args()
     if args.report:
