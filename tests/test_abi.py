@@ -210,3 +210,21 @@ def test_binding_checks_buffer_types_and_sizes(poem):
     with pytest.raises(TypeError):
         poem._need(None, torch.int32, rows + 1, "row_ptr")
     poem._need(None, torch.int32, rows, "order", optional=True)
+
+
+def test_binding_without_the_library_fails_at_import(tmp_path):
+    """No fallback: a copy of the package without libpoem.so refuses to import."""
+    import shutil
+    import subprocess
+    import sys
+
+    src = os.path.join(ROOT, "block_sparse_attention_poem_b200")
+    dst = tmp_path / "block_sparse_attention_poem_b200"
+    dst.mkdir()
+    for name in os.listdir(src):
+        if name.endswith(".py"):
+            shutil.copy(os.path.join(src, name), dst / name)
+    r = subprocess.run([sys.executable, "-c", "import block_sparse_attention_poem_b200"], cwd=tmp_path,
+                       env={**os.environ, "PYTHONPATH": str(tmp_path)}, capture_output=True, text=True, timeout=300)
+    assert r.returncode != 0
+    assert "libpoem.so not built" in r.stderr
