@@ -888,7 +888,7 @@ def _report_chunked(poem, steps, warmup):
     return out
 
 
-def _report_dense_context(poem, steps, warmup):
+def _report_dense_context(poem, steps, warmup, sizes=(32768, 131072)):
     """Context only (not the product path): dense causal GQA attention from the
     framework's own library kernel (torch scaled_dot_product_attention on the
     device) next to bsa_fwd with every causal block listed, on i.i.d. inputs."""
@@ -896,7 +896,7 @@ def _report_dense_context(poem, steps, warmup):
 
     out = []
     hq, hkv, d, B = 32, 8, 128, 128
-    for n in (32768, 131072):
+    for n in sizes:
         x = poem_synth.iid_layer(n, hq, hkv, d, seed=0)
         q, k, v = x["q"].cuda(), x["k"].cuda(), x["v"].cuda()
         qt, kt, vt = q.permute(1, 0, 2).unsqueeze(0), k.permute(1, 0, 2).unsqueeze(0), v.permute(1, 0, 2).unsqueeze(0)
@@ -1028,7 +1028,7 @@ def run_report(args):
         for rec in _report_chunked(poem, args.steps, args.warmup):
             print(json.dumps(rec), flush=True)
     if part in (None, "dense"):
-        for rec in _report_dense_context(poem, args.steps, args.warmup):
+        for rec in _report_dense_context(poem, args.steps, args.warmup, tuple(args.dense_n)):
             print(json.dumps(rec), flush=True)
     if part in (None, "sweep"):
         for rec in _report_sweep(poem, args.steps, args.warmup):
@@ -1059,6 +1059,8 @@ def main():
     ap.add_argument("--rho", type=float, default=0.5, help="practical: stage-1 shortlist fraction")
     ap.add_argument("--report", action="store_true",
                     help="measure every configuration (one JSON record each) instead of the benchmark line")
+    ap.add_argument("--dense-n", type=int, nargs="+", default=[32768, 131072],
+                    help="token counts of the dense-context report (multiples of 128)")
     ap.add_argument("--report-only", choices=["exact", "practical", "evaluation", "chunked", "dense", "sweep"],
                     default=None,
                     help="with --report: only this part")
