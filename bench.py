@@ -946,6 +946,51 @@ EVAL_LAYERS = [
 ]
 
 
+def _report_grouped(poem, steps, warmup):
+    """bsa_fwd against bsa_fwd_grouped (two query heads of a KV group sharing K/V tiles
+    over the union of their lists) on the 128K Llama-shaped layer's exact (tau = 0.05)
+    and practical (gamma = 0.95) lists; the outputs must be bit-identical."""
+    n, hq, hkv, d, B, base, _ = WORKLOADS["llama3.1-8b-layer-128k"]
+    x = poem_synth.heavy_block_layer(n, hq, hkv, d, block=B, rope_base=base, seed=0)
+    T = n // B
+    q, k, v = x["q"].cuda(), x["k"].cuda(), x["v"].cuda()
+    layer = poem.alloc_layer(q, k, block=B, practical=True)
+    o2 = torch.empty_like(layer.o)
+    ws2 = poem.alloc_workspace(256)
+    out = []
+    for sel in ("exact", "practical"):
+        if sel == "exact":
+            poem.prefill_layer(q, k, v, 0.05, layer=layer, block=B)
+        else:
+            poem.prefill_layer_practical(q, k, v, 1.0, 0.95, 0.5, layer=layer, block=B)
+        torch.cuda.synchronize()
+        rp = layer.row_ptr.cpu().numpy()
+        rfl = retained_flops(rp, layer.col_idx[: int(rp[-1])].cpu().numpy(), T, d, B)
+        times = {"bsa_fwd": [], "bsa_fwd_grouped": []}
+        for it in range(warmup + steps):
+            for key in times:  # interleaved, one launch each per iteration
+                ev = _events(2)
+                ev[0].record()
+                if key == "bsa_fwd":
+                    poem.bsa_fwd(q, k, v, layer.row_ptr, layer.col_idx, layer.o, layer.ws_fwd, order=layer.order,
+                                 shape=layer.shape)
+                else:
+                    poem.bsa_fwd_grouped(q, k, v, layer.row_ptr, layer.col_idx, o2, ws2, shape=layer.shape)
+                ev[1].record()
+                torch.cuda.synchronize()
+                if it >= warmup:
+                    times[key].append(ev[0].elapsed_time(ev[1]))
+        poem.poem_check(layer.ws_fwd)
+        poem.poem_check(ws2)
+        ms = {key: float(np.median(val)) for key, val in times.items()}
+        out.append({"config": "grouped-llama3.1-8b-layer-128k", "selector": sel,
+                    "density": round(int(rp[-1]) / (hq * T * (T + 1) // 2), 5),
+                    "ms": {key: round(val, 4) for key, val in ms.items()},
+                    "retained_tflops": {key: round(rfl / (val * 1e-3) / 1e12, 1) for key, val in ms.items()},
+                    "bit_identical": bool(torch.equal(o2.view(torch.int16), layer.o.view(torch.int16)))})
+    return out
+
+
 def _err_vs(o, o_dense):
     diff = o.float() - o_dense.float()
     return {"rel_fro": round(float(diff.norm() / o_dense.float().norm()), 5),
@@ -1027,6 +1072,9 @@ def run_report(args):
     if part in (None, "chunked"):
         for rec in _report_chunked(poem, args.steps, args.warmup):
             print(json.dumps(rec), flush=True)
+    if part in (None, "grouped"):
+        for rec in _report_grouped(poem, args.steps, args.warmup):
+            print(json.dumps(rec), flush=True)
     if part in (None, "dense"):
         for rec in _report_dense_context(poem, args.steps, args.warmup, tuple(args.dense_n)):
             print(json.dumps(rec), flush=True)
@@ -1061,7 +1109,8 @@ def main():
                     help="measure every configuration (one JSON record each) instead of the benchmark line")
     ap.add_argument("--dense-n", type=int, nargs="+", default=[32768, 131072],
                     help="token counts of the dense-context report (multiples of 128)")
-    ap.add_argument("--report-only", choices=["exact", "practical", "evaluation", "chunked", "dense", "sweep"],
+    ap.add_argument("--report-only", choices=["exact", "practical", "evaluation", "chunked", "dense", "grouped",
+                                                   "sweep"],
                     default=None,
                     help="with --report: only this part")
     args = ap.parse_args()

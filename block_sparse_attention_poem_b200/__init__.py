@@ -43,7 +43,7 @@ EXPORTED = (
     "poem_workspace_size", "poem_score", "poem_select", "poem_select_mass_only", "bsa_fwd",
     "poem_check", "poem_set_wait_limit_ns", "poem_status_string", "poem_last_error", "poem_select_noalloc",
     "poem_pooled_workspace_size", "poem_score_pooled", "poem_select_practical", "poem_select_ranked_budget",
-    "poem_select_per_head", "poem_select_practical_per_head",
+    "poem_select_per_head", "poem_select_practical_per_head", "bsa_fwd_grouped",
 )
 
 
@@ -96,6 +96,8 @@ def _load():
     lib.poem_select_practical.restype = st
     lib.bsa_fwd.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.bsa_fwd.restype = st
+    lib.bsa_fwd_grouped.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.bsa_fwd_grouped.restype = st
     lib.poem_check.argtypes = [vp, vp]
     lib.poem_check.restype = st
     lib.poem_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
@@ -352,6 +354,24 @@ def bsa_fwd(q, k, v, row_ptr, col_idx, o, ws, lse=None, order=None, shape: Shape
     _need(ws, torch.uint8, 0, "ws")
     _raise(_lib.bsa_fwd(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(row_ptr), _ptr(col_idx), _ptr(order),
                         _ptr(o), _ptr(lse), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)), "bsa_fwd")
+
+
+def bsa_fwd_grouped(q, k, v, row_ptr, col_idx, o, ws, lse=None, shape: Shape | None = None, stream=None,
+                    **shape_kw):
+    """bsa_fwd's outputs, with two query heads of a KV group sharing K/V tiles."""
+    _check_bf16(q, k, v, o)
+    _check_kv(k, v)
+    if o.shape != q.shape:
+        raise ValueError("o must have q's shape")
+    shape = shape or make_shape(q, k, o=o, **shape_kw)
+    rows, _ = _dims(shape)
+    _need(row_ptr, torch.int32, rows + 1, "row_ptr")
+    _need(col_idx, torch.int32, 0, "col_idx")  # must hold row_ptr[-1] entries (not checked: on the device)
+    _need(lse, torch.float32, shape.n_q_heads * shape.n_tokens, "lse", optional=True)
+    _need(ws, torch.uint8, 0, "ws")
+    _raise(_lib.bsa_fwd_grouped(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(row_ptr), _ptr(col_idx),
+                                _ptr(o), _ptr(lse), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
+           "bsa_fwd_grouped")
 
 
 def poem_check(ws, stream=None):

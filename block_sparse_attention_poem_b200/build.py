@@ -9,7 +9,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libpoem.so")
-SOURCES = ["poem_api.cu", "bsa_fwd.cu", "poem_score.cu", "poem_select.cu", "poem_select_noalloc.cu", "poem_pooled.cu"]
+SOURCES = ["poem_api.cu", "bsa_fwd.cu", "bsa_fwd_grouped.cu", "poem_score.cu", "poem_select.cu", "poem_select_noalloc.cu", "poem_pooled.cu"]
 HEADERS = ["sm100.cuh", "common.cuh"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = [

@@ -153,6 +153,8 @@ struct PoolParams {
 // Launchers (defined in the kernel translation units).
 cudaError_t launch_bsa_fwd(int head_dim, int block, const CUtensorMap& tmQ, const CUtensorMap& tmK,
                            const CUtensorMap& tmV, const FwdParams& p, int n_units, cudaStream_t stream);
+cudaError_t launch_bsa_fwd_grouped(int head_dim, int block, const CUtensorMap& tmQ, const CUtensorMap& tmK,
+                                   const CUtensorMap& tmV, const FwdParams& p, int n_kv_heads, cudaStream_t stream);
 cudaError_t launch_score(int head_dim, int block, const CUtensorMap& tmQs, const CUtensorMap& tmK,
                          const CUtensorMap& tmV, const ScoreParams& p, cudaStream_t stream);
 cudaError_t launch_select(const SelectParams& p, cudaStream_t stream);

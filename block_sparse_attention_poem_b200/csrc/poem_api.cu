@@ -372,44 +372,69 @@ poem_status poem_select_practical_per_head(const poem_shape* shape, const float*
                        stream, &pa);
 }
 
-poem_status bsa_fwd(const poem_shape* shape, const poem_bf16* q, const poem_bf16* k, const poem_bf16* v,
-                    const int32_t* row_ptr, const int32_t* col_idx, const int32_t* order, poem_bf16* o, float* lse,
-                    void* ws, size_t ws_bytes, void* stream) {
-  Layout L;
-  poem_status st = check_shape(shape, &L);
+// Checks, tensor maps and parameter block shared by bsa_fwd and bsa_fwd_grouped.
+static poem_status fwd_setup(const poem_shape* shape, const void* q, const void* k, const void* v,
+                             const int32_t* row_ptr, const int32_t* col_idx, const int32_t* order, void* o,
+                             float* lse, void* ws, size_t ws_bytes, Layout* L, CUtensorMap* tmQ, CUtensorMap* tmK,
+                             CUtensorMap* tmV, poem::FwdParams* p) {
+  poem_status st = check_shape(shape, L);
   if (st != POEM_OK) return st;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(row_ptr) || !aligned16(o) || !aligned16(ws) ||
       (col_idx && !aligned16(col_idx)) || (order && !aligned16(order)) || (lse && !aligned16(lse)))
     return arg_fail(POEM_ERR_INVALID_ARG, "pointers must be non-NULL and 16-byte aligned");
-  if (ws_bytes < fwd_ws_bytes(shape, L.T)) return arg_fail(POEM_ERR_WORKSPACE, "fwd workspace too small");
-  CUtensorMap tmQ, tmK, tmV;
-  if ((st = make_map_3d(&tmQ, q, shape->head_dim, shape->n_q_heads, shape->n_tokens, shape->q_stride_head,
+  if (ws_bytes < fwd_ws_bytes(shape, L->T)) return arg_fail(POEM_ERR_WORKSPACE, "fwd workspace too small");
+  if ((st = make_map_3d(tmQ, q, shape->head_dim, shape->n_q_heads, shape->n_tokens, shape->q_stride_head,
                         shape->q_stride_tok, 128)) != POEM_OK)
     return st;
-  if ((st = make_map_3d(&tmK, k, shape->head_dim, shape->n_kv_heads, L.n_kv, shape->kv_stride_head,
+  if ((st = make_map_3d(tmK, k, shape->head_dim, shape->n_kv_heads, L->n_kv, shape->kv_stride_head,
                         shape->kv_stride_tok, shape->block)) != POEM_OK)
     return st;
-  if ((st = make_map_3d(&tmV, v, shape->head_dim, shape->n_kv_heads, L.n_kv, shape->kv_stride_head,
+  if ((st = make_map_3d(tmV, v, shape->head_dim, shape->n_kv_heads, L->n_kv, shape->kv_stride_head,
                         shape->kv_stride_tok, shape->block)) != POEM_OK)
     return st;
-  poem::FwdParams p{};
-  p.row_ptr = row_ptr;
-  p.col_idx = col_idx;
-  p.order = order;
-  p.o = reinterpret_cast<__nv_bfloat16*>(o);
-  p.lse = lse;
-  p.o_stride_tok = shape->o_stride_tok;
-  p.o_stride_head = shape->o_stride_head;
-  p.n_tokens = shape->n_tokens;
-  p.n_q_heads = shape->n_q_heads;
-  p.n_tiles = L.T;
-  p.q_tile0 = L.t0;
-  p.group = L.G;
-  p.scale_log2 = L.scale * poem::kLog2e;
-  p.err = dev_err(ws);
+  *p = poem::FwdParams{};
+  p->row_ptr = row_ptr;
+  p->col_idx = col_idx;
+  p->order = order;
+  p->o = reinterpret_cast<__nv_bfloat16*>(o);
+  p->lse = lse;
+  p->o_stride_tok = shape->o_stride_tok;
+  p->o_stride_head = shape->o_stride_head;
+  p->n_tokens = shape->n_tokens;
+  p->n_q_heads = shape->n_q_heads;
+  p->n_tiles = L->T;
+  p->q_tile0 = L->t0;
+  p->group = L->G;
+  p->scale_log2 = L->scale * poem::kLog2e;
+  p->err = dev_err(ws);
+  return POEM_OK;
+}
+
+poem_status bsa_fwd(const poem_shape* shape, const poem_bf16* q, const poem_bf16* k, const poem_bf16* v,
+                    const int32_t* row_ptr, const int32_t* col_idx, const int32_t* order, poem_bf16* o, float* lse,
+                    void* ws, size_t ws_bytes, void* stream) {
+  Layout L;
+  CUtensorMap tmQ, tmK, tmV;
+  poem::FwdParams p;
+  poem_status st = fwd_setup(shape, q, k, v, row_ptr, col_idx, order, o, lse, ws, ws_bytes, &L, &tmQ, &tmK, &tmV, &p);
+  if (st != POEM_OK) return st;
   cudaError_t e = poem::launch_bsa_fwd(shape->head_dim, shape->block, tmQ, tmK, tmV, p, shape->n_q_heads * L.T,
                                        (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "bsa_fwd launch");
+  return POEM_OK;
+}
+
+poem_status bsa_fwd_grouped(const poem_shape* shape, const poem_bf16* q, const poem_bf16* k, const poem_bf16* v,
+                            const int32_t* row_ptr, const int32_t* col_idx, poem_bf16* o, float* lse, void* ws,
+                            size_t ws_bytes, void* stream) {
+  Layout L;
+  CUtensorMap tmQ, tmK, tmV;
+  poem::FwdParams p;
+  poem_status st = fwd_setup(shape, q, k, v, row_ptr, col_idx, nullptr, o, lse, ws, ws_bytes, &L, &tmQ, &tmK, &tmV, &p);
+  if (st != POEM_OK) return st;
+  cudaError_t e = poem::launch_bsa_fwd_grouped(shape->head_dim, shape->block, tmQ, tmK, tmV, p, shape->n_kv_heads,
+                                               (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "bsa_fwd_grouped launch");
   return POEM_OK;
 }
 

@@ -16,6 +16,7 @@
  *   poem_select  mandatory blocks + blocks in descending I_b until the bound
  *                above is <= tau; CSR block list per (head, tile)
  *   bsa_fwd      causal GQA block-sparse attention over the listed blocks
+ *   bsa_fwd_grouped  the same, with two query heads of a KV group sharing K/V tiles
  *
  * Conventions for every entry point
  *   - All pointers are device pointers unless stated, 16-byte aligned.  The
@@ -279,6 +280,20 @@ poem_status poem_select_practical_per_head(const poem_shape* shape, const float*
 poem_status bsa_fwd(const poem_shape* shape, const poem_bf16* q, const poem_bf16* k, const poem_bf16* v,
                     const int32_t* row_ptr, const int32_t* col_idx, const int32_t* order, poem_bf16* o,
                     float* lse, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * bsa_fwd_grouped -- the same computation and outputs as bsa_fwd (every row's
+ * renormalised output over its own list, Section 4.1), scheduled so that two
+ * query heads of one KV group share K/V tiles: one CTA takes query heads
+ * 2p, 2p + 1 of a group at one query tile and walks the union of their two
+ * lists, loading each block's K and V once for both heads; each head runs its
+ * attention only on the blocks of its own list.  Work order: KV head major,
+ * last tile first (no order argument).  Arguments, list rules, errors and
+ * workspace as bsa_fwd.
+ */
+poem_status bsa_fwd_grouped(const poem_shape* shape, const poem_bf16* q, const poem_bf16* k, const poem_bf16* v,
+                            const int32_t* row_ptr, const int32_t* col_idx, poem_bf16* o, float* lse, void* ws,
+                            size_t ws_bytes, void* stream);
 
 /*
  * Synchronise `stream`, read and clear the error word at the start of `ws`
