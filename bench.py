@@ -946,11 +946,12 @@ EVAL_LAYERS = [
 ]
 
 
-def _report_grouped(poem, steps, warmup):
+def _report_grouped(poem, steps, warmup, n_tokens=131072):
     """bsa_fwd against bsa_fwd_grouped (two query heads of a KV group sharing K/V tiles
     over the union of their lists) on the 128K Llama-shaped layer's exact (tau = 0.05)
     and practical (gamma = 0.95) lists; the outputs must be bit-identical."""
-    n, hq, hkv, d, B, base, _ = WORKLOADS["llama3.1-8b-layer-128k"]
+    _, hq, hkv, d, B, base, _ = WORKLOADS["llama3.1-8b-layer-128k"]
+    n = n_tokens
     x = poem_synth.heavy_block_layer(n, hq, hkv, d, block=B, rope_base=base, seed=0)
     T = n // B
     q, k, v = x["q"].cuda(), x["k"].cuda(), x["v"].cuda()
@@ -983,7 +984,7 @@ def _report_grouped(poem, steps, warmup):
         poem.poem_check(layer.ws_fwd)
         poem.poem_check(ws2)
         ms = {key: float(np.median(val)) for key, val in times.items()}
-        out.append({"config": "grouped-llama3.1-8b-layer-128k", "selector": sel,
+        out.append({"config": f"grouped-llama3.1-8b-layer-{n // 1024}k", "selector": sel,
                     "density": round(int(rp[-1]) / (hq * T * (T + 1) // 2), 5),
                     "ms": {key: round(val, 4) for key, val in ms.items()},
                     "retained_tflops": {key: round(rfl / (val * 1e-3) / 1e12, 1) for key, val in ms.items()},
@@ -1073,7 +1074,7 @@ def run_report(args):
         for rec in _report_chunked(poem, args.steps, args.warmup):
             print(json.dumps(rec), flush=True)
     if part in (None, "grouped"):
-        for rec in _report_grouped(poem, args.steps, args.warmup):
+        for rec in _report_grouped(poem, args.steps, args.warmup, args.grouped_n):
             print(json.dumps(rec), flush=True)
     if part in (None, "dense"):
         for rec in _report_dense_context(poem, args.steps, args.warmup, tuple(args.dense_n)):
@@ -1107,6 +1108,8 @@ def main():
     ap.add_argument("--rho", type=float, default=0.5, help="practical: stage-1 shortlist fraction")
     ap.add_argument("--report", action="store_true",
                     help="measure every configuration (one JSON record each) instead of the benchmark line")
+    ap.add_argument("--grouped-n", type=int, default=131072,
+                    help="token count of the grouped-attention report (a multiple of 128)")
     ap.add_argument("--dense-n", type=int, nargs="+", default=[32768, 131072],
                     help="token counts of the dense-context report (multiples of 128)")
     ap.add_argument("--report-only", choices=["exact", "practical", "evaluation", "chunked", "dense", "grouped",
