@@ -10,7 +10,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libpoem.so")
 SOURCES = ["poem_api.cu", "bsa_fwd.cu", "bsa_fwd_grouped.cu", "poem_score.cu", "poem_select.cu", "poem_select_noalloc.cu", "poem_pooled.cu"]
-HEADERS = ["sm100.cuh", "common.cuh"]
+HEADERS = ["sm100.cuh", "common.cuh", "fwd_common.cuh"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
