@@ -58,3 +58,28 @@ def test_expired_waits_report_timeout_and_context_recovers(poem):
     poem.poem_score(q, k, v, layer.I_hat, layer.m_hat, layer.ws_score, shape=layer.shape)
     assert poem.poem_check_status(layer.ws_score) == 0
     assert torch.isfinite(layer.I_hat).all()
+
+
+def test_grouped_expired_waits_report_timeout_and_context_recovers(poem):
+    """The same for bsa_fwd_grouped (one CTA per SM, two heads over a shared K/V ring)."""
+    n, hq, hkv, d, B = 2048, 8, 2, 128, 128
+    T = n // B
+    x = poem_synth.iid_layer(n, hq, hkv, d, seed=6)
+    q, k, v = x["q"].cuda(), x["k"].cuda(), x["v"].cuda()
+    rp, ci = poem_synth.random_block_lists(hq, T, 0.5, seed=6)
+    rpd, cid = torch.from_numpy(rp).cuda(), torch.from_numpy(ci).cuda()
+    ws = poem.alloc_workspace(256)
+    o = torch.empty_like(q)
+    try:
+        poem.poem_set_wait_limit_ns(0)
+        poem.bsa_fwd_grouped(q, k, v, rpd, cid, o, ws, block=B)
+        assert poem.STATUS[poem.poem_check_status(ws)] == "POEM_ERR_TIMEOUT"
+    finally:
+        poem.poem_set_wait_limit_ns(DEFAULT_LIMIT_NS)
+    torch.cuda.synchronize()
+    poem.bsa_fwd_grouped(q, k, v, rpd, cid, o, ws, block=B)
+    assert poem.poem_check_status(ws) == 0
+    o_ref = torch.empty_like(q)
+    poem.bsa_fwd(q, k, v, rpd, cid, o_ref, ws, block=B)
+    assert poem.poem_check_status(ws) == 0
+    assert torch.equal(o.view(torch.int16), o_ref.view(torch.int16))
