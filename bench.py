@@ -389,7 +389,8 @@ def run_ours(args):
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = (cpu_baseline_practical(x, n, hq, hkv, d, B, args.w, args.gamma, args.rho, args.cpu_budget_s)
-               if practical else cpu_baseline(x, n, hq, hkv, d, B, tau, args.cpu_budget_s))
+               if practical else cpu_baseline(x, n, hq, hkv, d, B, tau, args.cpu_budget_s,
+                                              gpu_rows=gpu_rows_fn(layer, T, B)))
     sel_cfg = ({"selector": "practical", "w": args.w, "gamma": args.gamma, "rho": args.rho} if practical
                else {"selector": "exact", "tau": tau})
     names = (("poem_score_pooled", "poem_select_practical") if practical else ("poem_score", "poem_select"))
@@ -433,6 +434,8 @@ def run_ours(args):
         "gpu_launches": launches_per_step * args.steps,
         "cpu_baseline": cpu,
     }
+    if cpu and "parity" in cpu:
+        line["oracle_parity"] = cpu.pop("parity")
     line.update(extra)
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -470,10 +473,28 @@ def quality_report(poem, q, k, v, layer, tau, n, hq, T, B, dev):
     return {"err_vs_dense": {"poem": err(layer.o), "mass_only_same_budget": err(o_mass)}}
 
 
-def cpu_baseline(x, n, hq, hkv, d, B, tau, budget_s):
+def gpu_rows_fn(layer, T, B):
+    """Host copies of one (head, tile) row of a whole-prefill layer: Î and m̂ of the
+    row, its block list and its output rows."""
+    def rows(h, i):
+        off = h * T * (T + 1) // 2 + i * (i + 1) // 2
+        r = h * T + i
+        a, b = (int(t) for t in layer.row_ptr[r:r + 2].cpu())
+        return (layer.I_hat[off:off + i + 1].cpu().numpy().astype(np.float64),
+                layer.m_hat[off:off + i + 1].cpu().numpy().astype(np.float64),
+                layer.col_idx[a:b].cpu().numpy(),
+                layer.o[i * B:(i + 1) * B, h].float().cpu().numpy())
+    return rows
+
+
+def cpu_baseline(x, n, hq, hkv, d, B, tau, budget_s, gpu_rows=None):
     """Oracle (fp64, host cores) on a bounded sample of (head, tile) units, scaled to
     a whole layer by work per unit (score ~ i+1 blocks, masked attention ~ kept
-    blocks; selection is negligible)."""
+    blocks; selection is negligible).  With `gpu_rows` the same units also cross-check
+    the CUDA path (outside the timed work): the worst Î or m̂ error as a fraction of its
+    tolerance (Î: 1e-3 relative + 1e-5 m_b R; m̂: 1e-3 relative + 1e-9), how many lists
+    equal the oracle's,
+    and the largest output error against the oracle's attention over the GPU's list."""
     import oracle
 
     oracle.build()
@@ -485,6 +506,14 @@ def cpu_baseline(x, n, hq, hkv, d, B, tau, budget_s):
     per_unit = []
     t_total = 0.0
     cand_tiles = [max(0, int(T * f) - 1) for f in (1 / 64, 1 / 16, 1 / 8, 1 / 4)]
+    R = float(x["v"].float().norm(dim=-1).max())
+    par = {"units": 0, "score_tol_ratio_max": 0.0, "lists_equal": 0, "o_max_abs": 0.0}
+
+    def one_row_list(r, lst):
+        rp = np.zeros(hq * T + 1, dtype=np.int32)
+        rp[r + 1:] = len(lst)
+        return rp, np.asarray(lst, dtype=np.int32)
+
     h = 0
     for i in cand_tiles:
         if t_total > budget_s:
@@ -493,26 +522,34 @@ def cpu_baseline(x, n, hq, hkv, d, B, tau, budget_s):
         Ih, mh = prob.score_units([(h, i)])
         off = oracle.tri_offset(T, h, i)
         keep, _ = oracle.select_row(i, Ih[off:off + i + 1], mh[off:off + i + 1], tau)
-        rp = np.zeros(hq * T + 1, dtype=np.int32)
         r = h * T + i
-        rp[r + 1:] = len(keep)
-        ci = np.zeros(hq * T, dtype=np.int32)
-        ci[: len(keep)] = keep
-        rp2 = rp.copy()
-        rp2[: r + 1] = 0
-        prob.masked_units([(h, i)], rp2, np.asarray(keep, dtype=np.int32))
+        prob.masked_units([(h, i)], *one_row_list(r, keep))
         dt = time.perf_counter() - t0
         t_total += dt
         units.append((h, i))
         per_unit.append(dt / (i + 1))
+        if gpu_rows is not None:
+            gI, gm, glist, go = gpu_rows(h, i)
+            rI, rm = Ih[off:off + i + 1], mh[off:off + i + 1]
+            tol_I = 1e-3 * rI + 1e-5 * rm * R + 1e-30
+            tol_m = 1e-3 * rm + 1e-9
+            par["units"] += 1
+            par["score_tol_ratio_max"] = max(par["score_tol_ratio_max"], float(np.max(np.abs(gI - rI) / tol_I)),
+                                             float(np.max(np.abs(gm - rm) / tol_m)))
+            par["lists_equal"] += int(np.array_equal(glist, np.asarray(keep)))
+            Og, _ = prob.masked_units([(h, i)], *one_row_list(r, glist))
+            par["o_max_abs"] = max(par["o_max_abs"], float(np.max(np.abs(go - np.asarray(Og[0])[:B]))))
         h = (h + 1) % hq
     rate = float(np.mean(per_unit))  # seconds per visible block of a unit
     total_blocks = hq * T * (T + 1) / 2
     est_ms = rate * total_blocks * 1e3
-    return {"value": round(est_ms, 1), "unit": "ms/layer", "cores": oracle.num_threads(), "kind": "oracle",
-            "sample": f"{len(units)} (head, tile) units at tiles {[u[1] for u in units]} (score + select + masked "
-                      f"attention), {t_total:.1f} s, scaled by visible blocks per unit to the whole layer",
-            "extrapolated": True}
+    out = {"value": round(est_ms, 1), "unit": "ms/layer", "cores": oracle.num_threads(), "kind": "oracle",
+           "sample": f"{len(units)} (head, tile) units at tiles {[u[1] for u in units]} (score + select + masked "
+                     f"attention), {t_total:.1f} s, scaled by visible blocks per unit to the whole layer",
+           "extrapolated": True}
+    if gpu_rows is not None:
+        out["parity"] = par
+    return out
 
 
 def cpu_baseline_practical(x, n, hq, hkv, d, B, w, gamma, rho, budget_s):
@@ -657,7 +694,8 @@ def _report_layer(poem, name, wl, tau, steps, warmup, mass_only, cpu_budget_s):
     if not mass_only:
         rec["err_vs_dense"].pop("mass_only_same_budget", None)
     if cpu_budget_s > 0:
-        cb = cpu_baseline(x, n, hq, hkv, d, B, tau, cpu_budget_s)
+        cb = cpu_baseline(x, n, hq, hkv, d, B, tau, cpu_budget_s, gpu_rows=gpu_rows_fn(layer, T, B))
+        rec["oracle_parity"] = cb.pop("parity")
         rec["oracle_ms_per_layer"] = cb["value"]
         rec["oracle_cores"] = cb["cores"]
         rec["oracle_note"] = cb["sample"]
@@ -676,11 +714,15 @@ def _report_sweep(poem, steps, warmup):
         T = n // B
         o = torch.empty_like(q)
         ws = poem.alloc_workspace(256)
+        # up to 16K tokens the working set is close to L2's size: write 256 MiB between launches
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda") if n <= 16384 else None
         for dens in SWEEP_DENSITY:
             rp, ci = poem_synth.random_block_lists(hq, T, dens, seed=0)
             rpd, cid = torch.from_numpy(rp).cuda(), torch.from_numpy(ci).cuda()
             times = []
             for it in range(warmup + steps):
+                if flush is not None:
+                    flush.zero_()  # evict this layer's inputs from L2 before the timed launch
                 ev = _events(2)
                 ev[0].record()
                 poem.bsa_fwd(q, k, v, rpd, cid, o, ws, block=B)
@@ -694,10 +736,12 @@ def _report_sweep(poem, steps, warmup):
             tf = rfl / (t * 1e-3) / 1e12
             out.append({"config": "bsa_fwd-sweep", "n_tokens": n, "density_target": dens,
                         "density": round(int(rp[-1]) / (hq * T * (T + 1) / 2), 5), "ms": round(t, 4),
+                        "ms_min": round(float(np.min(times)), 4),
+                        "l2": "256 MiB written between launches" if flush is not None else "inputs larger than L2",
                         "retained_tflops": round(tf, 2), "frac_burst": round(tf / peaks["bf16_tflops"], 4),
                         "frac_sustained": round(tf / peaks["bf16_tflops_sustained"], 4),
                         "dense_equiv_tflops": round(dense_flops(n, hq, d) / (t * 1e-3) / 1e12, 2)})
-        del q, k, v, o
+        del q, k, v, o, flush
         torch.cuda.empty_cache()
     return out
 

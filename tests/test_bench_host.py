@@ -65,3 +65,40 @@ def test_all_blocks_listed_equals_dense():
     row_ptr = np.concatenate([[0], np.cumsum([len(x) for x in rows])]).astype(np.int32)
     col_idx = np.array([b for x in rows for b in x], dtype=np.int32)
     assert bench.retained_flops(row_ptr, col_idx, n_tiles, d, B) == bench.dense_flops(n_tiles * B, hq, d)
+
+
+def test_sampled_oracle_cross_check_scores_a_planted_error():
+    """The benchmark's cross-check on sampled units: rows taken from the oracle itself
+    give zero errors and equal lists; a 0.3% error planted in one score row shows up
+    as ~3 tolerances, and a shifted output row as its shift."""
+    import oracle
+    import poem_synth
+
+    oracle.build()
+    n, hq, hkv, d, B, tau = 2048, 2, 1, 64, 128, 0.05
+    T = n // B
+    x = poem_synth.heavy_block_layer(n, hq, hkv, d, block=B, seed=3)
+    prob = oracle.Problem(q=poem_synth.bf16_bits(x["q"]), k=poem_synth.bf16_bits(x["k"]),
+                          v=poem_synth.bf16_bits(x["v"]), block=B, n_sample=16)
+
+    def rows_from_oracle(h, i, plant=False):
+        Ih, mh = prob.score_units([(h, i)])
+        off = oracle.tri_offset(T, h, i)
+        I, m = Ih[off:off + i + 1].copy(), mh[off:off + i + 1].copy()
+        keep, _ = oracle.select_row(i, I, m, tau)
+        rp = np.zeros(hq * T + 1, dtype=np.int32)
+        rp[h * T + i + 1:] = len(keep)
+        O, _ = prob.masked_units([(h, i)], rp, np.asarray(keep, dtype=np.int32))
+        o = np.asarray(O[0])[:B].copy()
+        if plant:
+            I[np.argmax(I)] *= 1.003
+            o[0, 0] += 0.25
+        return I, m, np.asarray(keep, dtype=np.int32), o
+
+    clean = bench.cpu_baseline(x, n, hq, hkv, d, B, tau, 1e9, gpu_rows=rows_from_oracle)["parity"]
+    assert clean["units"] >= 2 and clean["lists_equal"] == clean["units"]
+    assert clean["score_tol_ratio_max"] == 0.0 and clean["o_max_abs"] == 0.0
+    bad = bench.cpu_baseline(x, n, hq, hkv, d, B, tau, 1e9,
+                             gpu_rows=lambda h, i: rows_from_oracle(h, i, plant=True))["parity"]
+    assert 2.0 < bad["score_tol_ratio_max"] < 3.1
+    assert abs(bad["o_max_abs"] - 0.25) < 1e-9
