@@ -23,7 +23,7 @@
 //              first O_x += P_x V_x for x's previous block (if one is pending), then,
 //              if b is in x's list, S_x = Q_x K_b^T.  A head's P V therefore waits at
 //              most one union step, so each V tile is released one step after its
-//              block and the ring never holds more than two blocks' tiles; a K tile is
+//              block and the ring never needs more than two blocks' tiles; a K tile is
 //              released after its last S, a V tile after its last P V.
 // TMEM: head x has S/P at [256x, 256x + BN) and O at [256x + 128, 256x + 128 + D).
 #include <climits>
@@ -292,7 +292,7 @@ __global__ void __launch_bounds__(kThreadsGrouped, 1)
     }
   } else {
     // ============================ softmax warps ============================
-    const int rx = warp >> 2;                // 0: row A, 1: row B
+    const int rx = warp >> 2;                // 0: head A, 1: head B
     int hk_unused = 0;
     const PairRow R = pair_row(p, unit, rx, &hk_unused, false);
     const int r = tid & 127;                 // query row within the tile (TMEM lane)
