@@ -199,9 +199,15 @@ def test_select_bit_exact_on_identical_scores(poem, T, hq, hkv, seed):
             w = rng.random(i + 1) ** 4
             mh[off:off + i + 1] = (w / w.sum() * 1.3).astype(np.float32)
     shape = _fake_shape(poem, hq, hkv, T)
+    prev_rows = None
     for tau in (0.0, 0.002, 0.02, 0.1, 1e6):  # 1e6: only the mandatory blocks survive
         rp, ci, order, status = _gpu_select(poem, shape, Ih, mh, tau, hq * T)
         assert status == 0
+        # nested supports: a larger tau keeps a subset of every row (the cut is monotone in tau)
+        rows = csr_rows(rp, ci[:rp[-1]])
+        if prev_rows is not None:
+            assert all(set(a) <= set(b) for a, b in zip(rows, prev_rows))
+        prev_rows = rows
         rp_ref, ci_ref, _ = oracle.select_all(hq, T, Ih.astype(np.float64), mh.astype(np.float64), tau)
         assert np.array_equal(rp, rp_ref)
         assert np.array_equal(ci[:rp[-1]], ci_ref)
@@ -213,6 +219,66 @@ def test_select_bit_exact_on_identical_scores(poem, T, hq, hkv, seed):
             assert sorted(seg.tolist()) == list(range(g * G * T, (g + 1) * G * T))
             key = [(-lens[r], r) for r in seg]
             assert key == sorted(key)
+
+
+def _tau_cutting_between(I, m, i, a, b):
+    """A float32 tau whose stopping rule keeps candidate a and drops b (b right after
+    a in the (I desc, id asc) order) in row i, or None when no such tau exists."""
+    cand = sorted(range(1, max(i - 1, 1)), key=lambda c: (-I[c], c))
+    if a not in cand or b not in cand or cand.index(b) != cand.index(a) + 1:
+        return None
+    k = cand.index(a) + 1  # kept candidates: through a
+
+    def thr(kk):  # smallest tau that lets the suffix after kk be dropped
+        D = cand[kk:]
+        sI, sm = float(sum(I[c] for c in D)), float(sum(m[c] for c in D))
+        return sI / (1.0 - sm) if sm < 1.0 else np.inf
+
+    lo, hi = thr(k), thr(k - 1)
+    if not (np.isfinite(hi) and lo < hi):
+        return None
+    tau = float(np.float32(0.5 * (lo + hi)))
+    keep, _ = oracle.select_row(i, I[:i + 1], m[:i + 1], tau)
+    return tau if (a in keep.tolist() and b not in keep.tolist()) else None
+
+
+def test_ties_forced_by_duplicated_blocks(poem):
+    """Key blocks with identical K and V give bit-identical scores through the whole
+    score pass; with tau chosen so that a row's cut falls between the two copies, the
+    selector keeps the smaller id and drops the larger (the "Block ordering" tie-break)."""
+    n, hq, hkv, d, B = 2048, 2, 1, 128, 128
+    T = n // B
+    x = poem_synth.iid_layer(n, hq, hkv, d, seed=31)
+    pairs = [(2, 10), (3, 5), (7, 9)]
+    for a, b in pairs:
+        x["k"][b * B:(b + 1) * B] = x["k"][a * B:(a + 1) * B]
+        x["v"][b * B:(b + 1) * B] = x["v"][a * B:(a + 1) * B]
+    q, k, v = to_dev(x)
+    layer = poem.prefill_layer(q, k, v, 0.05, block=B)
+    for ws in (layer.ws_score, layer.ws_select, layer.ws_fwd):
+        poem.poem_check(ws)
+    Ig = layer.I_hat.cpu().numpy()
+    mg = layer.m_hat.cpu().numpy()
+    shape = _fake_shape(poem, hq, hkv, T)
+    decisive = 0
+    for h in range(hq):
+        for i in range(T):
+            off = oracle.tri_offset(T, h, i)
+            I = Ig[off:off + i + 1].astype(np.float64)
+            m = mg[off:off + i + 1].astype(np.float64)
+            for a, b in pairs:
+                if b >= i - 1:  # b must be a candidate (not mandatory) of tile i
+                    continue
+                assert Ig[off + a] == Ig[off + b] and mg[off + a] == mg[off + b], (h, i, a, b)
+                tau = _tau_cutting_between(I, m, i, a, b)
+                if tau is None:
+                    continue
+                rp, ci, _, st = _gpu_select(poem, shape, Ig, mg, tau, hq * T, want_order=False)
+                assert st == 0
+                row = csr_rows(rp, ci[:rp[-1]])[h * T + i]
+                assert a in row and b not in row, (h, i, a, b, tau)
+                decisive += 1
+    assert decisive > 0
 
 
 def test_select_mass_only_matches_oracle(poem):
