@@ -3,7 +3,6 @@ is bounded.  With the limit set to zero the waits run out, the kernels record
 POEM_ERR_TIMEOUT in the workspace error word, drain their in-flight copies and
 MMAs, release tensor memory and return; poem_check reports the status and the
 context stays usable (the next call with the normal limit is correct)."""
-import numpy as np
 import pytest
 import torch
 
