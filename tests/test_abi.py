@@ -95,6 +95,20 @@ def test_null_and_misaligned_pointers_rejected(poem):
     assert "16-byte" in poem.poem_last_error() or "n_sample" in poem.poem_last_error()
 
 
+def test_grouped_forward_validates_like_bsa_fwd(poem):
+    """bsa_fwd_grouped shares bsa_fwd's host checks: null or misaligned pointers,
+    a too-small workspace and unsupported shapes fail before any launch."""
+    sh = _shape(poem)
+    ok = ctypes.c_void_p(1 << 20)
+    mis = ctypes.c_void_p((1 << 20) + 8)
+    f = poem._lib.bsa_fwd_grouped
+    assert f(ctypes.byref(sh), None, ok, ok, ok, ok, ok, None, ok, 4096, None) == 1
+    assert f(ctypes.byref(sh), ok, mis, ok, ok, ok, ok, None, ok, 4096, None) == 1
+    assert f(ctypes.byref(sh), ok, ok, ok, ok, ok, ok, ctypes.c_void_p((1 << 20) + 4), ok, 4096, None) == 1  # lse
+    assert f(ctypes.byref(sh), ok, ok, ok, ok, ok, ok, None, ok, 8, None) == 6
+    assert f(ctypes.byref(_shape(poem, head_dim=96)), ok, ok, ok, ok, ok, ok, None, ok, 4096, None) == 2
+
+
 @pytest.mark.parametrize("tau", [-0.1, float("nan"), float("inf")])
 def test_select_rejects_bad_tau(poem, tau):
     sh = _shape(poem)
