@@ -180,6 +180,9 @@ void oracle_block_stats(const oracle_shape* s, const void* q, const void* k, con
 }
 
 /* ---- public: aggregated block scores per (head, tile) ----------------------- */
+/* Eq. (4) scores of "Attention deletion error" Sec. 4.1, taken on 16 strided sampled
+ * queries per tile and max-aggregated (the sampling and aggregation the note leaves
+ * open, fixed in the file header). */
 
 /* Offset of row (h, i) in the packed lower-triangular score arrays. */
 static size_t tri_offset(int n_tiles, int h, int i) {
@@ -221,6 +224,9 @@ void oracle_score_units(const oracle_shape* s, const void* q, const void* k, con
 }
 
 /* ---- public: selection ------------------------------------------------------ */
+/* The Eq. (4) triangle bound of "Attention deletion error" Sec. 4.1 turned into a
+ * stopping rule over the discarded candidates; ties and ascending order as in the
+ * "Block-Filtered Long-Context Attention" page, Appendix "Block ordering". */
 
 /* Ranking: larger score first, equal scores by smaller block id. */
 typedef struct { double key; int id; } ranked;
@@ -288,8 +294,9 @@ int oracle_select_row(int i, const double* Ihat, const double* mhat, double tau,
 }
 
 /*
- * Mass-only baseline: keep the mandatory blocks and the k_free candidates of
- * largest mhat (equal masses by smaller id).  Returns the list length.
+ * Mass-only baseline (the comparison at a matched block budget in the last section
+ * of "Attention deletion error"): keep the mandatory blocks and the k_free
+ * candidates of largest mhat (equal masses by smaller id).  Returns the list length.
  */
 int oracle_select_mass_only_row(int i, const double* mhat, int k_free, int* keep_out) {
     unsigned char* keep = (unsigned char*)calloc((size_t)i + 1, 1);
@@ -328,8 +335,8 @@ void oracle_select_rows(int n_tiles, int n_rows, const int* row_h, const int* ro
 
 /*
  * Softmax attention of query row t of head h restricted to the keys u <= t in
- * the listed blocks.  Writes o[d] and returns the log-sum-exp (-inf, o = 0,
- * when no key is visible).
+ * the listed blocks (o~ of "Attention deletion error" Sec. 4.1).  Writes o[d] and
+ * returns the log-sum-exp (-inf, o = 0, when no key is visible).
  */
 double oracle_masked_row(const oracle_shape* s, const void* q, const void* k, const void* v,
                          int h, int t, const int* blocks, int n_blocks, double* o) {
@@ -344,7 +351,8 @@ double oracle_masked_row(const oracle_shape* s, const void* q, const void* k, co
 }
 
 /*
- * Masked attention for every query row of the listed units.  Unit u covers
+ * Masked attention for every query row of the listed units: the renormalised
+ * output o~ of "Attention deletion error" Sec. 4.1 over each row's kept blocks.  Unit u covers
  * tile i = unit_i[u] of head h = unit_h[u]; its block list is
  * col_idx[row_ptr[r] .. row_ptr[r+1]) with r = h * n_tiles + i.  Output rows
  * go to O[(u*B + j) * d + c] and lse[u*B + j], j = 0..B-1.
@@ -366,7 +374,8 @@ void oracle_masked_units(const oracle_shape* s, const void* q, const void* k, co
     }
 }
 
-/* Dense attention for every row of the listed units (same output layout). */
+/* Dense attention (o of "Attention deletion error" Sec. 4.1) for every row of the
+ * listed units (same output layout). */
 void oracle_dense_units(const oracle_shape* s, const void* q, const void* k, const void* v,
                         int n_units, const int* unit_h, const int* unit_i, double* O, double* lse) {
     const int B = s->block, d = s->head_dim;
