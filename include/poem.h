@@ -188,16 +188,24 @@ poem_status poem_select_ranked_budget(const poem_shape* shape, const float* scor
  * all device memory up front and must not let a library grow its footprint while
  * it serves, or a plug-in that is only handed pointers by its host.  This entry
  * point takes the same inputs and outputs as poem_select but no workspace: its
- * scratch lives in a fixed 8 MiB array inside the library's device image, which
- * every GPU that loads the library holds until the process exits.  It calls no
- * allocator of any kind.
+ * scratch lives in a fixed 8 MiB array inside the library's device image.  It
+ * calls no allocator of any kind.
+ *   - When the 8 MiB is committed: CUDA loads the array's device module on a
+ *     device lazily, at the first poem_select_noalloc call made with that device
+ *     current; from then on the device holds the 8 MiB until the process exits.
+ *     A caller that reserves device memory up front makes one call (any valid
+ *     shape) before its reservation, so that this first call cannot run out of
+ *     memory.
  *   - Shapes whose selection scratch (poem_workspace_size's select_bytes) exceeds
- *     8 MiB are rejected with POEM_ERR_WORKSPACE and a message in poem_last_error
- *     (e.g. 32 heads x 256 tiles fits; 32 heads x 1024 tiles does not).
+ *     8 MiB are rejected with POEM_ERR_WORKSPACE (e.g. 32 heads x 256 tiles fits;
+ *     32 heads x 1024 tiles does not).  Every refusal leaves a message in
+ *     poem_last_error.
  *   - All calls share the array and each call overwrites it: calls whose kernels
  *     overlap on the GPU (other streams, other host threads) race; serialise them.
  *   - The first call on a device resolves the array's device address with that
- *     device current; make that first call before any stream capture.
+ *     device current; make that first call before any stream capture.  After a
+ *     device reset (cudaDeviceReset) the next call finds the old address gone and
+ *     resolves it again.
  *   - There is no workspace error word to poll: a col_idx that is too small is
  *     seen by comparing row_ptr[n_q_heads*T] with col_capacity after the call.
  */

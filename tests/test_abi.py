@@ -125,6 +125,29 @@ def test_select_rejects_small_workspace_and_negative_capacity(poem):
                                  None) == 1
 
 
+def test_select_noalloc_host_refusals_set_the_message(poem):
+    """poem_select_noalloc refuses bad arguments on the host, before resolving its
+    scratch array, and leaves a message for every refusal."""
+    f = poem._lib.poem_select_noalloc
+    ok = ctypes.c_void_p(1 << 20)
+    mis = ctypes.c_void_p((1 << 20) + 4)
+    poem._lib.poem_select(ctypes.byref(_shape(poem)), ok, ok, ctypes.c_float(-1.0), ok, ok, 100, None, ok, 1 << 30,
+                          None)  # leaves an unrelated message behind
+    cases = [
+        (_shape(poem, n_tokens=1024 * 128, n_q_heads=32, n_kv_heads=8, q_stride_tok=4096, kv_stride_tok=1024),
+         ok, 0.05, 100, 6, "static maximum"),
+        (_shape(poem), ok, float("nan"), 100, 1, "poem_select_noalloc: tau"),
+        (_shape(poem), ok, 0.05, -1, 1, "col_capacity"),
+        (_shape(poem), mis, 0.05, 100, 1, "aligned"),
+        (_shape(poem, head_dim=96), ok, 0.05, 100, 2, "head_dim"),
+    ]
+    for sh, ih, tau, cap, status, text in cases:
+        poem._lib.poem_select(ctypes.byref(_shape(poem)), ok, ok, ctypes.c_float(-1.0), ok, ok, 100, None, ok,
+                              1 << 30, None)
+        assert f(ctypes.byref(sh), ih, ok, ctypes.c_float(tau), ok, ok, cap, None, None) == status
+        assert text in poem.poem_last_error(), (text, poem.poem_last_error())
+
+
 def test_status_strings(poem):
     for code, name in poem.STATUS.items():
         assert poem.poem_status_string(code) == name

@@ -89,3 +89,26 @@ def test_noalloc_refuses_shapes_beyond_its_fixed_scratch(poem):
                                        _p(dummy), dummy.numel(), None, None)
     assert poem.STATUS[st] == "POEM_ERR_WORKSPACE"
     assert "static maximum" in poem.poem_last_error()
+
+
+def test_noalloc_refusals_leave_a_message(poem):
+    """Every refusal sets poem_last_error, so a caller never reads an earlier call's text."""
+    shape = _shape(poem, 4, 2, 8)
+    buf = torch.zeros(4096, dtype=torch.int32, device="cuda")
+    f = torch.zeros(4096, dtype=torch.float32, device="cuda")
+    poem._lib.poem_select_noalloc(ctypes.byref(_shape(poem, 32, 8, 1024)), _p(f), _p(f), ctypes.c_float(0.05),
+                                  _p(buf), _p(buf), buf.numel(), None, None)
+    assert "static maximum" in poem.poem_last_error()
+    st = poem._lib.poem_select_noalloc(ctypes.byref(shape), _p(f), _p(f), ctypes.c_float(float("nan")), _p(buf),
+                                       _p(buf), buf.numel(), None, None)
+    assert poem.STATUS[st] == "POEM_ERR_INVALID_ARG"
+    msg = poem.poem_last_error()
+    assert msg and "tau" in msg
+    st = poem._lib.poem_select_noalloc(ctypes.byref(shape), _p(f), _p(f), ctypes.c_float(0.05), _p(buf), _p(buf),
+                                       -1, None, None)
+    assert poem.STATUS[st] == "POEM_ERR_INVALID_ARG"
+    assert "col_capacity" in poem.poem_last_error()
+    st = poem._lib.poem_select_noalloc(ctypes.byref(shape), None, _p(f), ctypes.c_float(0.05), _p(buf), _p(buf),
+                                       buf.numel(), None, None)
+    assert poem.STATUS[st] == "POEM_ERR_INVALID_ARG"
+    assert "aligned" in poem.poem_last_error()
