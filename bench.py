@@ -20,7 +20,8 @@ whole job's: max-over-ranks time / (N * K).
 
 --impl reference times the fp64 CPU oracle (test infrastructure; the reference
 arm of this benchmark) on a bounded sample of the same layer's (head, tile)
-units on the host cores and extrapolates to ms/layer by the work per unit.
+units on the host cores -- tile pairs (i, T-1-i), the last tile included, run in
+parallel over the host threads -- and extrapolates to ms/layer by visible blocks.
 """
 from __future__ import annotations
 
@@ -380,11 +381,22 @@ def run_ours(args):
                       "h2d_bytes_per_step": h2d_bytes, "d2h_bytes_per_step": d2h_bytes,
                       "mode": "serial: copy in, compute, copy out on one stream"}
 
+    # The practical selector on the same inputs (a nested record; the headline value
+    # stays the exact selector's).
+    prac, prac_o, prac_layer = None, None, None
+    if not practical and not args.no_practical:
+        prac, prac_o, prac_layer = practical_record(poem, q, k, v, args, n, hq, d, B, peaks, peak_src)
+        prac["gpu_launches"] = 7 * args.steps
+
     extra = {}
     if not args.no_quality and rank == 0:
-        extra = quality_report(poem, q, k, v, layer, tau, n, hq, T, B, dev)
+        extra = quality_report(poem, q, k, v, layer, tau, n, hq, T, B, dev,
+                               extra_outputs={"practical": prac_o} if prac_o is not None else None)
         if practical:
             extra["err_vs_dense"]["practical"] = extra["err_vs_dense"].pop("poem")
+        if prac is not None and "practical" in extra.get("err_vs_dense", {}):
+            prac["err_vs_dense"] = extra["err_vs_dense"].pop("practical")
+    del prac_o, prac_layer
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -436,6 +448,8 @@ def run_ours(args):
     }
     if cpu and "parity" in cpu:
         line["oracle_parity"] = cpu.pop("parity")
+    if prac is not None:
+        line["practical"] = prac
     line.update(extra)
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -443,9 +457,69 @@ def run_ours(args):
         torch.distributed.destroy_process_group()
 
 
-def quality_report(poem, q, k, v, layer, tau, n, hq, T, B, dev):
+def practical_record(poem, q, k, v, args, n, hq, d, B, peaks, peak_src):
+    """The practical selector (pooled estimates, mass shortlist rho, rerank
+    log m~ + w log d~, pooled-mass threshold gamma) timed on the same inputs with the
+    same loop as the headline line: W warm-up steps, K steps with CUDA events around
+    each call.  Returns (record, output, layer)."""
+    T = n // B
+    lay = poem.alloc_layer(q, k, block=B, practical=True)
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        if ev:
+            ev[0].record(stream)
+        poem.poem_score_pooled(q, k, v, lay.m_pool, lay.d_pool, lay.ws_pooled, shape=lay.shape)
+        if ev:
+            ev[1].record(stream)
+        poem.poem_select_practical(lay.shape, lay.m_pool, lay.d_pool, args.w, args.gamma, args.rho, lay.row_ptr,
+                                   lay.col_idx, lay.ws_select, order=lay.order)
+        if ev:
+            ev[2].record(stream)
+        poem.bsa_fwd(q, k, v, lay.row_ptr, lay.col_idx, lay.o, lay.ws_fwd, order=lay.order, shape=lay.shape)
+        if ev:
+            ev[3].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for s_ in range(args.steps):
+        step(evs[s_])
+    t1.record(stream)
+    torch.cuda.synchronize()
+    for ws in (lay.ws_pooled, lay.ws_select, lay.ws_fwd):
+        poem.poem_check(ws)
+    ms = t0.elapsed_time(t1) / args.steps
+    pool_ms = float(np.mean([e[0].elapsed_time(e[1]) for e in evs]))
+    sel_ms = float(np.mean([e[1].elapsed_time(e[2]) for e in evs]))
+    fwd_ms = float(np.mean([e[2].elapsed_time(e[3]) for e in evs]))
+    rp = lay.row_ptr.cpu().numpy()
+    ci = lay.col_idx[: int(rp[-1])].cpu().numpy()
+    rflops = retained_flops(rp, ci, T, d, B)
+    tf = rflops / (fwd_ms * 1e-3) / 1e12
+    rec = {"selector": "practical", "w": args.w, "gamma": args.gamma, "rho": args.rho,
+           "ms_per_layer": round(ms, 4), "steps": args.steps, "warmup": args.warmup,
+           "breakdown_ms": {"poem_score_pooled": round(pool_ms, 4), "poem_select_practical": round(sel_ms, 4),
+                            "bsa_fwd": round(fwd_ms, 4)},
+           "density": round(int(rp[-1]) / (hq * T * (T + 1) // 2), 5),
+           "score_select_over_fwd": round((pool_ms + sel_ms) / fwd_ms, 4),
+           "roofline": {"bound": "tensor", "kernel": "bsa_fwd", "achieved": round(tf, 2),
+                        "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                        "frac": round(tf / peaks["bf16_tflops_sustained"], 4),
+                        "frac_of_burst_peak": round(tf / peaks["bf16_tflops"], 4),
+                        "peak_source": peak_src + ", sustained bf16 (kernel timed inside a long step)",
+                        "algorithmic_flops_per_launch": rflops, "traffic": None,
+                        "traffic_note": "no ncu capture of bsa_fwd on these lists"}}
+    return rec, lay.o, lay
+
+
+def quality_report(poem, q, k, v, layer, tau, n, hq, T, B, dev, extra_outputs=None):
     """Output error of the POEM lists and of mass-only lists at the same budget,
-    both against dense attention (bsa_fwd over every causal block)."""
+    both against dense attention (bsa_fwd over every causal block); extra_outputs
+    (name -> O) are compared with the same dense output."""
     rp_all, ci_all = poem_synth.random_block_lists(1, T, 1.0, seed=0)
     counts = np.diff(rp_all)
     rp_dense = np.concatenate([[0], np.cumsum(np.tile(counts, hq))]).astype(np.int32)
@@ -470,7 +544,10 @@ def quality_report(poem, q, k, v, layer, tau, n, hq, T, B, dev):
                 "rel_fro": float(diff.norm() / o_dense.float().norm()),
                 "max_row_l2": float(diff.norm(dim=-1).max())}
 
-    return {"err_vs_dense": {"poem": err(layer.o), "mass_only_same_budget": err(o_mass)}}
+    out = {"poem": err(layer.o), "mass_only_same_budget": err(o_mass)}
+    for name, o in (extra_outputs or {}).items():
+        out[name] = err(o)
+    return {"err_vs_dense": out}
 
 
 def gpu_rows_fn(layer, T, B):
@@ -487,67 +564,88 @@ def gpu_rows_fn(layer, T, B):
     return rows
 
 
-def cpu_baseline(x, n, hq, hkv, d, B, tau, budget_s, gpu_rows=None):
-    """Oracle (fp64, host cores) on a bounded sample of (head, tile) units, scaled to
-    a whole layer by work per unit (score ~ i+1 blocks, masked attention ~ kept
-    blocks; selection is negligible).  With `gpu_rows` the same units also cross-check
-    the CUDA path (outside the timed work): the worst Î or m̂ error as a fraction of its
-    tolerance (Î: 1e-3 relative + 1e-5 m_b R; m̂: 1e-3 relative + 1e-9), how many lists
-    equal the oracle's,
-    and the largest output error against the oracle's attention over the GPU's list."""
+def oracle_sample_units(hq, T, n_pairs, salt=0):
+    """(head, tile) units for the oracle baseline: n_pairs pairs of tiles (i, T-1-i)
+    with i spread over [0, T/2) from i = 0, so that every pair holds T + 1 visible
+    blocks (the pairs balance across the host threads) and the sample holds the last
+    tile T-1."""
+    units = []
+    for p_ in range(n_pairs):
+        i = min(T // 2, int(p_ * (T / 2) / n_pairs)) if T > 1 else 0
+        h = (p_ * 7 + salt) % hq
+        units.append((h, T - 1 - i))
+        if T - 1 - i != i or T == 1:
+            units.append(((h + 1) % hq, i))
+    return sorted(set(units), key=lambda u: -u[1])  # largest first (dynamic schedule)
+
+
+def cpu_baseline(x, n, hq, hkv, d, B, tau, budget_s, gpu_rows=None, n_pairs=None, salt=0):
+    """Oracle (fp64, host cores) on a sample of (head, tile) units -- scores, selection
+    and masked attention over the kept blocks -- run as one batch over all host
+    threads (units in parallel), scaled to the whole layer by visible blocks (score
+    ~ i+1 blocks, masked attention ~ kept blocks; selection is negligible).  With
+    `gpu_rows` the same units also cross-check the CUDA path (outside the timed work):
+    the worst Î or m̂ error as a fraction of its tolerance (Î: 1e-3 relative + 1e-5
+    m_b R; m̂: 1e-3 relative + 1e-9), how many lists equal the oracle's, and the
+    largest output error against the oracle's attention over the GPU's list."""
     import oracle
 
     oracle.build()
     T = n // B
     prob = oracle.Problem(q=poem_synth.bf16_bits(x["q"]), k=poem_synth.bf16_bits(x["k"]),
                           v=poem_synth.bf16_bits(x["v"]), block=B, n_sample=16)
-    # sample: tiles spread over the causal range, growing until the budget is used
-    units = []
-    per_unit = []
-    t_total = 0.0
-    cand_tiles = [max(0, int(T * f) - 1) for f in (1 / 64, 1 / 16, 1 / 8, 1 / 4)]
+    cores = oracle.num_threads()
+    units = oracle_sample_units(hq, T, n_pairs or max(2, cores), salt)
     R = float(x["v"].float().norm(dim=-1).max())
-    par = {"units": 0, "score_tol_ratio_max": 0.0, "lists_equal": 0, "o_max_abs": 0.0}
 
-    def one_row_list(r, lst):
-        rp = np.zeros(hq * T + 1, dtype=np.int32)
-        rp[r + 1:] = len(lst)
-        return rp, np.asarray(lst, dtype=np.int32)
+    t0 = time.perf_counter()
+    Ih, mh = prob.score_units(units)
+    rows = [(h, i) for h, i in units]
+    ref_rp, ref_ci, _ = oracle.select_all(hq, T, Ih, mh, tau, rows=rows)
+    # the kept lists as a layer-wide CSR (rows not sampled are empty)
+    counts = np.zeros(hq * T, dtype=np.int32)
+    lists = {}
+    for u, (h, i) in enumerate(units):
+        lists[h * T + i] = ref_ci[ref_rp[u]:ref_rp[u + 1]]
+        counts[h * T + i] = len(lists[h * T + i])
+    rp = np.zeros(hq * T + 1, dtype=np.int32)
+    rp[1:] = np.cumsum(counts)
+    ci = np.concatenate([lists[r] for r in sorted(lists)]).astype(np.int32)
+    prob.masked_units(units, rp, ci)
+    t_total = time.perf_counter() - t0
 
-    h = 0
-    for i in cand_tiles:
-        if t_total > budget_s:
-            break
-        t0 = time.perf_counter()
-        Ih, mh = prob.score_units([(h, i)])
-        off = oracle.tri_offset(T, h, i)
-        keep, _ = oracle.select_row(i, Ih[off:off + i + 1], mh[off:off + i + 1], tau)
-        r = h * T + i
-        prob.masked_units([(h, i)], *one_row_list(r, keep))
-        dt = time.perf_counter() - t0
-        t_total += dt
-        units.append((h, i))
-        per_unit.append(dt / (i + 1))
-        if gpu_rows is not None:
+    sampled_blocks = sum(i + 1 for _, i in units)
+    total_blocks = hq * T * (T + 1) / 2
+    est_ms = t_total * total_blocks / sampled_blocks * 1e3
+    out = {"value": round(est_ms, 1), "unit": "ms/layer", "cores": min(cores, len(units)), "kind": "oracle",
+           "sample": f"{len(units)} (head, tile) units, tile pairs (i, T-1-i) spread over the causal range "
+                     f"(tiles {min(u[1] for u in units)}..{max(u[1] for u in units)} of {T}), score + select + "
+                     f"masked attention in one batch over the host threads, {t_total:.1f} s, scaled by visible "
+                     f"blocks to the whole layer",
+           "extrapolated": True}
+    if gpu_rows is not None:
+        par = {"units": 0, "score_tol_ratio_max": 0.0, "lists_equal": 0, "o_max_abs": 0.0}
+        g_counts = np.zeros(hq * T, dtype=np.int32)
+        g_lists = {}
+        for h, i in units:
             gI, gm, glist, go = gpu_rows(h, i)
+            off = oracle.tri_offset(T, h, i)
             rI, rm = Ih[off:off + i + 1], mh[off:off + i + 1]
             tol_I = 1e-3 * rI + 1e-5 * rm * R + 1e-30
             tol_m = 1e-3 * rm + 1e-9
             par["units"] += 1
             par["score_tol_ratio_max"] = max(par["score_tol_ratio_max"], float(np.max(np.abs(gI - rI) / tol_I)),
                                              float(np.max(np.abs(gm - rm) / tol_m)))
-            par["lists_equal"] += int(np.array_equal(glist, np.asarray(keep)))
-            Og, _ = prob.masked_units([(h, i)], *one_row_list(r, glist))
-            par["o_max_abs"] = max(par["o_max_abs"], float(np.max(np.abs(go - np.asarray(Og[0])[:B]))))
-        h = (h + 1) % hq
-    rate = float(np.mean(per_unit))  # seconds per visible block of a unit
-    total_blocks = hq * T * (T + 1) / 2
-    est_ms = rate * total_blocks * 1e3
-    out = {"value": round(est_ms, 1), "unit": "ms/layer", "cores": oracle.num_threads(), "kind": "oracle",
-           "sample": f"{len(units)} (head, tile) units at tiles {[u[1] for u in units]} (score + select + masked "
-                     f"attention), {t_total:.1f} s, scaled by visible blocks per unit to the whole layer",
-           "extrapolated": True}
-    if gpu_rows is not None:
+            par["lists_equal"] += int(np.array_equal(glist, lists[h * T + i]))
+            g_lists[h * T + i] = (np.asarray(glist, dtype=np.int32), go)
+            g_counts[h * T + i] = len(glist)
+        g_rp = np.zeros(hq * T + 1, dtype=np.int32)
+        g_rp[1:] = np.cumsum(g_counts)
+        g_ci = np.concatenate([g_lists[r][0] for r in sorted(g_lists)]).astype(np.int32)
+        Og, _ = prob.masked_units(units, g_rp, g_ci)
+        for u, (h, i) in enumerate(units):
+            go = g_lists[h * T + i][1]
+            par["o_max_abs"] = max(par["o_max_abs"], float(np.max(np.abs(go - np.asarray(Og[u])[:B]))))
         out["parity"] = par
     return out
 
@@ -599,7 +697,7 @@ def run_reference(args):
     practical = args.selector == "practical"
     for s in range(args.warmup + args.steps):
         cb = (cpu_baseline_practical(x, n, hq, hkv, d, B, args.w, args.gamma, args.rho, budget) if practical
-              else cpu_baseline(x, n, hq, hkv, d, B, tau, budget))
+              else cpu_baseline(x, n, hq, hkv, d, B, tau, budget, n_pairs=args.ref_pairs, salt=s))
         if s >= args.warmup:
             vals.append(cb["value"])
     v = float(np.mean(vals))
@@ -1141,8 +1239,12 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-quality", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-practical", action="store_true",
+                    help="skip the nested practical-selector record of the default (exact) run")
     ap.add_argument("--cpu-budget-s", type=float, default=15.0)
     ap.add_argument("--ref-step-budget-s", type=float, default=8.0)
+    ap.add_argument("--ref-pairs", type=int, default=4,
+                    help="reference arm: tile pairs (i, T-1-i) per step (the sample rotates over heads)")
     ap.add_argument("--selector", choices=["exact", "practical"], default="exact")
     ap.add_argument("--shard", choices=["replicas", "heads"], default="replicas",
                     help="N > 1: independent whole-layer replicas (weak scaling) or one layer split by KV-head "

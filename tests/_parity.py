@@ -79,6 +79,17 @@ def score_err_excess(gpu_I, ref_I, gpu_m, ref_m, R: float):
     return float(max(np.max(np.abs(gI - rI) / tolI), np.max(np.abs(gm - rm) / tolm)))
 
 
+def masked_rows_threaded(prob, items):
+    """Oracle masked-attention rows for a list of (h, token, blocks) items, computed
+    concurrently on the host cores (each oracle call is one row, single-threaded,
+    and releases the interpreter lock).  Returns an array [len(items), d]."""
+    from concurrent.futures import ThreadPoolExecutor
+
+    with ThreadPoolExecutor(max_workers=max(1, oracle.num_threads())) as ex:
+        rows = list(ex.map(lambda it: prob.masked_row(it[0], it[1], it[2])[0], items))
+    return np.stack(rows) if rows else np.zeros((0, prob.head_dim))
+
+
 def max_value_norm(v: torch.Tensor) -> float:
     return float(v.float().norm(dim=-1).max())
 

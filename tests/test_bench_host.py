@@ -102,3 +102,17 @@ def test_sampled_oracle_cross_check_scores_a_planted_error():
                              gpu_rows=lambda h, i: rows_from_oracle(h, i, plant=True))["parity"]
     assert 2.0 < bad["score_tol_ratio_max"] < 3.1
     assert abs(bad["o_max_abs"] - 0.25) < 1e-9
+
+
+def test_oracle_sample_reaches_the_last_tile_and_balances_pairs():
+    """The CPU-baseline sample: at least 16 units at 128K, the last tile included,
+    every tile pair (i, T-1-i) holding T + 1 visible blocks."""
+    T = 1024
+    units = bench.oracle_sample_units(32, T, 16)
+    tiles = sorted(i for _, i in units)
+    assert len(units) >= 16 and tiles[-1] == T - 1 and tiles[0] == 0
+    lo = [i for i in tiles if i < T // 2]
+    hi = sorted((i for i in tiles if i >= T // 2), reverse=True)
+    assert len(lo) == len(hi) and all(a + b == T - 1 for a, b in zip(lo, hi))
+    assert units == sorted(units, key=lambda u: -u[1])
+    assert len(set(units)) == len(units) and all(0 <= h < 32 for h, _ in units)

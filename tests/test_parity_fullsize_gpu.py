@@ -2,20 +2,23 @@
 (poem_score -> poem_select with a work order -> bsa_fwd following that order).
 
 The oracle cannot run a whole 128K layer, so it checks a deterministic sample of
-(head, tile) units -- the first and last tiles of several heads and a few in
-between.  Units are independent in every step, so each sampled unit is an exact
-check of that unit: its scores I_hat/m_hat for all visible blocks, its block
-list (against the oracle's selection on the oracle's own scores, cut rule), and
-all 128 output rows of bsa_fwd (against oracle masked attention on the GPU's
-list)."""
+(head, tile) units: every 16th tile of every 4th head plus the first three and the
+last three tiles of every head (about 700 units at 128K, 560 at 64K).  Units are
+independent in every step, so each sampled unit is an exact check of that unit:
+its scores I_hat/m_hat for all visible blocks and its block list (against the
+oracle's selection on the oracle's own scores, cut rule).  bsa_fwd's output is
+checked against oracle masked attention on the GPU's list: all 128 rows of the
+last tile of every head, and 8 spread rows (0, 17, ..., 119, 127) of every other
+sampled unit -- the oracle computes each row on its own, so a sampled row is an
+exact check of that row."""
 import numpy as np
 import pytest
 import torch
 
 import oracle
 import poem_synth
-from _parity import (FWD_MAX_ABS, FWD_MEAN_ABS, compare_fwd, csr_rows, lists_agree_at_cut, max_value_norm,
-                     problem_from, score_err_excess)
+from _parity import (FWD_MAX_ABS, FWD_MEAN_ABS, compare_fwd, csr_rows, lists_agree_at_cut, masked_rows_threaded,
+                     max_value_norm, problem_from, score_err_excess)
 
 pytestmark = pytest.mark.gpu
 
@@ -39,7 +42,19 @@ def _sample_units(hq, T, extra):
     return sorted(units)
 
 
-def _check_layer(poem, x, B, tau, units):
+def _survey_units(hq, T):
+    """Every 16th tile of every 4th head, and the first and last three tiles of every head."""
+    units = {(h, i) for h in range(0, hq, 4) for i in range(0, T, 16)}
+    units |= {(h, i) for h in range(hq) for i in (0, 1, 2, T - 3, T - 2, T - 1) if 0 <= i < T}
+    return sorted(units)
+
+
+SAMPLED_ROWS = (0, 17, 34, 51, 68, 85, 102, 119, 127)
+
+
+def _check_layer(poem, x, B, tau, units, full_units=None, row_sample=False):
+    """full_units: units whose every output row is checked (default: all of units);
+    with row_sample, the other units are checked on SAMPLED_ROWS."""
     q, k, v = x["q"].cuda(), x["k"].cuda(), x["v"].cuda()
     hq = q.shape[1]
     T = q.shape[0] // B
@@ -63,9 +78,18 @@ def _check_layer(poem, x, B, tau, units):
     full_ref = [ref_rows.get(r, gpu_rows[r]) for r in range(hq * T)]
     _, bad = lists_agree_at_cut(gpu_rows, full_ref, Ir, mr, hq, T, tau)
     assert not bad, bad
-    O_ref, _ = prob.masked_units(units, rp, ci)
-    mx, mean = compare_fwd(layer.o, O_ref, units, B)
+    full = list(units) if full_units is None else sorted(full_units)
+    O_ref, _ = prob.masked_units(full, rp, ci)
+    mx, mean = compare_fwd(layer.o, O_ref, full, B)
     assert mx <= FWD_MAX_ABS and mean <= FWD_MEAN_ABS, (mx, mean)
+    if row_sample:
+        rest = [u for u in units if u not in set(full)]
+        items = [(h, i * B + r, gpu_rows[h * T + i]) for h, i in rest for r in SAMPLED_ROWS if r < B]
+        ref = masked_rows_threaded(prob, items)
+        og = layer.o.float().cpu().numpy()
+        got = np.stack([og[t, h] for h, t, _ in items])
+        e = np.abs(got - ref)
+        assert float(e.max()) <= FWD_MAX_ABS and float(e.mean()) <= FWD_MEAN_ABS, (float(e.max()), float(e.mean()))
     # work order: a permutation of the rows
     assert sorted(layer.order.cpu().numpy().tolist()) == list(range(hq * T))
     return rp
@@ -76,7 +100,9 @@ def test_llama_layer_128k(poem):
     n, hq, hkv, d, B = 131072, 32, 8, 128, 128
     x = poem_synth.heavy_block_layer(n, hq, hkv, d, block=B, rope_base=500000.0, seed=0)
     T = n // B
-    rp = _check_layer(poem, x, B, 0.05, _sample_units(hq, T, [(7, 300), (20, 1000)]))
+    units = _survey_units(hq, T)
+    assert len(units) >= 128
+    rp = _check_layer(poem, x, B, 0.05, units, full_units=[(h, T - 1) for h in range(hq)], row_sample=True)
     assert rp[-1] > 0
 
 
@@ -85,7 +111,9 @@ def test_qwen3_14b_layer_64k(poem):
     n, hq, hkv, d, B = 65536, 40, 8, 128, 128
     x = poem_synth.heavy_block_layer(n, hq, hkv, d, block=B, rope_base=1000000.0, seed=0)
     T = n // B
-    _check_layer(poem, x, B, 0.05, _sample_units(hq, T, [(39, 255), (12, 401)]))
+    units = _survey_units(hq, T)
+    assert len(units) >= 96
+    _check_layer(poem, x, B, 0.05, units, full_units=[(h, T - 1) for h in range(hq)], row_sample=True)
 
 
 @pytest.mark.parametrize("tau", [0.02, 0.05, 0.1])
