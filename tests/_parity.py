@@ -63,6 +63,26 @@ def compare_fwd_excess(o_gpu: torch.Tensor, O_ref: np.ndarray, units, block: int
     return worst, tot / cnt
 
 
+def bf16_half_ulp(x):
+    """Half a bf16 unit in the last place at |x| (8 significant bits): the most that
+    rounding a value of that magnitude to bf16 can move it (2^(e-8) for |x| in
+    [2^e, 2^(e+1)))."""
+    ax = np.maximum(np.abs(np.asarray(x, np.float64)), 2.0 ** -126)
+    return np.ldexp(1.0, (np.floor(np.log2(ax)) - 8).astype(np.int64))
+
+
+def fwd_out_excess(o_gpu_rows, o_ref_rows):
+    """bsa_fwd rows (bf16 values, as floats) against oracle rows: the largest ratio
+    |o_gpu - o_ref| / (FWD_MAX_ABS + bf16_half_ulp(o_ref)) (<= 1 passes) and the mean
+    abs error.  FWD_MAX_ABS bounds the fp32-accumulated arithmetic; the output buffer
+    is bf16, and storing a value in it moves it by up to half a bf16 ulp -- 0.0078 at
+    |o| in [2, 4), 0.0156 at [4, 8) -- which no kernel can avoid."""
+    got = np.asarray(o_gpu_rows, np.float64)
+    ref = np.asarray(o_ref_rows, np.float64)
+    e = np.abs(got - ref)
+    return float(np.max(e / (FWD_MAX_ABS + bf16_half_ulp(ref)))), float(e.mean())
+
+
 def score_err_excess(gpu_I, ref_I, gpu_m, ref_m, R: float):
     """Largest violation ratio of the score tolerances (<= 1 passes):
       |dI_b| <= SCORE_REL * I_b + 1e-5 * m_b * R

@@ -8,17 +8,21 @@ independent in every step, so each sampled unit is an exact check of that unit:
 its scores I_hat/m_hat for all visible blocks and its block list (against the
 oracle's selection on the oracle's own scores, cut rule).  bsa_fwd's output is
 checked against oracle masked attention on the GPU's list: all 128 rows of the
-last tile of every head, and 8 spread rows (0, 17, ..., 119, 127) of every other
+last tile of every head, and 9 spread rows (0, 17, ..., 119, 127) of every other
 sampled unit -- the oracle computes each row on its own, so a sampled row is an
-exact check of that row."""
+exact check of that row.  The output bound is the contract's 1e-2 on the
+fp32-accumulated arithmetic plus half a bf16 ulp of the value for the bf16 output
+buffer: the sample reaches the first rows of every head, where a query attends to
+a few keys and |o| reaches 4, and storing such a value in bf16 alone moves it by up
+to 0.0156."""
 import numpy as np
 import pytest
 import torch
 
 import oracle
 import poem_synth
-from _parity import (FWD_MAX_ABS, FWD_MEAN_ABS, compare_fwd, csr_rows, lists_agree_at_cut, masked_rows_threaded,
-                     max_value_norm, problem_from, score_err_excess)
+from _parity import (FWD_MAX_ABS, FWD_MEAN_ABS, compare_fwd, csr_rows, fwd_out_excess, lists_agree_at_cut,
+                     masked_rows_threaded, max_value_norm, problem_from, score_err_excess)
 
 pytestmark = pytest.mark.gpu
 
@@ -80,16 +84,17 @@ def _check_layer(poem, x, B, tau, units, full_units=None, row_sample=False):
     assert not bad, bad
     full = list(units) if full_units is None else sorted(full_units)
     O_ref, _ = prob.masked_units(full, rp, ci)
-    mx, mean = compare_fwd(layer.o, O_ref, full, B)
-    assert mx <= FWD_MAX_ABS and mean <= FWD_MEAN_ABS, (mx, mean)
+    og = layer.o.float().cpu().numpy()
+    got = np.stack([og[i * B:(i + 1) * B, h] for h, i in full])
+    worst, mean = fwd_out_excess(got, O_ref)
+    assert worst <= 1.0 and mean <= FWD_MEAN_ABS, (worst, mean)
     if row_sample:
         rest = [u for u in units if u not in set(full)]
         items = [(h, i * B + r, gpu_rows[h * T + i]) for h, i in rest for r in SAMPLED_ROWS if r < B]
         ref = masked_rows_threaded(prob, items)
-        og = layer.o.float().cpu().numpy()
         got = np.stack([og[t, h] for h, t, _ in items])
-        e = np.abs(got - ref)
-        assert float(e.max()) <= FWD_MAX_ABS and float(e.mean()) <= FWD_MEAN_ABS, (float(e.max()), float(e.mean()))
+        worst, mean = fwd_out_excess(got, ref)
+        assert worst <= 1.0 and mean <= FWD_MEAN_ABS, (worst, mean)
     # work order: a permutation of the rows
     assert sorted(layer.order.cpu().numpy().tolist()) == list(range(hq * T))
     return rp
