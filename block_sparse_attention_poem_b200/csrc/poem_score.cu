@@ -26,12 +26,15 @@
 // Pipeline (one CTA per SM, TMEM fully allocated):
 //   TMEM  S0 [0,128)  S1 [128,256)  -- S double-buffered: S_{b+1} is computed while
 //                                      the softmax of block b runs
-//         O / P V [256,384)           -- pass 1: running O; pass 2: P_b V_b
-//         o [384,512)                 -- pass 2: the row's dense output (from pass 1)
-//   smem  Q tile, 2-stage K ring, 2-stage V ring (160 KB at d = 128)
-//   warps 0-3 softmax (one sampled query per thread), warps 4-7 (pass 2 only) the
-//         norm of P_b V_b - m_b o while the softmax warps move on to block b+1,
-//         then one TMA warp and one MMA-issuing warp.
+//         accumulators [256,384) and [384,512): P_b V_b of block b goes to
+//         accumulator b % 2 -- pass 1: the even and the odd blocks' partial outputs;
+//         pass 2: P_b V_b of one block, double-buffered for the norm warps
+//   smem  Q tile, 3-stage K ring, 2-stage V ring (192 KB at d = 128)
+//   pass 1: warps 0-3 and 4-7 are two softmax warpgroups, one for the even and one
+//           for the odd blocks, each with its own running max and sum (merged at
+//           the end); pass 2: warps 0-3 softmax, warps 4-7 the norm of
+//           P_b V_b - m_b o with o held in registers.  Warp 8 issues TMA loads;
+//           warp 9 issues the MMAs, converged, from one elected lane.
 //   MMA order: S_0, S_1, PV_0, S_2, PV_1, ...
 //
 // Precision: P enters the P V contraction as a hi/lo pair of bf16 matrices
@@ -53,32 +56,33 @@ struct ScoreCfg {
   static constexpr int kGroups = 8;        // groups of 16 sampled queries per CTA
   static constexpr int kRowsPerGroup = 16;
   static constexpr int kChunks = D / 64;
-  static constexpr int kStages = 2;
+  static constexpr int kStagesK = 3;       // K ring: a load is issued two blocks ahead of its use
+  static constexpr int kStagesV = 2;
   static constexpr int kQBytes = M * D * 2;
   static constexpr int kKVBytes = BN * D * 2;
   static constexpr int kOffQ = 0;
   static constexpr int kOffK = kOffQ + kQBytes;
-  static constexpr int kOffV = kOffK + kStages * kKVBytes;
-  static constexpr int kOffBar = kOffV + kStages * kKVBytes;
-  static constexpr int kOffM = kOffBar + 256;                 // m_b hand-off, [2][128] floats
+  static constexpr int kOffV = kOffK + kStagesK * kKVBytes;
+  static constexpr int kOffBar = kOffV + kStagesV * kKVBytes;
+  static constexpr int kOffM = kOffBar + 256;                 // [2][128] floats: m_b hand-off (pass 2)
+                                                              // or the odd warpgroup's max / sum (pass 1)
   // at least 120 KB so that one CTA (holding all 512 TMEM columns) occupies an SM
   static constexpr int kSmemBytes = (kOffM + 2 * 128 * 4 + 1024) > 122880 ? (kOffM + 2 * 128 * 4 + 1024) : 122880;
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kColS = 0;     // S buffer s at [128 s, 128 s + BN)
-  static constexpr uint32_t kColO = 256;   // O (pass 1) or P_b V_b (pass 2)
-  static constexpr uint32_t kColOd = 384;  // pass 2: dense output o of the row
-  static constexpr int kWarpProd = (PASS == 2) ? 8 : 4;
-  static constexpr int kWarpMma = kWarpProd + 1;
-  static constexpr int kThreads = (kWarpMma + 1) * 32;
+  static constexpr uint32_t kColAcc = 256; // accumulator s at [256 + 128 s, 256 + 128 s + D)
+  static constexpr int kWarpProd = 8;      // warps 0-7 compute, 8 TMA, 9 MMA
+  static constexpr int kWarpMma = 9;
+  static constexpr int kThreads = 320;
   static constexpr uint32_t kIdescQK = idesc_bf16_f32(M, BN, 0);
   static constexpr uint32_t kIdescPV = idesc_bf16_f32(M, D, 1);
 };
 
 struct ScoreBarriers {
   uint64_t q_full;
-  uint64_t k_full[2], k_empty[2], v_full[2], v_empty[2];
+  uint64_t k_full[3], k_empty[3], v_full[2], v_empty[2];
   uint64_t s_full[2], p_full[2];
-  uint64_t pv_full, pv_empty;    // P V accumulator done / released by the norm warps
+  uint64_t acc_full[2], acc_empty[2];  // accumulator s done / released by the norm warps (pass 2)
   uint64_t m_ready[2], m_empty[2];
   uint64_t drain;
   uint32_t tmem_base;
@@ -114,12 +118,13 @@ __device__ __forceinline__ void score_cta_coords(int cta, int ctas_per_g, int& g
   z0 = c * 8;
 }
 
-// p = 2^(s * scale * log2e - m) for one row's BN scores (masked columns > lim when
-// MASKED), written back over S as interleaved bf16 P_hi / P_lo words; *msum += sum p.
-// (Summing the unrounded p instead of P_hi + P_lo changes m_b by an unbiased
-// ~2^-18 relative error per weight.)
+// p = 2^(s * scale * log2e - m) for one row's BN scores (re-read from TMEM in 64-column
+// halves; masked columns > lim exactly 0 when MASKED), written back over S as
+// interleaved bf16 P_hi / P_lo words (per 16-key k-step: 8 words P_hi, then 8 words
+// P_lo = p - P_hi rounded to bf16).  Returns sum p.  (Summing the unrounded p instead
+// of P_hi + P_lo changes the sum by an unbiased ~2^-18 relative error per weight.)
 template <int BN, bool MASKED>
-__device__ __forceinline__ void split_chunks(uint32_t tS, float sl2, float m_use, int lim, float* msum) {
+__device__ __forceinline__ float exp_split_store(uint32_t tS, float sl2, float m_use, int lim) {
   const uint64_t scale2 = f2_pack(sl2, sl2);
   const uint64_t negm2 = f2_pack(-m_use, -m_use);
   uint64_t acc = f2_pack(0.f, 0.f);
@@ -132,12 +137,13 @@ __device__ __forceinline__ void split_chunks(uint32_t tS, float sl2, float m_use
     tmem_reg_fence(a[0]);
     tmem_reg_fence(a[1]);
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      uint32_t out[32];
+    for (int ks = 0; ks < 4; ++ks) {  // the four 16-key k-steps of this half
+      const uint32_t* src = a[ks >> 1] + (ks & 1) * 16;
+      uint32_t out[16];
 #pragma unroll
-      for (int x = 0; x < 16; ++x) {
-        const int col = cp * 64 + h * 32 + 2 * x;
-        const uint64_t xv = f2_fma(f2_pack(__uint_as_float(a[h][2 * x]), __uint_as_float(a[h][2 * x + 1])), scale2, negm2);
+      for (int x = 0; x < 8; ++x) {
+        const int col = cp * 64 + ks * 16 + 2 * x;
+        const uint64_t xv = f2_fma(f2_pack(__uint_as_float(src[2 * x]), __uint_as_float(src[2 * x + 1])), scale2, negm2);
         float x0, x1;
         f2_unpack(xv, x0, x1);
         float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
@@ -147,17 +153,43 @@ __device__ __forceinline__ void split_chunks(uint32_t tS, float sl2, float m_use
         }
         acc = f2_add(acc, f2_pack(p0, p1));
         const uint32_t wh = pack_bf16x2(p0, p1);
-        const uint32_t wl = pack_bf16x2(p0 - bf16lo_to_f32(wh), p1 - bf16hi_to_f32(wh));
-        // k-step (x / 8): words 0-7 P_hi, 8-15 P_lo
-        out[(x >> 3) * 16 + (x & 7)] = wh;
-        out[(x >> 3) * 16 + 8 + (x & 7)] = wl;
+        out[x] = wh;
+        out[8 + x] = pack_bf16x2(p0 - bf16lo_to_f32(wh), p1 - bf16hi_to_f32(wh));
       }
-      tmem_st32(tS + cp * 64 + h * 32, out);
+      tmem_st16(tS + cp * 64 + ks * 16, out);
     }
   }
   float a0, a1;
   f2_unpack(acc, a0, a1);
-  *msum += a0 + a1;
+  return a0 + a1;
+}
+
+// Maximum of one row's visible scores (columns <= lim when MASKED), read in 64-column halves.
+template <int BN, bool MASKED>
+__device__ __forceinline__ float row_max(uint32_t tS, int lim) {
+  float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+  for (int cp = 0; cp < BN / 64; ++cp) {
+    uint32_t a[2][32];
+    tmem_ld32(tS + cp * 64, a[0]);
+    tmem_ld32(tS + cp * 64 + 32, a[1]);
+    tmem_ld_wait();
+    tmem_reg_fence(a[0]);
+    tmem_reg_fence(a[1]);
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+      for (int x = 0; x < 32; x += 2) {
+        if (MASKED) {
+          const int col = cp * 64 + h * 32 + x;
+          mx[h] = fmax3(mx[h], (col <= lim) ? __uint_as_float(a[h][x]) : -INFINITY,
+                        (col + 1 <= lim) ? __uint_as_float(a[h][x + 1]) : -INFINITY);
+        } else {
+          mx[h] = fmax3(mx[h], __uint_as_float(a[h][x]), __uint_as_float(a[h][x + 1]));
+        }
+      }
+  }
+  return fmaxf(mx[0], mx[1]);
 }
 
 template <int D, int BN, int PASS>
@@ -188,18 +220,20 @@ __global__ void __launch_bounds__(ScoreCfg<D, BN, PASS>::kThreads, 1)
 
   if (tid == 0) {
     mbar_init(&sb->q_full, 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < 3; ++s) {
       mbar_init(&sb->k_full[s], 1);
       mbar_init(&sb->k_empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
       mbar_init(&sb->v_full[s], 1);
       mbar_init(&sb->v_empty[s], 1);
       mbar_init(&sb->s_full[s], 1);
       mbar_init(&sb->p_full[s], 128);
+      mbar_init(&sb->acc_full[s], 1);
+      mbar_init(&sb->acc_empty[s], 128);
       mbar_init(&sb->m_ready[s], 128);
       mbar_init(&sb->m_empty[s], 128);
     }
-    mbar_init(&sb->pv_full, 1);
-    mbar_init(&sb->pv_empty, 128);
     mbar_init(&sb->drain, 1);
     sb->abort_flag = 0;
     fence_barrier_init();
@@ -227,77 +261,86 @@ __global__ void __launch_bounds__(ScoreCfg<D, BN, PASS>::kThreads, 1)
       }
       int k_issued = 0, v_issued = 0;
       for (int b = 0; b < nb && !sb->abort_flag; ++b) {
-        const int s = b & 1;
-        const uint32_t par = ((b >> 1) & 1) ^ 1;  // completion #(b/2 - 1) of the stage's empty barrier
-        if (!wait_or_abort(&sb->k_empty[s], par, sb, p.err)) break;
-        mbar_arrive_expect_tx(&sb->k_full[s], C::kKVBytes);
+        // stage of block b and the completion of its empty barrier to wait for
+        // (#(b / stages - 1); a fresh barrier passes the parity-1 wait at once)
+        const int sk = b % C::kStagesK, sv = b & 1;
+        if (!wait_or_abort(&sb->k_empty[sk], ((b / C::kStagesK) & 1) ^ 1, sb, p.err)) break;
+        mbar_arrive_expect_tx(&sb->k_full[sk], C::kKVBytes);
         for (int c = 0; c < C::kChunks; ++c)
-          tma_load_3d(sK + s * C::kKVBytes + c * (BN * 128), &tmK, &sb->k_full[s], c * 64, g, b * BN);
+          tma_load_3d(sK + sk * C::kKVBytes + c * (BN * 128), &tmK, &sb->k_full[sk], c * 64, g, b * BN);
         ++k_issued;
-        if (!wait_or_abort(&sb->v_empty[s], par, sb, p.err)) break;
-        mbar_arrive_expect_tx(&sb->v_full[s], C::kKVBytes);
+        if (!wait_or_abort(&sb->v_empty[sv], ((b >> 1) & 1) ^ 1, sb, p.err)) break;
+        mbar_arrive_expect_tx(&sb->v_full[sv], C::kKVBytes);
         for (int c = 0; c < C::kChunks; ++c)
-          tma_load_3d(sV + s * C::kKVBytes + c * (BN * 128), &tmV, &sb->v_full[s], c * 64, g, b * BN);
+          tma_load_3d(sV + sv * C::kKVBytes + c * (BN * 128), &tmV, &sb->v_full[sv], c * 64, g, b * BN);
         ++v_issued;
       }
       // Drain: the last load issued into each stage must have landed.
       mbar_wait(&sb->q_full, 0, kDrainNs);
-      for (int b = max(0, k_issued - 2); b < k_issued; ++b) mbar_wait(&sb->k_full[b & 1], (b >> 1) & 1, kDrainNs);
+      for (int b = max(0, k_issued - C::kStagesK); b < k_issued; ++b)
+        mbar_wait(&sb->k_full[b % C::kStagesK], (b / C::kStagesK) & 1, kDrainNs);
       for (int b = max(0, v_issued - 2); b < v_issued; ++b) mbar_wait(&sb->v_full[b & 1], (b >> 1) & 1, kDrainNs);
     }
   } else if (warp == C::kWarpMma) {
     // ============================ MMA issuer ============================
-    if (lane == 0) {
-      const uint32_t tO = tmem + C::kColO;
-      const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV);
-      bool ok = wait_or_abort(&sb->q_full, 0, sb, p.err);
-      // P V_j with P = P_hi + P_lo read from S buffer j % 2.  Pass 1 accumulates over
-      // blocks; pass 2 starts a fresh accumulator per block, once the norm warps have
-      // read the previous one.
-      auto issue_pv = [&](int j) -> bool {
-        const int s = j & 1;
-        if (!wait_or_abort(&sb->p_full[s], (j >> 1) & 1, sb, p.err)) return false;
-        if (!wait_or_abort(&sb->v_full[s], (j >> 1) & 1, sb, p.err)) return false;
-        if (PASS == 2 && j > 0 && !wait_or_abort(&sb->pv_empty, (j - 1) & 1, sb, p.err)) return false;
-        tc_fence_after();
-        const uint32_t tP = tmem + C::kColS + s * 128;
-        const uint32_t aVs = aV + s * C::kKVBytes;
+    // The whole warp runs this loop converged (waits and operands are warp-uniform);
+    // one elected lane issues each MMA and commit.
+    // Order S_0, S_1, PV_0, S_2, PV_1, ...: S_b lands in S buffer b % 2 and P_b V_b in
+    // accumulator b % 2.  Pass 1 accumulates each accumulator over its blocks (the even
+    // and odd blocks' partial outputs); pass 2 starts a fresh one per block, once the
+    // norm warps have read the accumulator's previous block (b - 2).
+    const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV);
+    bool ok = warp_wait(&sb->q_full, 0, sb, p.err);
+    auto issue_pv = [&](int j) -> bool {
+      const int s = j & 1;
+      const uint32_t par = (j >> 1) & 1;
+      if (!warp_wait(&sb->p_full[s], par, sb, p.err)) return false;
+      if (!warp_wait(&sb->v_full[s], par, sb, p.err)) return false;
+      if (PASS == 2 && j >= 2 && !warp_wait(&sb->acc_empty[s], par ^ 1, sb, p.err)) return false;
+      tc_fence_after();
+      const uint32_t tP = tmem + C::kColS + s * 128;
+      const uint32_t tAcc = tmem + C::kColAcc + s * 128;
+      const uint32_t aVs = aV + s * C::kKVBytes;
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk) {
-          // keys [16 kk, 16 kk + 16): P_hi words at [16 kk, +8), P_lo at [16 kk + 8, +8)
-          const uint64_t bdesc = smem_desc_sw128(aVs + kk * 2048, BN * 128, 1024);
-          const bool fresh = (PASS == 2 || j == 0) && kk == 0;
-          mma_ts(tO, tP + kk * 16, bdesc, C::kIdescPV, fresh ? 0u : 1u);
-          mma_ts(tO, tP + kk * 16 + 8, bdesc, C::kIdescPV, 1u);
-        }
-        mma_commit(&sb->v_empty[s]);
-        mma_commit(&sb->pv_full);
-        return true;
-      };
-      for (int b = 0; b < nb && ok; ++b) {
-        const int s = b & 1;
-        if (!wait_or_abort(&sb->k_full[s], (b >> 1) & 1, sb, p.err)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t tS = tmem + C::kColS + s * 128;
-        const uint32_t aKs = aK + s * C::kKVBytes;
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t koff = (kk & 3) * 32;
-          const uint64_t adesc = smem_desc_sw128(aQ + (kk >> 2) * (C::M * 128) + koff, 16, 1024);
-          const uint64_t bdesc = smem_desc_sw128(aKs + (kk >> 2) * (BN * 128) + koff, 16, 1024);
-          mma_ss(tS, adesc, bdesc, C::kIdescQK, kk > 0 ? 1u : 0u);
-        }
-        mma_commit(&sb->s_full[s]);
-        mma_commit(&sb->k_empty[s]);
-        if (b > 0 && !issue_pv(b - 1)) { ok = false; break; }
+      for (int kk = 0; kk < BN / 16; ++kk) {
+        // keys [16 kk, 16 kk + 16): P_hi words at [16 kk, +8), P_lo at [16 kk + 8, +8)
+        const uint64_t bdesc = smem_desc_sw128(aVs + kk * 2048, BN * 128, 1024);
+        const bool fresh = (PASS == 2 || j < 2) && kk == 0;
+        mma_ts_warp(tAcc, tP + kk * 16, bdesc, C::kIdescPV, fresh ? 0u : 1u);
+        mma_ts_warp(tAcc, tP + kk * 16 + 8, bdesc, C::kIdescPV, 1u);
       }
-      if (ok && nb > 0) issue_pv(nb - 1);
-      mma_commit(&sb->drain);
-      mbar_wait(&sb->drain, 0, kDrainNs);
+      mma_commit_warp(&sb->v_empty[s]);
+      mma_commit_warp(&sb->acc_full[s]);
+      return true;
+    };
+    for (int b = 0; b < nb && ok; ++b) {
+      const int s = b & 1;
+      const int sk = b % C::kStagesK;
+      if (!warp_wait(&sb->k_full[sk], (b / C::kStagesK) & 1, sb, p.err)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t tS = tmem + C::kColS + s * 128;
+      const uint32_t aKs = aK + sk * C::kKVBytes;
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t koff = (kk & 3) * 32;
+        const uint64_t adesc = smem_desc_sw128(aQ + (kk >> 2) * (C::M * 128) + koff, 16, 1024);
+        const uint64_t bdesc = smem_desc_sw128(aKs + (kk >> 2) * (BN * 128) + koff, 16, 1024);
+        mma_ss_warp(tS, adesc, bdesc, C::kIdescQK, kk > 0 ? 1u : 0u);
+      }
+      mma_commit_warp(&sb->s_full[s]);
+      mma_commit_warp(&sb->k_empty[sk]);
+      if (b > 0 && !issue_pv(b - 1)) { ok = false; break; }
     }
-  } else if (warp < 4) {
-    // ============================ softmax warps ============================
-    const int r = tid;
+    if (ok && nb > 0) issue_pv(nb - 1);
+    mma_commit_warp(&sb->drain);
+    mbar_wait(&sb->drain, 0, kDrainNs);
+  } else if (PASS == 1) {
+    // ================== pass 1: two softmax warpgroups ==================
+    // Warpgroup wg (warps 4 wg .. 4 wg + 3) owns S buffer wg and accumulator wg and
+    // runs the online softmax of the blocks b = wg, wg + 2, ...; each keeps its own
+    // running max and sum.  The two partial outputs are merged at the end.
+    const int wg = warp >> 2;
+    const int r = tid & 127;                 // TMEM lane = row
     const int zl = r >> 4;
     const int j = r & 15;
     const int z = z0 + zl;
@@ -306,114 +349,135 @@ __global__ void __launch_bounds__(ScoreCfg<D, BN, PASS>::kThreads, 1)
     const int hq = g * G + (valid ? z - i * G : 0);
     const int qpos = valid ? (i + t0) * BN + j * p.sample_stride : -1;  // key position; -1: padding row
     const int64_t srow = ((int64_t)hq * p.n_tiles + i) * p.n_sample + j;  // sampled-row index
-    const uint32_t lane_off = ((uint32_t)(warp * 32) << 16);
-    const uint32_t tO = tmem + lane_off + C::kColO;
+    const uint32_t lane_off = ((uint32_t)((warp & 3) * 32) << 16);
+    const uint32_t tS = tmem + lane_off + C::kColS + wg * 128;
+    const uint32_t tAcc = tmem + lane_off + C::kColAcc + wg * 128;
     const float sl2 = p.scale_log2;
     float m_run = -INFINITY, l_run = 0.f;
-    const float lse2 = (PASS == 2 && valid) ? p.ws_lse[srow] : 0.f;
+    bool ok = true;
+    for (int b = wg; b < nb; b += 2) {
+      if (!warp_wait(&sb->s_full[wg], (b >> 1) & 1, sb, p.err)) { ok = false; break; }
+      tc_fence_after();
+      const int lim = qpos - b * BN;  // columns <= lim are visible to this query
+      const float mx = (b < i_lo) ? row_max<BN, false>(tS, lim) : row_max<BN, true>(tS, lim);
+      const float m_new = fmaxf(m_run, mx * sl2);
+      const bool grow = (m_new > m_run + 8.0f);
+      float alpha = 1.f;
+      if (grow) {
+        alpha = (m_run == -INFINITY) ? 0.f : ex2_approx(m_run - m_new);
+        m_run = m_new;
+      }
+      // S_b complete implies P V_{b-2} (issued before S_b) complete: this warpgroup's
+      // accumulator may be rescaled in place.
+      if (b >= 2 && __any_sync(0xffffffffu, grow)) {
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t ov[32];
+          tmem_ld32(tAcc + c * 32, ov);
+          tmem_ld_wait();
+          tmem_reg_fence(ov);
+#pragma unroll
+          for (int x = 0; x < 32; ++x) ov[x] = __float_as_uint(__uint_as_float(ov[x]) * alpha);
+          tmem_st32(tAcc + c * 32, ov);
+        }
+      }
+      l_run *= alpha;
+      const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
+      if (b < i_lo)
+        l_run += exp_split_store<BN, false>(tS, sl2, m_use, lim);
+      else
+        l_run += exp_split_store<BN, true>(tS, sl2, m_use, lim);
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&sb->p_full[wg]);
+    }
+    // This warpgroup's last P V: its accumulator's final phase.  The previous phase
+    // (block b - 2) completed before the last S this warpgroup saw, so the wait is at
+    // most one phase behind the barrier.
+    const int n_mine = (nb - wg + 1) / 2;
+    if (n_mine > 0 && __all_sync(0xffffffffu, ok) && !warp_wait(&sb->acc_full[wg], (n_mine - 1) & 1, sb, p.err))
+      ok = false;
+    float* sm_mB = sm_m;         // odd warpgroup's running max and sum, per row
+    float* sm_lB = sm_m + 128;
+    if (wg == 1) {
+      sm_mB[r] = m_run;
+      sm_lB[r] = l_run;
+    }
+    tc_fence_before();
+    named_barrier_sync(1, 256);
+    tc_fence_after();
+    if (wg == 0 && __all_sync(0xffffffffu, ok && !sb->abort_flag)) {
+      const bool have_b = (nb >= 2);  // accumulator 1 holds data only if there is an odd block
+      const float mB = have_b ? sm_mB[r] : -INFINITY;
+      const float lB = have_b ? sm_lB[r] : 0.f;
+      const float m = fmaxf(m_run, mB);
+      const float aA = (m_run == -INFINITY) ? 0.f : ex2_approx(m_run - m);
+      const float aB = (mB == -INFINITY) ? 0.f : ex2_approx(mB - m);
+      const float l = l_run * aA + lB * aB;
+      const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+      const float wA = aA * inv_l, wB = aB * inv_l;
+      const uint32_t tAccB = tmem + lane_off + C::kColAcc + 128;
+      float* dst = p.ws_o + srow * D;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t oa[32], ob[32];
+        tmem_ld32(tAcc + c * 32, oa);
+        if (have_b) tmem_ld32(tAccB + c * 32, ob);
+        tmem_ld_wait();
+        tmem_reg_fence(oa);
+        tmem_reg_fence(ob);
+        if (valid) {
+          float4* d4 = reinterpret_cast<float4*>(dst + c * 32);
+#pragma unroll
+          for (int x = 0; x < 8; ++x) {
+            float v4[4];
+#pragma unroll
+            for (int y = 0; y < 4; ++y) {
+              const float va = __uint_as_float(oa[4 * x + y]) * wA;
+              v4[y] = have_b ? fmaf(__uint_as_float(ob[4 * x + y]), wB, va) : va;
+            }
+            d4[x] = make_float4(v4[0], v4[1], v4[2], v4[3]);
+          }
+        }
+      }
+      if (valid) p.ws_lse[srow] = (l > 0.f) ? m + __log2f(l) : -INFINITY;
+    }
+  } else if (warp < 4) {
+    // ====================== pass 2: softmax warps 0-3 ======================
+    const int r = tid;
+    const int zl = r >> 4;
+    const int j = r & 15;
+    const int z = z0 + zl;
+    const bool valid = (z < n_groups);
+    const int i = valid ? z / G : 0;
+    const int hq = g * G + (valid ? z - i * G : 0);
+    const int qpos = valid ? (i + t0) * BN + j * p.sample_stride : -1;
+    const int64_t srow = ((int64_t)hq * p.n_tiles + i) * p.n_sample + j;
+    const uint32_t lane_off = ((uint32_t)(warp * 32) << 16);
+    const float sl2 = p.scale_log2;
+    const float lse2 = valid ? p.ws_lse[srow] : 0.f;
     bool ok = true;
     for (int b = 0; b < nb; ++b) {
       const int s = b & 1;
       const uint32_t tS = tmem + lane_off + C::kColS + s * 128;
       if (!warp_wait(&sb->s_full[s], (b >> 1) & 1, sb, p.err)) { ok = false; break; }
       tc_fence_after();
-      const int lim = qpos - b * BN;  // columns <= lim are visible to this query
-      float m_use;
-      if (PASS == 1) {
-        float mx = -INFINITY;
-        {
-          uint32_t raw[BN / 32][32];
-#pragma unroll
-          for (int c = 0; c < BN / 32; ++c) tmem_ld32(tS + c * 32, raw[c]);
-          tmem_ld_wait();
-#pragma unroll
-          for (int c = 0; c < BN / 32; ++c) tmem_reg_fence(raw[c]);
-          if (b < i_lo) {
-#pragma unroll
-            for (int c = 0; c < BN / 32; ++c)
-#pragma unroll
-              for (int x = 0; x < 32; x += 2)
-                mx = fmax3(mx, __uint_as_float(raw[c][x]), __uint_as_float(raw[c][x + 1]));
-          } else {
-#pragma unroll
-            for (int c = 0; c < BN / 32; ++c)
-#pragma unroll
-              for (int x = 0; x < 32; ++x) mx = fmaxf(mx, (c * 32 + x <= lim) ? __uint_as_float(raw[c][x]) : -INFINITY);
-          }
-        }
-        const float m_new = fmaxf(m_run, mx * sl2);
-        const bool grow = (m_new > m_run + 8.0f);
-        float alpha = 1.f;
-        if (grow) {
-          alpha = (m_run == -INFINITY) ? 0.f : ex2_approx(m_run - m_new);
-          m_run = m_new;
-        }
-        // Rescaling O needs P V_{b-1} complete (S_b may finish before it).
-        if (b > 0 && __any_sync(0xffffffffu, grow)) {
-          if (!warp_wait(&sb->pv_full, (b - 1) & 1, sb, p.err)) { ok = false; break; }
-          tc_fence_after();
-#pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t ov[32];
-            tmem_ld32(tO + c * 32, ov);
-            tmem_ld_wait();
-            tmem_reg_fence(ov);
-#pragma unroll
-            for (int x = 0; x < 32; ++x) ov[x] = __float_as_uint(__uint_as_float(ov[x]) * alpha);
-            tmem_st32(tO + c * 32, ov);
-          }
-        }
-        l_run *= alpha;
-        m_use = (m_run == -INFINITY) ? 0.f : m_run;
-      } else {
-        m_use = lse2;
-      }
-      float msum = 0.f;
-      if (b < i_lo)
-        split_chunks<BN, false>(tS, sl2, m_use, lim, &msum);
-      else
-        split_chunks<BN, true>(tS, sl2, m_use, lim, &msum);
-      if (PASS == 1) {
-        l_run += msum;
-      } else {
-        // hand m_b to the norm warps (slot s is free once block b-2's norm read it)
-        if (b >= 2 && !wait_or_abort(&sb->m_empty[s], ((b >> 1) & 1) ^ 1, sb, p.err)) ok = false;
-        sm_m[s * 128 + r] = valid ? msum : 0.f;
-        mbar_arrive(&sb->m_ready[s]);
-      }
+      const int lim = qpos - b * BN;
+      const float msum = (b < i_lo) ? exp_split_store<BN, false>(tS, sl2, lse2, lim)
+                                    : exp_split_store<BN, true>(tS, sl2, lse2, lim);
+      // hand m_b to the norm warps (slot s is free once block b-2's norm read it)
+      if (b >= 2 && !wait_or_abort(&sb->m_empty[s], ((b >> 1) & 1) ^ 1, sb, p.err)) ok = false;
+      sm_m[s * 128 + r] = valid ? msum : 0.f;
+      mbar_arrive(&sb->m_ready[s]);
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&sb->p_full[s]);
       if (!__all_sync(0xffffffffu, ok)) break;
     }
-    if (PASS == 1 && __all_sync(0xffffffffu, ok && !sb->abort_flag)) {
-      // P V_{nb-2} may still be in flight: observe its completion first, so the wait for
-      // P V_{nb-1} is never two phases behind the barrier.
-      const bool prev_ok = (nb < 2) || warp_wait(&sb->pv_full, (nb - 2) & 1, sb, p.err);
-      if (prev_ok && warp_wait(&sb->pv_full, (nb - 1) & 1, sb, p.err)) {
-        tc_fence_after();
-        const float inv_l = (l_run > 0.f) ? 1.f / l_run : 0.f;
-        float* dst = p.ws_o + srow * D;
-        uint32_t ov[D / 32][32];
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) tmem_ld32(tO + c * 32, ov[c]);
-        tmem_ld_wait();
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          tmem_reg_fence(ov[c]);
-          if (valid) {
-            float4* d4 = reinterpret_cast<float4*>(dst + c * 32);
-#pragma unroll
-            for (int x = 0; x < 8; ++x)
-              d4[x] = make_float4(__uint_as_float(ov[c][4 * x]) * inv_l, __uint_as_float(ov[c][4 * x + 1]) * inv_l,
-                                  __uint_as_float(ov[c][4 * x + 2]) * inv_l, __uint_as_float(ov[c][4 * x + 3]) * inv_l);
-          }
-        }
-        if (valid) p.ws_lse[srow] = (l_run > 0.f) ? m_run + __log2f(l_run) : -INFINITY;
-      }
-    }
-  } else if (PASS == 2) {
-    // ====================== norm warps (pass 2, warps 4-7) ======================
+  } else {
+    // ====================== pass 2: norm warps 4-7 ======================
+    // The row's dense output o (pass 1) stays in registers; per block b the
+    // accumulator b % 2 holds P_b V_b, and I_b = || P_b V_b - m_b o ||.
     const int r = tid - 128;                 // TMEM lane = row
     const int zl = r >> 4;
     const int j = r & 15;
@@ -423,59 +487,46 @@ __global__ void __launch_bounds__(ScoreCfg<D, BN, PASS>::kThreads, 1)
     const int hq = g * G + (valid ? z - i * G : 0);
     const int64_t srow = ((int64_t)hq * p.n_tiles + i) * p.n_sample + j;
     const uint32_t lane_off = ((uint32_t)((warp - 4) * 32) << 16);
-    const uint32_t tPV = tmem + lane_off + C::kColO;
-    const uint32_t tOd = tmem + lane_off + C::kColOd;
-    // the row's dense output o (pass 1) into TMEM columns [384, 384 + D)
+    float od[D];
     {
       const float4* o4 = reinterpret_cast<const float4*>(p.ws_o + srow * D);
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t w[32];
-#pragma unroll
-        for (int x = 0; x < 8; ++x) {
-          const float4 v = valid ? o4[c * 8 + x] : make_float4(0.f, 0.f, 0.f, 0.f);
-          w[4 * x] = __float_as_uint(v.x);
-          w[4 * x + 1] = __float_as_uint(v.y);
-          w[4 * x + 2] = __float_as_uint(v.z);
-          w[4 * x + 3] = __float_as_uint(v.w);
-        }
-        tmem_st32(tOd + c * 32, w);
+      for (int x = 0; x < D / 4; ++x) {
+        const float4 v = valid ? o4[x] : make_float4(0.f, 0.f, 0.f, 0.f);
+        od[4 * x] = v.x;
+        od[4 * x + 1] = v.y;
+        od[4 * x + 2] = v.z;
+        od[4 * x + 3] = v.w;
       }
-      tmem_st_wait();
     }
     const int64_t tri = row_off(p.n_tiles, t0, hq, i);
     for (int b = 0; b < nb; ++b) {
       const int s = b & 1;
-      if (!warp_wait(&sb->pv_full, b & 1, sb, p.err)) break;
-      if (!warp_wait(&sb->m_ready[s], (b >> 1) & 1, sb, p.err)) break;
+      const uint32_t par = (b >> 1) & 1;
+      if (!warp_wait(&sb->acc_full[s], par, sb, p.err)) break;
+      if (!warp_wait(&sb->m_ready[s], par, sb, p.err)) break;
       tc_fence_after();
       const float mb_row = sm_m[s * 128 + r];
       mbar_arrive(&sb->m_empty[s]);
+      const uint32_t tAcc = tmem + lane_off + C::kColAcc + s * 128;
       const uint64_t negm2 = f2_pack(-mb_row, -mb_row);
       uint64_t acc2 = f2_pack(0.f, 0.f);
 #pragma unroll
-      for (int hf = 0; hf < D / 64; ++hf) {
-        uint32_t pv[2][32], od[2][32];
-        tmem_ld32(tPV + hf * 64, pv[0]);
-        tmem_ld32(tPV + hf * 64 + 32, pv[1]);
-        tmem_ld32(tOd + hf * 64, od[0]);
-        tmem_ld32(tOd + hf * 64 + 32, od[1]);
+      for (int c = 0; c < D / 16; ++c) {
+        uint32_t pv[16];
+        tmem_ld16(tAcc + c * 16, pv);
         tmem_ld_wait();
+        tmem_reg_fence16(pv);
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          tmem_reg_fence(pv[h]);
-          tmem_reg_fence(od[h]);
-#pragma unroll
-          for (int x = 0; x < 32; x += 2) {
-            const uint64_t e = f2_fma(negm2, f2_pack(__uint_as_float(od[h][x]), __uint_as_float(od[h][x + 1])),
-                                      f2_pack(__uint_as_float(pv[h][x]), __uint_as_float(pv[h][x + 1])));
-            acc2 = f2_fma(e, e, acc2);
-          }
+        for (int x = 0; x < 16; x += 2) {
+          const uint64_t e = f2_fma(negm2, f2_pack(od[c * 16 + x], od[c * 16 + x + 1]),
+                                    f2_pack(__uint_as_float(pv[x]), __uint_as_float(pv[x + 1])));
+          acc2 = f2_fma(e, e, acc2);
         }
       }
-      // P V_b has been read: the accumulator may be reused for block b+1.
+      // P V_b has been read: the accumulator may take block b + 2.
       tc_fence_before();
-      mbar_arrive(&sb->pv_empty);
+      mbar_arrive(&sb->acc_empty[s]);
       float a0, a1;
       f2_unpack(acc2, a0, a1);
       float Ib = valid ? sqrtf(a0 + a1) : 0.f;
