@@ -31,12 +31,19 @@ from dataclasses import dataclass
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libpoem.so")
+# POEM_LIBRARY_VARIANT=checks selects the debug build (device bounds checks,
+# libpoem_checks.so from build.py's "checks" variant); there is no other choice and
+# no fallback: a missing library fails the import.
+_VARIANT = os.environ.get("POEM_LIBRARY_VARIANT", "release")
+if _VARIANT not in ("release", "checks"):
+    raise ImportError(f"POEM_LIBRARY_VARIANT must be 'release' or 'checks', not {_VARIANT!r}")
+LIB_PATH = os.path.join(_HERE, "libpoem.so" if _VARIANT == "release" else "libpoem_checks.so")
 
 POEM_OK = 0
 STATUS = {
     0: "POEM_OK", 1: "POEM_ERR_INVALID_ARG", 2: "POEM_ERR_UNSUPPORTED", 3: "POEM_ERR_CUDA",
     4: "POEM_ERR_TIMEOUT", 5: "POEM_ERR_CAPACITY", 6: "POEM_ERR_WORKSPACE", 7: "POEM_ERR_BAD_LIST",
+    8: "POEM_ERR_BOUNDS",
 }
 
 EXPORTED = (
@@ -66,7 +73,7 @@ class Shape(ctypes.Structure):
 
 def _load():
     if not os.path.exists(LIB_PATH):
-        raise ImportError(f"libpoem.so not built at {LIB_PATH}; run block_sparse_attention_poem_b200/build.py")
+        raise ImportError(f"{os.path.basename(LIB_PATH)} not built at {LIB_PATH}; run block_sparse_attention_poem_b200/build.py")
     lib = ctypes.CDLL(LIB_PATH)
     vp, sp, i64, sz = ctypes.c_void_p, ctypes.POINTER(Shape), ctypes.c_int64, ctypes.c_size_t
     st = ctypes.c_int

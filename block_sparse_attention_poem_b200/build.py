@@ -1,4 +1,9 @@
-"""Build libpoem.so (the CUDA library behind include/poem.h) in-tree for sm_100a."""
+"""Build libpoem.so (the CUDA library behind include/poem.h) in-tree for sm_100a.
+
+variant="checks" builds libpoem_checks.so, the same sources compiled with
+-DPOEM_CHECKS: device-side bounds checks that skip an out-of-range access and
+report POEM_ERR_BOUNDS through poem_check.  The binding loads it when the
+environment variable POEM_LIBRARY_VARIANT is "checks"."""
 from __future__ import annotations
 
 import os
@@ -9,8 +14,9 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libpoem.so")
-SOURCES = ["poem_api.cu", "bsa_fwd.cu", "bsa_fwd_grouped.cu", "poem_score.cu", "poem_select.cu", "poem_select_noalloc.cu", "poem_pooled.cu"]
-HEADERS = ["sm100.cuh", "common.cuh", "fwd_common.cuh"]
+LIBS = {"release": LIB, "checks": os.path.join(PKG, "libpoem_checks.so")}
+SOURCES = ["poem_api.cu", "bsa_fwd.cu", "bsa_fwd_grouped.cu", "poem_score.cu", "poem_score_pass1.cu", "poem_select.cu", "poem_select_noalloc.cu", "poem_pooled.cu"]
+HEADERS = ["sm100.cuh", "common.cuh", "fwd_common.cuh", "score_common.cuh"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -19,24 +25,27 @@ FLAGS = [
 ]
 
 
-def _stale() -> bool:
-    if not os.path.exists(LIB):
+def _stale(lib: str) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     deps = [os.path.join(CSRC, f) for f in SOURCES + HEADERS] + [os.path.join(ROOT, "include", "poem.h")]
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if force or _stale():
+def build(force: bool = False, verbose: bool = False, variant: str = "release") -> str:
+    lib = LIBS[variant]
+    if force or _stale(lib):
         cmd = [NVCC, *FLAGS]
+        if variant == "checks":
+            cmd += ["-DPOEM_CHECKS"]
         if verbose:
             cmd += ["-Xptxas", "-v"]
-        cmd += ["-o", LIB] + [os.path.join(CSRC, f) for f in SOURCES]
+        cmd += ["-o", lib] + [os.path.join(CSRC, f) for f in SOURCES]
         subprocess.run(cmd, check=True)
-    return LIB
+    return lib
 
 
 if __name__ == "__main__":
-    build(force=True, verbose="-v" in sys.argv)
-    print(LIB)
+    v = "checks" if "--checks" in sys.argv else "release"
+    print(build(force=True, verbose="-v" in sys.argv, variant=v))

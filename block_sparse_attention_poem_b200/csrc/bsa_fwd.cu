@@ -99,8 +99,8 @@ __global__ void __launch_bounds__(kThreadsFwd, 2)
     mbar_init(&sb->v_full, 1);
     mbar_init(&sb->v_empty, 1);
     mbar_init(&sb->s_full, 1);
-    mbar_init(&sb->p_half[0], 128);
-    mbar_init(&sb->p_half[1], 128);
+    mbar_init(&sb->p_half[0], 4);  // one arrival per softmax warp
+    mbar_init(&sb->p_half[1], 4);
     mbar_init(&sb->o_full, 1);
     mbar_init(&sb->drain, 1);
     sb->abort_flag = 0;

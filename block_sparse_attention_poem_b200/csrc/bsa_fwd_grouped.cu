@@ -144,8 +144,8 @@ __global__ void __launch_bounds__(kThreadsGrouped, 1)
     for (int x = 0; x < 2; ++x) {
       mbar_init(&sb->q_full[x], 1);
       mbar_init(&sb->s_full[x], 1);
-      mbar_init(&sb->p_half[x][0], 128);
-      mbar_init(&sb->p_half[x][1], 128);
+      mbar_init(&sb->p_half[x][0], 4);  // one arrival per softmax warp
+      mbar_init(&sb->p_half[x][1], 4);
       mbar_init(&sb->o_full[x], 1);
     }
     mbar_init(&sb->drain, 1);

@@ -95,6 +95,7 @@ struct ScoreParams {
   int sample_stride;   // B / S
   float scale_log2;
   DevErr err;
+  int64_t n_entries;     // entries of I_hat / m_hat (bounds of the debug build)
 };
 
 struct SelectParams {
@@ -122,6 +123,7 @@ struct SelectParams {
   double rho;    // stage-1 shortlist fraction of the candidates
   int practical;
   DevErr err;
+  int64_t n_entries;  // entries of the per-row scratch (bounds of the debug build)
 };
 
 // Mean pooling and pooled score estimates for the practical selector.
@@ -157,6 +159,8 @@ cudaError_t launch_bsa_fwd_grouped(int head_dim, int block, const CUtensorMap& t
                                    const CUtensorMap& tmV, const FwdParams& p, int n_kv_heads, cudaStream_t stream);
 cudaError_t launch_score(int head_dim, int block, const CUtensorMap& tmQs, const CUtensorMap& tmK,
                          const CUtensorMap& tmV, const ScoreParams& p, cudaStream_t stream);
+cudaError_t launch_score_pass1(int head_dim, int block, const CUtensorMap& tmQs, const CUtensorMap& tmK,
+                               const CUtensorMap& tmV, const ScoreParams& p, int grid, cudaStream_t stream);
 cudaError_t launch_select(const SelectParams& p, cudaStream_t stream);
 cudaError_t launch_pooled(int head_dim, PoolParams p, cudaStream_t stream);
 

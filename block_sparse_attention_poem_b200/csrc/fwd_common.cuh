@@ -69,7 +69,7 @@ __device__ __forceinline__ void exp_pack_store(uint32_t tS, float sl2, float m_u
     // this half of P (and any O rescale before it) is in TMEM: its P V MMAs may start
     tmem_st_wait();
     tc_fence_before();
-    mbar_arrive(&p_half[hf]);
+    warp_arrive(&p_half[hf]);
   }
   float a0, a1;
   f2_unpack(acc, a0, a1);

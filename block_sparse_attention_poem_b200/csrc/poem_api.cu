@@ -76,6 +76,8 @@ size_t tri_entries(const poem_shape* s, const Layout& L) {
   return (size_t)s->n_q_heads * (size_t)poem::row_entries(L.T, L.t0);
 }
 
+// Score workspace: header (error word), then the dense outputs o [rows, D] fp32 and
+// the log-sum-exps [rows] of the sampled queries (pass 1 -> pass 2).
 size_t score_ws_bytes(const poem_shape* s, int T) {
   const size_t rows = (size_t)s->n_q_heads * T * s->n_sample;
   return poem::kWsHeader + round_up(rows * s->head_dim * sizeof(float), 256) + round_up(rows * sizeof(float), 256);
@@ -189,11 +191,13 @@ poem_status poem_score(const poem_shape* shape, const poem_bf16* q, const poem_b
     return st;
   const size_t rows = (size_t)shape->n_q_heads * L.T * shape->n_sample;
   uint8_t* base = reinterpret_cast<uint8_t*>(ws);
+  const size_t off_o = poem::kWsHeader;
+  const size_t off_lse = off_o + round_up(rows * shape->head_dim * sizeof(float), 256);
   poem::ScoreParams p{};
   p.I_hat = I_hat;
   p.m_hat = m_hat;
-  p.ws_o = reinterpret_cast<float*>(base + poem::kWsHeader);
-  p.ws_lse = reinterpret_cast<float*>(base + poem::kWsHeader + round_up(rows * shape->head_dim * sizeof(float), 256));
+  p.ws_o = reinterpret_cast<float*>(base + off_o);
+  p.ws_lse = reinterpret_cast<float*>(base + off_lse);
   p.n_tokens = shape->n_tokens;
   p.n_q_heads = shape->n_q_heads;
   p.n_kv_heads = shape->n_kv_heads;
@@ -204,6 +208,7 @@ poem_status poem_score(const poem_shape* shape, const poem_bf16* q, const poem_b
   p.sample_stride = shape->block / shape->n_sample;
   p.scale_log2 = L.scale * poem::kLog2e;
   p.err = dev_err(ws);
+  p.n_entries = (int64_t)tri_entries(shape, L);
   cudaError_t e = poem::launch_score(shape->head_dim, shape->block, tmQs, tmK, tmV, p, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "poem_score launch");
   return POEM_OK;
@@ -265,6 +270,7 @@ static poem_status select_common(const poem_shape* shape, const float* I_hat, co
     p.rho = practical->rho;
   }
   p.err = dev_err(ws);
+  p.n_entries = (int64_t)tri_entries(shape, L);
   cudaError_t e = poem::launch_select(p, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "poem_select launch");
   return POEM_OK;
@@ -454,6 +460,8 @@ poem_status poem_check(void* stream, void* ws) {
   if (word & poem::kErrBadList) return POEM_ERR_BAD_LIST;
   if (word & poem::kErrCapacity) return POEM_ERR_CAPACITY;
   if (word & poem::kErrBadParam) return POEM_ERR_INVALID_ARG;
+  if (word & poem::kErrBounds)
+    return arg_fail(POEM_ERR_BOUNDS, "a device bounds check of the debug build failed (the access was skipped)");
   return POEM_OK;
 }
 
@@ -469,6 +477,7 @@ const char* poem_status_string(poem_status s) {
     case POEM_ERR_CAPACITY: return "POEM_ERR_CAPACITY";
     case POEM_ERR_WORKSPACE: return "POEM_ERR_WORKSPACE";
     case POEM_ERR_BAD_LIST: return "POEM_ERR_BAD_LIST";
+    case POEM_ERR_BOUNDS: return "POEM_ERR_BOUNDS";
   }
   return "POEM_ERR_UNKNOWN";
 }

@@ -9,10 +9,12 @@
 // and max-aggregated:  I_hat[h, i, b] = max_j I_b(q_j),  m_hat likewise.
 //
 // Two passes over the key blocks, both on the tensor cores:
-//   pass 1: dense causal attention of the sampled queries -> o (fp32) and the
-//           log-sum-exp of their scaled logits (log2 units) in the workspace.
-//   pass 2: recompute S, form the exact normalised p = 2^(s log2e scale - lse),
-//           per block r_b = P_b V_b - m_b o and its norm, max over the 16 queries.
+//   pass 1 (poem_score_pass1.cu): dense causal attention of the sampled queries ->
+//           o (fp32) and the log-sum-exp of their scaled logits (log2 units) in the
+//           workspace.
+//   pass 2 (this file): recompute S, form the exact normalised
+//           p = 2^(s log2e scale - lse), per block r_b = P_b V_b - m_b o and its norm,
+//           max over the 16 queries.
 //
 // Packing: one CTA owns 8 groups of 16 sampled queries that share a KV head --
 // groups are enumerated per KV head in (tile, query head) order, so a CTA covers
@@ -23,18 +25,15 @@
 // q_tile0 + i: its sampled queries sit at key positions (q_tile0 + i) B + j (B / S)
 // and its score row has q_tile0 + i + 1 entries (row_off layout).
 //
-// Pipeline (one CTA per SM, TMEM fully allocated):
+// Pass 2 pipeline (one CTA per SM, TMEM fully allocated):
 //   TMEM  S0 [0,128)  S1 [128,256)  -- S double-buffered: S_{b+1} is computed while
 //                                      the softmax of block b runs
 //         accumulators [256,384) and [384,512): P_b V_b of block b goes to
-//         accumulator b % 2 -- pass 1: the even and the odd blocks' partial outputs;
-//         pass 2: P_b V_b of one block, double-buffered for the norm warps
+//         accumulator b % 2, double-buffered for the norm warps
 //   smem  Q tile, 3-stage K ring, 2-stage V ring (192 KB at d = 128)
-//   pass 1: warps 0-3 and 4-7 are two softmax warpgroups, one for the even and one
-//           for the odd blocks, each with its own running max and sum (merged at
-//           the end); pass 2: warps 0-3 softmax, warps 4-7 the norm of
-//           P_b V_b - m_b o with o held in registers.  Warp 8 issues TMA loads;
-//           warp 9 issues the MMAs, converged, from one elected lane.
+//   warps 0-3 softmax, warps 4-7 the norm of P_b V_b - m_b o with o held in
+//   registers; warp 8 issues TMA loads; warp 9 issues the MMAs, converged, from one
+//   elected lane.
 //   MMA order: S_0, S_1, PV_0, S_2, PV_1, ...
 //
 // Precision: P enters the P V contraction as a hi/lo pair of bf16 matrices
@@ -46,11 +45,12 @@
 // wait's completion is a precondition of the barrier's next phase), so parity
 // waits cannot alias.
 #include "common.cuh"
+#include "score_common.cuh"
 
 namespace poem {
 namespace {
 
-template <int D, int BN, int PASS>
+template <int D, int BN>
 struct ScoreCfg {
   static constexpr int M = 128;
   static constexpr int kGroups = 8;        // groups of 16 sampled queries per CTA
@@ -64,14 +64,13 @@ struct ScoreCfg {
   static constexpr int kOffK = kOffQ + kQBytes;
   static constexpr int kOffV = kOffK + kStagesK * kKVBytes;
   static constexpr int kOffBar = kOffV + kStagesV * kKVBytes;
-  static constexpr int kOffM = kOffBar + 256;                 // [2][128] floats: m_b hand-off (pass 2)
-                                                              // or the odd warpgroup's max / sum (pass 1)
+  static constexpr int kOffM = kOffBar + 256;                 // [2][128] floats: m_b hand-off
   // at least 120 KB so that one CTA (holding all 512 TMEM columns) occupies an SM
   static constexpr int kSmemBytes = (kOffM + 2 * 128 * 4 + 1024) > 122880 ? (kOffM + 2 * 128 * 4 + 1024) : 122880;
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kColS = 0;     // S buffer s at [128 s, 128 s + BN)
   static constexpr uint32_t kColAcc = 256; // accumulator s at [256 + 128 s, 256 + 128 s + D)
-  static constexpr int kWarpProd = 8;      // warps 0-7 compute, 8 TMA, 9 MMA
+  static constexpr int kWarpProd = 8;      // warps 0-3 softmax, 4-7 norm, 8 TMA, 9 MMA
   static constexpr int kWarpMma = 9;
   static constexpr int kThreads = 320;
   static constexpr uint32_t kIdescQK = idesc_bf16_f32(M, BN, 0);
@@ -118,85 +117,14 @@ __device__ __forceinline__ void score_cta_coords(int cta, int ctas_per_g, int& g
   z0 = c * 8;
 }
 
-// p = 2^(s * scale * log2e - m) for one row's BN scores (re-read from TMEM in 64-column
-// halves; masked columns > lim exactly 0 when MASKED), written back over S as
-// interleaved bf16 P_hi / P_lo words (per 16-key k-step: 8 words P_hi, then 8 words
-// P_lo = p - P_hi rounded to bf16).  Returns sum p.  (Summing the unrounded p instead
-// of P_hi + P_lo changes the sum by an unbiased ~2^-18 relative error per weight.)
-template <int BN, bool MASKED>
-__device__ __forceinline__ float exp_split_store(uint32_t tS, float sl2, float m_use, int lim) {
-  const uint64_t scale2 = f2_pack(sl2, sl2);
-  const uint64_t negm2 = f2_pack(-m_use, -m_use);
-  uint64_t acc = f2_pack(0.f, 0.f);
-#pragma unroll
-  for (int cp = 0; cp < BN / 64; ++cp) {
-    uint32_t a[2][32];
-    tmem_ld32(tS + cp * 64, a[0]);
-    tmem_ld32(tS + cp * 64 + 32, a[1]);
-    tmem_ld_wait();
-    tmem_reg_fence(a[0]);
-    tmem_reg_fence(a[1]);
-#pragma unroll
-    for (int ks = 0; ks < 4; ++ks) {  // the four 16-key k-steps of this half
-      const uint32_t* src = a[ks >> 1] + (ks & 1) * 16;
-      uint32_t out[16];
-#pragma unroll
-      for (int x = 0; x < 8; ++x) {
-        const int col = cp * 64 + ks * 16 + 2 * x;
-        const uint64_t xv = f2_fma(f2_pack(__uint_as_float(src[2 * x]), __uint_as_float(src[2 * x + 1])), scale2, negm2);
-        float x0, x1;
-        f2_unpack(xv, x0, x1);
-        float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
-        if (MASKED) {
-          if (col > lim) p0 = 0.f;
-          if (col + 1 > lim) p1 = 0.f;
-        }
-        acc = f2_add(acc, f2_pack(p0, p1));
-        const uint32_t wh = pack_bf16x2(p0, p1);
-        out[x] = wh;
-        out[8 + x] = pack_bf16x2(p0 - bf16lo_to_f32(wh), p1 - bf16hi_to_f32(wh));
-      }
-      tmem_st16(tS + cp * 64 + ks * 16, out);
-    }
-  }
-  float a0, a1;
-  f2_unpack(acc, a0, a1);
-  return a0 + a1;
-}
+using score::exp_split_store;
+using score::row_max;
 
-// Maximum of one row's visible scores (columns <= lim when MASKED), read in 64-column halves.
-template <int BN, bool MASKED>
-__device__ __forceinline__ float row_max(uint32_t tS, int lim) {
-  float mx[2] = {-INFINITY, -INFINITY};
-#pragma unroll
-  for (int cp = 0; cp < BN / 64; ++cp) {
-    uint32_t a[2][32];
-    tmem_ld32(tS + cp * 64, a[0]);
-    tmem_ld32(tS + cp * 64 + 32, a[1]);
-    tmem_ld_wait();
-    tmem_reg_fence(a[0]);
-    tmem_reg_fence(a[1]);
-#pragma unroll
-    for (int h = 0; h < 2; ++h)
-#pragma unroll
-      for (int x = 0; x < 32; x += 2) {
-        if (MASKED) {
-          const int col = cp * 64 + h * 32 + x;
-          mx[h] = fmax3(mx[h], (col <= lim) ? __uint_as_float(a[h][x]) : -INFINITY,
-                        (col + 1 <= lim) ? __uint_as_float(a[h][x + 1]) : -INFINITY);
-        } else {
-          mx[h] = fmax3(mx[h], __uint_as_float(a[h][x]), __uint_as_float(a[h][x + 1]));
-        }
-      }
-  }
-  return fmaxf(mx[0], mx[1]);
-}
-
-template <int D, int BN, int PASS>
-__global__ void __launch_bounds__(ScoreCfg<D, BN, PASS>::kThreads, 1)
-    poem_score_kernel(const __grid_constant__ CUtensorMap tmQs, const __grid_constant__ CUtensorMap tmK,
+template <int D, int BN>
+__global__ void __launch_bounds__(ScoreCfg<D, BN>::kThreads, 1)
+    poem_score_pass2_kernel(const __grid_constant__ CUtensorMap tmQs, const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV, const ScoreParams p) {
-  using C = ScoreCfg<D, BN, PASS>;
+  using C = ScoreCfg<D, BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem + C::kOffQ;
@@ -228,11 +156,11 @@ __global__ void __launch_bounds__(ScoreCfg<D, BN, PASS>::kThreads, 1)
       mbar_init(&sb->v_full[s], 1);
       mbar_init(&sb->v_empty[s], 1);
       mbar_init(&sb->s_full[s], 1);
-      mbar_init(&sb->p_full[s], 128);
+      mbar_init(&sb->p_full[s], 4);  // barriers signalled by 4 warps: one arrival per warp
       mbar_init(&sb->acc_full[s], 1);
-      mbar_init(&sb->acc_empty[s], 128);
-      mbar_init(&sb->m_ready[s], 128);
-      mbar_init(&sb->m_empty[s], 128);
+      mbar_init(&sb->acc_empty[s], 4);
+      mbar_init(&sb->m_ready[s], 4);
+      mbar_init(&sb->m_empty[s], 4);
     }
     mbar_init(&sb->drain, 1);
     sb->abort_flag = 0;
@@ -286,9 +214,8 @@ __global__ void __launch_bounds__(ScoreCfg<D, BN, PASS>::kThreads, 1)
     // The whole warp runs this loop converged (waits and operands are warp-uniform);
     // one elected lane issues each MMA and commit.
     // Order S_0, S_1, PV_0, S_2, PV_1, ...: S_b lands in S buffer b % 2 and P_b V_b in
-    // accumulator b % 2.  Pass 1 accumulates each accumulator over its blocks (the even
-    // and odd blocks' partial outputs); pass 2 starts a fresh one per block, once the
-    // norm warps have read the accumulator's previous block (b - 2).
+    // accumulator b % 2, started fresh once the norm warps have read the accumulator's
+    // previous block (b - 2).
     const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV);
     bool ok = warp_wait(&sb->q_full, 0, sb, p.err);
     auto issue_pv = [&](int j) -> bool {
@@ -296,7 +223,7 @@ __global__ void __launch_bounds__(ScoreCfg<D, BN, PASS>::kThreads, 1)
       const uint32_t par = (j >> 1) & 1;
       if (!warp_wait(&sb->p_full[s], par, sb, p.err)) return false;
       if (!warp_wait(&sb->v_full[s], par, sb, p.err)) return false;
-      if (PASS == 2 && j >= 2 && !warp_wait(&sb->acc_empty[s], par ^ 1, sb, p.err)) return false;
+      if (j >= 2 && !warp_wait(&sb->acc_empty[s], par ^ 1, sb, p.err)) return false;
       tc_fence_after();
       const uint32_t tP = tmem + C::kColS + s * 128;
       const uint32_t tAcc = tmem + C::kColAcc + s * 128;
@@ -305,8 +232,7 @@ __global__ void __launch_bounds__(ScoreCfg<D, BN, PASS>::kThreads, 1)
       for (int kk = 0; kk < BN / 16; ++kk) {
         // keys [16 kk, 16 kk + 16): P_hi words at [16 kk, +8), P_lo at [16 kk + 8, +8)
         const uint64_t bdesc = smem_desc_sw128(aVs + kk * 2048, BN * 128, 1024);
-        const bool fresh = (PASS == 2 || j < 2) && kk == 0;
-        mma_ts_warp(tAcc, tP + kk * 16, bdesc, C::kIdescPV, fresh ? 0u : 1u);
+        mma_ts_warp(tAcc, tP + kk * 16, bdesc, C::kIdescPV, kk > 0 ? 1u : 0u);
         mma_ts_warp(tAcc, tP + kk * 16 + 8, bdesc, C::kIdescPV, 1u);
       }
       mma_commit_warp(&sb->v_empty[s]);
@@ -334,114 +260,6 @@ __global__ void __launch_bounds__(ScoreCfg<D, BN, PASS>::kThreads, 1)
     if (ok && nb > 0) issue_pv(nb - 1);
     mma_commit_warp(&sb->drain);
     mbar_wait(&sb->drain, 0, kDrainNs);
-  } else if (PASS == 1) {
-    // ================== pass 1: two softmax warpgroups ==================
-    // Warpgroup wg (warps 4 wg .. 4 wg + 3) owns S buffer wg and accumulator wg and
-    // runs the online softmax of the blocks b = wg, wg + 2, ...; each keeps its own
-    // running max and sum.  The two partial outputs are merged at the end.
-    const int wg = warp >> 2;
-    const int r = tid & 127;                 // TMEM lane = row
-    const int zl = r >> 4;
-    const int j = r & 15;
-    const int z = z0 + zl;
-    const bool valid = (z < n_groups);
-    const int i = valid ? z / G : 0;
-    const int hq = g * G + (valid ? z - i * G : 0);
-    const int qpos = valid ? (i + t0) * BN + j * p.sample_stride : -1;  // key position; -1: padding row
-    const int64_t srow = ((int64_t)hq * p.n_tiles + i) * p.n_sample + j;  // sampled-row index
-    const uint32_t lane_off = ((uint32_t)((warp & 3) * 32) << 16);
-    const uint32_t tS = tmem + lane_off + C::kColS + wg * 128;
-    const uint32_t tAcc = tmem + lane_off + C::kColAcc + wg * 128;
-    const float sl2 = p.scale_log2;
-    float m_run = -INFINITY, l_run = 0.f;
-    bool ok = true;
-    for (int b = wg; b < nb; b += 2) {
-      if (!warp_wait(&sb->s_full[wg], (b >> 1) & 1, sb, p.err)) { ok = false; break; }
-      tc_fence_after();
-      const int lim = qpos - b * BN;  // columns <= lim are visible to this query
-      const float mx = (b < i_lo) ? row_max<BN, false>(tS, lim) : row_max<BN, true>(tS, lim);
-      const float m_new = fmaxf(m_run, mx * sl2);
-      const bool grow = (m_new > m_run + 8.0f);
-      float alpha = 1.f;
-      if (grow) {
-        alpha = (m_run == -INFINITY) ? 0.f : ex2_approx(m_run - m_new);
-        m_run = m_new;
-      }
-      // S_b complete implies P V_{b-2} (issued before S_b) complete: this warpgroup's
-      // accumulator may be rescaled in place.
-      if (b >= 2 && __any_sync(0xffffffffu, grow)) {
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t ov[32];
-          tmem_ld32(tAcc + c * 32, ov);
-          tmem_ld_wait();
-          tmem_reg_fence(ov);
-#pragma unroll
-          for (int x = 0; x < 32; ++x) ov[x] = __float_as_uint(__uint_as_float(ov[x]) * alpha);
-          tmem_st32(tAcc + c * 32, ov);
-        }
-      }
-      l_run *= alpha;
-      const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
-      if (b < i_lo)
-        l_run += exp_split_store<BN, false>(tS, sl2, m_use, lim);
-      else
-        l_run += exp_split_store<BN, true>(tS, sl2, m_use, lim);
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(&sb->p_full[wg]);
-    }
-    // This warpgroup's last P V: its accumulator's final phase.  The previous phase
-    // (block b - 2) completed before the last S this warpgroup saw, so the wait is at
-    // most one phase behind the barrier.
-    const int n_mine = (nb - wg + 1) / 2;
-    if (n_mine > 0 && __all_sync(0xffffffffu, ok) && !warp_wait(&sb->acc_full[wg], (n_mine - 1) & 1, sb, p.err))
-      ok = false;
-    float* sm_mB = sm_m;         // odd warpgroup's running max and sum, per row
-    float* sm_lB = sm_m + 128;
-    if (wg == 1) {
-      sm_mB[r] = m_run;
-      sm_lB[r] = l_run;
-    }
-    tc_fence_before();
-    named_barrier_sync(1, 256);
-    tc_fence_after();
-    if (wg == 0 && __all_sync(0xffffffffu, ok && !sb->abort_flag)) {
-      const bool have_b = (nb >= 2);  // accumulator 1 holds data only if there is an odd block
-      const float mB = have_b ? sm_mB[r] : -INFINITY;
-      const float lB = have_b ? sm_lB[r] : 0.f;
-      const float m = fmaxf(m_run, mB);
-      const float aA = (m_run == -INFINITY) ? 0.f : ex2_approx(m_run - m);
-      const float aB = (mB == -INFINITY) ? 0.f : ex2_approx(mB - m);
-      const float l = l_run * aA + lB * aB;
-      const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
-      const float wA = aA * inv_l, wB = aB * inv_l;
-      const uint32_t tAccB = tmem + lane_off + C::kColAcc + 128;
-      float* dst = p.ws_o + srow * D;
-#pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t oa[32], ob[32];
-        tmem_ld32(tAcc + c * 32, oa);
-        if (have_b) tmem_ld32(tAccB + c * 32, ob);
-        tmem_ld_wait();
-        tmem_reg_fence(oa);
-        tmem_reg_fence(ob);
-        if (valid) {
-          float4* d4 = reinterpret_cast<float4*>(dst + c * 32);
-#pragma unroll
-          for (int x = 0; x < 8; ++x) {
-            float v4[4];
-#pragma unroll
-            for (int y = 0; y < 4; ++y) {
-              const float va = __uint_as_float(oa[4 * x + y]) * wA;
-              v4[y] = have_b ? fmaf(__uint_as_float(ob[4 * x + y]), wB, va) : va;
-            }
-            d4[x] = make_float4(v4[0], v4[1], v4[2], v4[3]);
-          }
-        }
-      }
-      if (valid) p.ws_lse[srow] = (l > 0.f) ? m + __log2f(l) : -INFINITY;
-    }
   } else if (warp < 4) {
     // ====================== pass 2: softmax warps 0-3 ======================
     const int r = tid;
@@ -455,7 +273,8 @@ __global__ void __launch_bounds__(ScoreCfg<D, BN, PASS>::kThreads, 1)
     const int64_t srow = ((int64_t)hq * p.n_tiles + i) * p.n_sample + j;
     const uint32_t lane_off = ((uint32_t)(warp * 32) << 16);
     const float sl2 = p.scale_log2;
-    const float lse2 = valid ? p.ws_lse[srow] : 0.f;
+    const bool in_ws = POEM_IN_BOUNDS(p.err, srow, (int64_t)p.n_q_heads * p.n_tiles * p.n_sample);
+    const float lse2 = (valid && in_ws) ? p.ws_lse[srow] : 0.f;
     bool ok = true;
     for (int b = 0; b < nb; ++b) {
       const int s = b & 1;
@@ -466,12 +285,12 @@ __global__ void __launch_bounds__(ScoreCfg<D, BN, PASS>::kThreads, 1)
       const float msum = (b < i_lo) ? exp_split_store<BN, false>(tS, sl2, lse2, lim)
                                     : exp_split_store<BN, true>(tS, sl2, lse2, lim);
       // hand m_b to the norm warps (slot s is free once block b-2's norm read it)
-      if (b >= 2 && !wait_or_abort(&sb->m_empty[s], ((b >> 1) & 1) ^ 1, sb, p.err)) ok = false;
+      if (b >= 2 && !warp_wait(&sb->m_empty[s], ((b >> 1) & 1) ^ 1, sb, p.err)) ok = false;
       sm_m[s * 128 + r] = valid ? msum : 0.f;
-      mbar_arrive(&sb->m_ready[s]);
+      warp_arrive(&sb->m_ready[s]);
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(&sb->p_full[s]);
+      warp_arrive(&sb->p_full[s]);
       if (!__all_sync(0xffffffffu, ok)) break;
     }
   } else {
@@ -490,9 +309,10 @@ __global__ void __launch_bounds__(ScoreCfg<D, BN, PASS>::kThreads, 1)
     float od[D];
     {
       const float4* o4 = reinterpret_cast<const float4*>(p.ws_o + srow * D);
+      const bool in_ws = POEM_IN_BOUNDS(p.err, srow, (int64_t)p.n_q_heads * p.n_tiles * p.n_sample);
 #pragma unroll
       for (int x = 0; x < D / 4; ++x) {
-        const float4 v = valid ? o4[x] : make_float4(0.f, 0.f, 0.f, 0.f);
+        const float4 v = (valid && in_ws) ? o4[x] : make_float4(0.f, 0.f, 0.f, 0.f);
         od[4 * x] = v.x;
         od[4 * x + 1] = v.y;
         od[4 * x + 2] = v.z;
@@ -507,7 +327,7 @@ __global__ void __launch_bounds__(ScoreCfg<D, BN, PASS>::kThreads, 1)
       if (!warp_wait(&sb->m_ready[s], par, sb, p.err)) break;
       tc_fence_after();
       const float mb_row = sm_m[s * 128 + r];
-      mbar_arrive(&sb->m_empty[s]);
+      warp_arrive(&sb->m_empty[s]);
       const uint32_t tAcc = tmem + lane_off + C::kColAcc + s * 128;
       const uint64_t negm2 = f2_pack(-mb_row, -mb_row);
       uint64_t acc2 = f2_pack(0.f, 0.f);
@@ -526,7 +346,7 @@ __global__ void __launch_bounds__(ScoreCfg<D, BN, PASS>::kThreads, 1)
       }
       // P V_b has been read: the accumulator may take block b + 2.
       tc_fence_before();
-      mbar_arrive(&sb->acc_empty[s]);
+      warp_arrive(&sb->acc_empty[s]);
       float a0, a1;
       f2_unpack(acc2, a0, a1);
       float Ib = valid ? sqrtf(a0 + a1) : 0.f;
@@ -536,7 +356,7 @@ __global__ void __launch_bounds__(ScoreCfg<D, BN, PASS>::kThreads, 1)
         Ib = fmaxf(Ib, __shfl_xor_sync(0xffffffffu, Ib, off));
         mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, off));
       }
-      if (j == 0 && valid && b <= i + t0) {
+      if (j == 0 && valid && b <= i + t0 && POEM_IN_BOUNDS(p.err, tri + b, p.n_entries)) {
         p.I_hat[tri + b] = Ib;
         p.m_hat[tri + b] = mb;
       }
@@ -552,24 +372,25 @@ __global__ void __launch_bounds__(ScoreCfg<D, BN, PASS>::kThreads, 1)
   }
 }
 
-template <int D, int BN, int PASS>
-cudaError_t launch_pass(const CUtensorMap& tmQs, const CUtensorMap& tmK, const CUtensorMap& tmV,
-                        const ScoreParams& p, int grid, cudaStream_t stream) {
-  using C = ScoreCfg<D, BN, PASS>;
-  cudaError_t e = ensure_smem_limit(poem_score_kernel<D, BN, PASS>, C::kSmemBytes);
+template <int D, int BN>
+cudaError_t launch_pass2(const CUtensorMap& tmQs, const CUtensorMap& tmK, const CUtensorMap& tmV,
+                         const ScoreParams& p, int grid, cudaStream_t stream) {
+  using C = ScoreCfg<D, BN>;
+  cudaError_t e = ensure_smem_limit(poem_score_pass2_kernel<D, BN>, C::kSmemBytes);
   if (e != cudaSuccess) return e;
-  poem_score_kernel<D, BN, PASS><<<grid, C::kThreads, C::kSmemBytes, stream>>>(tmQs, tmK, tmV, p);
+  poem_score_pass2_kernel<D, BN><<<grid, C::kThreads, C::kSmemBytes, stream>>>(tmQs, tmK, tmV, p);
   return cudaGetLastError();
 }
 
+// Pass 1 (poem_score_pass1.cu: o and lse of the sampled queries), then pass 2.
 template <int D, int BN>
 cudaError_t launch_score_t(const CUtensorMap& tmQs, const CUtensorMap& tmK, const CUtensorMap& tmV,
                            const ScoreParams& p, cudaStream_t stream) {
   const int ctas_per_g = (p.n_tiles * p.group + 7) / 8;
   const int grid = p.n_kv_heads * ctas_per_g;
-  cudaError_t e = launch_pass<D, BN, 1>(tmQs, tmK, tmV, p, grid, stream);
+  cudaError_t e = launch_score_pass1(D, BN, tmQs, tmK, tmV, p, grid, stream);
   if (e != cudaSuccess) return e;
-  return launch_pass<D, BN, 2>(tmQs, tmK, tmV, p, grid, stream);
+  return launch_pass2<D, BN>(tmQs, tmK, tmV, p, grid, stream);
 }
 
 }  // namespace

@@ -1,0 +1,349 @@
+// poem_score_pass1.cu -- pass 1 of the exact block scores (sm_100a): the dense causal
+// attention of the sampled queries.
+//
+// For the 16 strided sampled queries q_j = iB + j (B / 16) of every (head, query tile)
+// this pass computes the dense softmax output o and the log-sum-exp of the scaled
+// logits (log2 units) -- o is the dense reference output of the reading note
+// "Attention deletion error", Section 4.1, against which pass 2 (poem_score.cu)
+// measures every block's deviation I_b = || P_b V_b - m_b o || (Equation (4)).
+// P enters the P V contraction as a bf16 hi/lo pair (two MMAs into one accumulator,
+// ~16 significant bits), because I_b can cancel and needs o to ~1e-6 relative.
+//
+// Packing as in pass 2: one CTA per SM holds 8 groups of 16 sampled queries of one KV
+// head (2 adjacent tiles x 4 query heads for 4-way GQA), gathered by one 4-D TMA box
+// per group, and sweeps key blocks 0 .. (largest tile of the CTA).
+//
+// Pipeline:
+//   TMEM  S buffers s = 0, 1, 2 at [128 s, 128 s + BN); O at [384, 384 + D).  With
+//         three S buffers the MMAs run up to two blocks ahead of the softmax, so the
+//         softmax warps process blocks back to back.
+//   smem  Q tile, 3-stage K ring, 2-stage V ring (192 KB at d = 128).
+//   warps 0-3: online softmax, one sampled query per thread (running max with a lazy
+//         rescale of O when the max grows by more than 2^8); warp 4: TMA, K and V
+//         rings advancing independently; warp 5: MMAs, converged, issued by one
+//         elected lane.
+//   MMA order: S_0, S_1, S_2, PV_0, S_3, PV_1, ...  (S_b follows P V_{b-3}, which
+//   freed its S buffer).
+//
+// Every mbarrier wait is made at most one phase behind its barrier.  A rescale of O at
+// block b waits for P V_{b-1} on accumulator barrier (b - 1) % 2: S_b complete implies
+// P V_{b-3} complete, and P V_{b+1} cannot start before this block's P, so that
+// barrier is within one phase of the wait.  The end of the sweep waits on its own
+// barrier (o_full), committed once after the last P V.
+#include "common.cuh"
+#include "fwd_common.cuh"
+#include "score_common.cuh"
+
+namespace poem {
+namespace {
+
+template <int D, int BN>
+struct P1Cfg {
+  static constexpr int M = 128;
+  static constexpr int kGroups = 8;
+  static constexpr int kRowsPerGroup = 16;
+  static constexpr int kChunks = D / 64;
+  static constexpr int kStagesK = 3;
+  static constexpr int kStagesV = 2;
+  static constexpr int kQBytes = M * D * 2;
+  static constexpr int kKVBytes = BN * D * 2;
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffK = kOffQ + kQBytes;
+  static constexpr int kOffV = kOffK + kStagesK * kKVBytes;
+  static constexpr int kOffBar = kOffV + kStagesV * kKVBytes;
+  // at least 120 KB so that one CTA (holding all 512 TMEM columns) occupies an SM
+  static constexpr int kSmemBytes = (kOffBar + 256 + 1024) > 122880 ? (kOffBar + 256 + 1024) : 122880;
+  static constexpr uint32_t kTmemCols = 512;
+  static constexpr uint32_t kColO = 384;
+  static constexpr int kWarpProd = 4;
+  static constexpr int kWarpMma = 5;
+  static constexpr int kThreads = 192;
+  static constexpr uint32_t kIdescQK = idesc_bf16_f32(M, BN, 0);
+  static constexpr uint32_t kIdescPV = idesc_bf16_f32(M, D, 1);
+};
+
+struct P1Barriers {
+  uint64_t q_full;
+  uint64_t k_full[3], k_empty[3];
+  uint64_t v_full[2], v_empty[2];
+  uint64_t s_full[3], p_full[3];
+  uint64_t acc_full[2];  // P V_j complete, on barrier j % 2
+  uint64_t o_full;       // the last P V complete
+  uint64_t drain;
+  uint32_t tmem_base;
+  volatile int abort_flag;
+};
+
+using fwd::kDrainNs;
+using fwd::wait_or_abort;
+using score::exp_split_store_regs;
+using score::load_row;
+using score::row_max_regs;
+
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, P1Barriers* sb, const DevErr& e) {
+  return __all_sync(0xffffffffu, wait_or_abort(bar, parity, sb, e));
+}
+
+// CTA -> (KV head, first group): KV-head-major, the CTAs holding the last tiles first.
+__device__ __forceinline__ void p1_cta_coords(int cta, int ctas_per_g, int& g, int& z0) {
+  g = cta / ctas_per_g;
+  const int c = ctas_per_g - 1 - (cta - g * ctas_per_g);
+  z0 = c * 8;
+}
+
+template <int D, int BN>
+__global__ void __launch_bounds__(P1Cfg<D, BN>::kThreads, 1)
+    poem_score_pass1_kernel(const __grid_constant__ CUtensorMap tmQs, const __grid_constant__ CUtensorMap tmK,
+                            const __grid_constant__ CUtensorMap tmV, const ScoreParams p) {
+  using C = P1Cfg<D, BN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = smem + C::kOffQ;
+  uint8_t* sK = smem + C::kOffK;
+  uint8_t* sV = smem + C::kOffV;
+  P1Barriers* sb = reinterpret_cast<P1Barriers*>(smem + C::kOffBar);
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+  const int G = p.group;
+  const int n_groups = p.n_tiles * G;  // per KV head
+  const int ctas_per_g = (n_groups + 7) / 8;
+  int g, z0;
+  p1_cta_coords(blockIdx.x, ctas_per_g, g, z0);
+  const int z_last = min(z0 + 7, n_groups - 1);
+  const int t0 = p.q_tile0;
+  const int nb = z_last / G + 1 + t0;  // key blocks 0 .. largest (global) tile of the CTA
+  const int i_lo = z0 / G + t0;        // blocks < i_lo need no causal mask
+
+  if (tid == 0) {
+    mbar_init(&sb->q_full, 1);
+    for (int s = 0; s < 3; ++s) {
+      mbar_init(&sb->k_full[s], 1);
+      mbar_init(&sb->k_empty[s], 1);
+      mbar_init(&sb->s_full[s], 1);
+      mbar_init(&sb->p_full[s], 4);  // one arrival per softmax warp
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&sb->v_full[s], 1);
+      mbar_init(&sb->v_empty[s], 1);
+      mbar_init(&sb->acc_full[s], 1);
+    }
+    mbar_init(&sb->o_full, 1);
+    mbar_init(&sb->drain, 1);
+    sb->abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == C::kWarpMma) tmem_alloc<C::kTmemCols>(&sb->tmem_base);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sb->tmem_base;
+
+  if (warp == C::kWarpProd) {
+    // ============================ TMA producer ============================
+    // K and V rings advance independently: K_b is loaded once S_{b-3} has released its
+    // stage, V_b once P V_{b-2} has.
+    if (lane == 0) {
+      tma_prefetch_desc(&tmQs);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      mbar_arrive_expect_tx(&sb->q_full, C::kQBytes);
+      for (int zl = 0; zl < C::kGroups; ++zl) {
+        const int z = z0 + zl;  // groups past the end read out-of-range tiles: zero-filled
+        const int i = z / G;
+        const int hq = g * G + (z - i * G);
+        for (int c = 0; c < C::kChunks; ++c)
+          tma_load_4d(sQ + c * (C::M * 128) + zl * (C::kRowsPerGroup * 128), &tmQs, &sb->q_full, c * 64, hq, 0,
+                      i);
+      }
+      int kb = 0, vb = 0;
+      uint64_t t_last = globaltimer_ns();
+      while ((kb < nb || vb < nb) && !sb->abort_flag) {
+        bool progressed = false;
+        // a fresh stage passes the parity-1 test at once; later, completion #(b/stages - 1)
+        if (kb < nb && mbar_try_wait(&sb->k_empty[kb % 3], ((kb / 3) & 1) ^ 1)) {
+          const int s = kb % 3;
+          mbar_arrive_expect_tx(&sb->k_full[s], C::kKVBytes);
+          for (int c = 0; c < C::kChunks; ++c)
+            tma_load_3d(sK + s * C::kKVBytes + c * (BN * 128), &tmK, &sb->k_full[s], c * 64, g, kb * BN);
+          ++kb;
+          progressed = true;
+        }
+        if (vb < kb && mbar_try_wait(&sb->v_empty[vb & 1], ((vb >> 1) & 1) ^ 1)) {
+          const int s = vb & 1;
+          mbar_arrive_expect_tx(&sb->v_full[s], C::kKVBytes);
+          for (int c = 0; c < C::kChunks; ++c)
+            tma_load_3d(sV + s * C::kKVBytes + c * (BN * 128), &tmV, &sb->v_full[s], c * 64, g, vb * BN);
+          ++vb;
+          progressed = true;
+        }
+        if (progressed) {
+          t_last = globaltimer_ns();
+        } else if (globaltimer_ns() - t_last > p.err.timeout_ns) {
+          sb->abort_flag = 1;
+          raise_err(p.err, kErrTimeout);
+          break;
+        }
+      }
+      // Drain: the last load issued into each stage must have landed.
+      mbar_wait(&sb->q_full, 0, kDrainNs);
+      for (int b = max(0, kb - 3); b < kb; ++b) mbar_wait(&sb->k_full[b % 3], (b / 3) & 1, kDrainNs);
+      for (int b = max(0, vb - 2); b < vb; ++b) mbar_wait(&sb->v_full[b & 1], (b >> 1) & 1, kDrainNs);
+    }
+  } else if (warp == C::kWarpMma) {
+    // ============================ MMA issuer ============================
+    const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV);
+    const uint32_t tO = tmem + C::kColO;
+    bool ok = warp_wait(&sb->q_full, 0, sb, p.err);
+    auto issue_pv = [&](int j) -> bool {
+      const int s = j % 3, sv = j & 1;
+      if (!warp_wait(&sb->p_full[s], (j / 3) & 1, sb, p.err)) return false;
+      if (!warp_wait(&sb->v_full[sv], (j >> 1) & 1, sb, p.err)) return false;
+      tc_fence_after();
+      const uint32_t tP = tmem + s * 128;
+      const uint32_t aVs = aV + sv * C::kKVBytes;
+#pragma unroll
+      for (int kk = 0; kk < BN / 16; ++kk) {
+        // keys [16 kk, 16 kk + 16): P_hi words at [16 kk, +8), P_lo at [16 kk + 8, +8)
+        const uint64_t bdesc = smem_desc_sw128(aVs + kk * 2048, BN * 128, 1024);
+        mma_ts_warp(tO, tP + kk * 16, bdesc, C::kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
+        mma_ts_warp(tO, tP + kk * 16 + 8, bdesc, C::kIdescPV, 1u);
+      }
+      mma_commit_warp(&sb->v_empty[sv]);
+      mma_commit_warp(&sb->acc_full[j & 1]);
+      if (j == nb - 1) mma_commit_warp(&sb->o_full);
+      return true;
+    };
+    for (int b = 0; b < nb && ok; ++b) {
+      if (b >= 3 && !issue_pv(b - 3)) { ok = false; break; }
+      const int s = b % 3;
+      if (!warp_wait(&sb->k_full[s], (b / 3) & 1, sb, p.err)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t tS = tmem + s * 128;
+      const uint32_t aKs = aK + s * C::kKVBytes;
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t koff = (kk & 3) * 32;
+        const uint64_t adesc = smem_desc_sw128(aQ + (kk >> 2) * (C::M * 128) + koff, 16, 1024);
+        const uint64_t bdesc = smem_desc_sw128(aKs + (kk >> 2) * (BN * 128) + koff, 16, 1024);
+        mma_ss_warp(tS, adesc, bdesc, C::kIdescQK, kk > 0 ? 1u : 0u);
+      }
+      mma_commit_warp(&sb->s_full[s]);
+      mma_commit_warp(&sb->k_empty[s]);
+    }
+    for (int j = max(0, nb - 3); j < nb && ok; ++j)
+      if (!issue_pv(j)) ok = false;
+    mma_commit_warp(&sb->drain);
+    mbar_wait(&sb->drain, 0, kDrainNs);
+  } else {
+    // ============================ softmax warps ============================
+    const int r = tid;                       // TMEM lane = sampled row
+    const int zl = r >> 4;
+    const int j = r & 15;
+    const int z = z0 + zl;
+    const bool valid = (z < n_groups);
+    const int i = valid ? z / G : 0;
+    const int hq = g * G + (valid ? z - i * G : 0);
+    const int qpos = valid ? (i + t0) * BN + j * p.sample_stride : -1;  // key position; -1: padding row
+    const int64_t srow = ((int64_t)hq * p.n_tiles + i) * p.n_sample + j;
+    const uint32_t lane_off = ((uint32_t)(warp * 32) << 16);
+    const uint32_t tO = tmem + lane_off + C::kColO;
+    const float sl2 = p.scale_log2;
+    float m_run = -INFINITY, l_run = 0.f;
+    bool ok = true;
+    for (int b = 0; b < nb; ++b) {
+      const int s = b % 3;
+      const uint32_t tS = tmem + lane_off + s * 128;
+      if (!warp_wait(&sb->s_full[s], (b / 3) & 1, sb, p.err)) { ok = false; break; }
+      tc_fence_after();
+      const int lim = qpos - b * BN;  // columns <= lim are visible to this query
+      uint32_t a[BN / 32][32];        // the row of S, read once
+      load_row<BN>(tS, a);
+      const float mx = (b < i_lo) ? row_max_regs<BN, false>(a, lim) : row_max_regs<BN, true>(a, lim);
+      const float m_new = fmaxf(m_run, mx * sl2);
+      const bool grow = (m_new > m_run + 8.0f);
+      float alpha = 1.f;
+      if (grow) {
+        alpha = (m_run == -INFINITY) ? 0.f : ex2_approx(m_run - m_new);
+        m_run = m_new;
+      }
+      if (b >= 1 && __any_sync(0xffffffffu, grow)) {
+        // O holds P V_0 .. P V_{b-1} once P V_{b-1} is complete; P V_b waits for this
+        // block's P, so O may then be rescaled in place.
+        if (!warp_wait(&sb->acc_full[(b - 1) & 1], ((b - 1) >> 1) & 1, sb, p.err)) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t ov[32];
+          tmem_ld32(tO + c * 32, ov);
+          tmem_ld_wait();
+          tmem_reg_fence(ov);
+#pragma unroll
+          for (int x = 0; x < 32; ++x) ov[x] = __float_as_uint(__uint_as_float(ov[x]) * alpha);
+          tmem_st32(tO + c * 32, ov);
+        }
+      }
+      l_run *= alpha;
+      const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
+      l_run += (b < i_lo) ? exp_split_store_regs<BN, false>(tS, a, sl2, m_use, lim)
+                          : exp_split_store_regs<BN, true>(tS, a, sl2, m_use, lim);
+      tmem_st_wait();
+      tc_fence_before();
+      warp_arrive(&sb->p_full[s]);
+    }
+    // ---- epilogue: o = O / l and lse = m + log2(l) (log2 units) ----
+    if (__all_sync(0xffffffffu, ok && !sb->abort_flag) && warp_wait(&sb->o_full, 0, sb, p.err)) {
+      tc_fence_after();
+      const float inv_l = (l_run > 0.f) ? 1.f / l_run : 0.f;
+      float* dst = p.ws_o + srow * D;
+      const bool in_ws = POEM_IN_BOUNDS(p.err, srow, (int64_t)p.n_q_heads * p.n_tiles * p.n_sample);
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t ov[32];
+        tmem_ld32(tO + c * 32, ov);
+        tmem_ld_wait();
+        tmem_reg_fence(ov);
+        if (valid && in_ws) {
+          float4* d4 = reinterpret_cast<float4*>(dst + c * 32);
+#pragma unroll
+          for (int x = 0; x < 8; ++x)
+            d4[x] = make_float4(__uint_as_float(ov[4 * x]) * inv_l, __uint_as_float(ov[4 * x + 1]) * inv_l,
+                                __uint_as_float(ov[4 * x + 2]) * inv_l, __uint_as_float(ov[4 * x + 3]) * inv_l);
+        }
+      }
+      if (valid && in_ws) p.ws_lse[srow] = (l_run > 0.f) ? m_run + __log2f(l_run) : -INFINITY;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == C::kWarpMma) {
+    __syncwarp();
+    tmem_dealloc<C::kTmemCols>(tmem);
+  }
+}
+
+template <int D, int BN>
+cudaError_t launch_p1_t(const CUtensorMap& tmQs, const CUtensorMap& tmK, const CUtensorMap& tmV,
+                        const ScoreParams& p, int grid, cudaStream_t stream) {
+  using C = P1Cfg<D, BN>;
+  cudaError_t e = ensure_smem_limit(poem_score_pass1_kernel<D, BN>, C::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  poem_score_pass1_kernel<D, BN><<<grid, C::kThreads, C::kSmemBytes, stream>>>(tmQs, tmK, tmV, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_score_pass1(int head_dim, int block, const CUtensorMap& tmQs, const CUtensorMap& tmK,
+                               const CUtensorMap& tmV, const ScoreParams& p, int grid, cudaStream_t stream) {
+  if (head_dim == 128 && block == 128) return launch_p1_t<128, 128>(tmQs, tmK, tmV, p, grid, stream);
+  if (head_dim == 128 && block == 64) return launch_p1_t<128, 64>(tmQs, tmK, tmV, p, grid, stream);
+  if (head_dim == 64 && block == 128) return launch_p1_t<64, 128>(tmQs, tmK, tmV, p, grid, stream);
+  if (head_dim == 64 && block == 64) return launch_p1_t<64, 64>(tmQs, tmK, tmV, p, grid, stream);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace poem

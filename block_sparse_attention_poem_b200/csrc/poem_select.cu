@@ -219,8 +219,11 @@ __device__ void emit_row(const SelectParams& p, const int* keep, int row, int i,
   int pos = block_excl_scan_int(cnt, tmpi, &total);
   int32_t* dst = p.scratch + off;
   for (int b = b0; b < b1; ++b)
-    if (keep[b]) dst[pos++] = b;
-  if (threadIdx.x == 0) p.counts[row] = total;
+    if (keep[b]) {
+      if (POEM_IN_BOUNDS(p.err, off + pos, p.n_entries)) dst[pos] = b;
+      ++pos;
+    }
+  if (threadIdx.x == 0 && POEM_IN_BOUNDS(p.err, row, (int64_t)p.n_q_heads * p.n_tiles)) p.counts[row] = total;
 }
 
 __global__ void __launch_bounds__(kSelThreads) select_rows_kernel(const SelectParams p) {
@@ -450,11 +453,12 @@ __global__ void __launch_bounds__(128) gather_lists_kernel(const SelectParams p)
   const int i = row - h * T;
   const int64_t start = p.row_ptr[row];
   const int n = p.counts[row];
-  const int32_t* src = p.scratch + row_off(T, p.q_tile0, h, i);
+  const int64_t off = row_off(T, p.q_tile0, h, i);
+  const int32_t* src = p.scratch + off;
   const int64_t cap = p.col_capacity;
   for (int x = threadIdx.x; x < n; x += blockDim.x) {
     const int64_t d = start + x;
-    if (d < cap) p.col_idx[d] = src[x];
+    if (d < cap && POEM_IN_BOUNDS(p.err, off + x, p.n_entries)) p.col_idx[d] = src[x];
   }
   if (threadIdx.x == 0 && start + n > cap) raise_err(p.err, kErrCapacity);
 }

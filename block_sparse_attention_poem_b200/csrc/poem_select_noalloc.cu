@@ -152,6 +152,7 @@ extern "C" poem_status poem_select_noalloc(const poem_shape* shape, const float*
   p.tau = (double)tau;
   p.mass_only = 0;
   p.err = poem::DevErr{reinterpret_cast<uint32_t*>(base), 0};
+  p.n_entries = (int64_t)shape->n_q_heads * poem::row_entries(T, p.q_tile0);
   e = poem::launch_select(p, s);
   if (e != cudaSuccess) {
     forget_current_device();

@@ -18,6 +18,7 @@ enum : uint32_t {
   kErrBadList = 2u,      // a block id outside 0..tile (skipped)
   kErrCapacity = 4u,     // col_idx capacity too small (output truncated)
   kErrBadParam = 8u,     // a per-head threshold was NaN, negative or infinite (row kept whole)
+  kErrBounds = 16u,      // debug builds (POEM_CHECKS): an index outside its buffer (access skipped)
 };
 
 struct DevErr {
@@ -28,6 +29,20 @@ struct DevErr {
 __device__ __forceinline__ void raise_err(const DevErr& e, uint32_t bits) {
   if (e.word) atomicOr(e.word, bits);
 }
+
+// Bounds check of the debug build (compiled with -DPOEM_CHECKS): an index outside
+// [0, n) sets kErrBounds and the caller skips the access.  Release builds compile
+// every check to `true`.
+__device__ __forceinline__ bool in_bounds_check(const DevErr& e, int64_t idx, int64_t n) {
+  if (idx >= 0 && idx < n) return true;
+  raise_err(e, kErrBounds);
+  return false;
+}
+#ifdef POEM_CHECKS
+#define POEM_IN_BOUNDS(err, idx, n) ::poem::in_bounds_check((err), (int64_t)(idx), (int64_t)(n))
+#else
+#define POEM_IN_BOUNDS(err, idx, n) true
+#endif
 
 __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;
@@ -69,6 +84,15 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "r"(smem_u32(bar)), "r"(parity)
       : "memory");
   return ok != 0;
+}
+
+// One arrival for a whole converged warp: the lanes meet at __syncwarp (which also
+// orders their earlier memory writes before lane 0's release-arrive).  Barriers
+// signalled this way count warps, not threads; arriving once per warp instead of
+// once per thread keeps 128 serialised shared-memory arrivals off the critical path.
+__device__ __forceinline__ void warp_arrive(uint64_t* bar) {
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
 }
 
 // Wait for the phase with the given parity to complete, at most limit_ns.

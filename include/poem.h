@@ -57,7 +57,8 @@ typedef enum poem_status {
   POEM_ERR_TIMEOUT = 4,     /* device: a bounded wait gave up (reported by poem_check)  */
   POEM_ERR_CAPACITY = 5,    /* col_capacity too small (device: reported by poem_check)  */
   POEM_ERR_WORKSPACE = 6,   /* ws_bytes smaller than poem_workspace_size reports        */
-  POEM_ERR_BAD_LIST = 7     /* device: a listed block id outside 0..tile (skipped)      */
+  POEM_ERR_BAD_LIST = 7,    /* device: a listed block id outside 0..tile (skipped)      */
+  POEM_ERR_BOUNDS = 8       /* device, debug build only: an index outside its buffer   */
 } poem_status;
 
 /*
@@ -307,7 +308,14 @@ poem_status bsa_fwd_grouped(const poem_shape* shape, const poem_bf16* q, const p
  * Synchronise `stream`, read and clear the error word at the start of `ws`
  * (a workspace passed to one of the calls above) and map it to a status:
  * POEM_ERR_TIMEOUT, POEM_ERR_BAD_LIST, POEM_ERR_CAPACITY, POEM_ERR_INVALID_ARG
- * (a bad per-head threshold), or POEM_OK.
+ * (a bad per-head threshold), POEM_ERR_BOUNDS (a failed bounds check of the
+ * debug build, see below), or POEM_OK.
+ *
+ * Debug build: the library compiled with -DPOEM_CHECKS (libpoem_checks.so, built
+ * by the package's build script) adds device-side bounds checks on the packed
+ * score writes, the sampled-query workspace and the selection scratch; an index
+ * outside its buffer skips the access and sets POEM_ERR_BOUNDS.  Release builds
+ * compile the checks away.
  */
 poem_status poem_check(void* stream, void* ws);
 

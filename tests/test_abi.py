@@ -42,6 +42,28 @@ def test_library_exports_every_declared_symbol(poem):
     assert set(_declared()) <= set(poem.EXPORTED)
 
 
+def test_checks_build_exports_the_same_symbols(poem):
+    """The debug build (bounds checks compiled in), when built, exports every entry point."""
+    from block_sparse_attention_poem_b200 import build
+
+    path = build.LIBS["checks"]
+    if not os.path.exists(path):
+        pytest.skip("libpoem_checks.so not built")
+    lib = ctypes.CDLL(path)
+    for name in _declared():
+        assert hasattr(lib, name), name
+
+
+def test_binding_rejects_an_unknown_library_variant(tmp_path):
+    import subprocess
+    import sys
+
+    env = dict(os.environ, POEM_LIBRARY_VARIANT="fast")
+    r = subprocess.run([sys.executable, "-c", "import block_sparse_attention_poem_b200"], cwd=ROOT, env=env,
+                       capture_output=True, text=True)
+    assert r.returncode != 0 and "POEM_LIBRARY_VARIANT" in r.stderr
+
+
 def _shape(poem, **kw):
     base = dict(n_tokens=1024, n_q_heads=4, n_kv_heads=2, head_dim=128, block=128, n_sample=16, softmax_scale=0.0,
                 q_offset=0, q_stride_tok=512, q_stride_head=128, kv_stride_tok=256, kv_stride_head=128,

@@ -383,6 +383,19 @@ def test_score_shift_invariance(poem):
     assert np.array_equal(m0, m1)
 
 
+def test_score_large_value_range(poem):
+    """Values scaled by powers of two up to 2^16 (far beyond unit scale): the scores
+    scale with V and still match the oracle (the P V contraction keeps V in bf16)."""
+    x = poem_synth.heavy_block_layer(2048, 4, 1, 128, block=128, seed=21)
+    for scale in (2.0 ** -8, 2.0 ** 16):
+        xs = dict(x)
+        xs["v"] = (x["v"].float() * scale).to(torch.bfloat16)  # a power of two: exact in bf16
+        Ig, mg, status = _gpu_score(poem, xs, 128)
+        assert status == 0
+        Ir, mr = problem_from(xs, 128).score_all()
+        assert score_err_excess(Ig, Ir, mg, mr, max_value_norm(xs["v"])) <= 1.0, scale
+
+
 # ---------------------------------------------------------------------------
 # the whole layer
 # ---------------------------------------------------------------------------
