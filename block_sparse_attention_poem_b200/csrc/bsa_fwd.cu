@@ -14,10 +14,10 @@
 //              O in TMEM only when the max grows by more than 2^8, and runs the
 //              epilogue (O / l -> bf16, lse).
 //   warp 4     TMA producer: Q once, then K_j and V_j of every listed block.
-//   warp 5     MMA issuer (one thread): S = Q K_j^T (SS form), O += P V_j (P read
-//              from TMEM) in two 64-key halves, each started as soon as the softmax
-//              warps have written that half of P; completion tracked with
-//              tcgen05.commit -> mbarriers.
+//   warp 5     MMA issuer (converged warp; one elected lane issues): S = Q K_j^T
+//              (SS form), O += P V_j (P read from TMEM) in two 64-key halves, each
+//              started as soon as the softmax warps have written that half of P;
+//              completion tracked with tcgen05.commit -> mbarriers.
 // TMEM: 256 columns per CTA -- S/P at [0, BN), O at [128, 128 + D).  Shared
 // memory holds one Q, one K and one V tile (96 KB at D = BN = 128), so two CTAs
 // run per SM and their softmax / MMA phases interleave on the tensor cores.
@@ -57,6 +57,7 @@ using fwd::block_ok;
 using fwd::exp_pack_store;
 using fwd::kDrainNs;
 using fwd::wait_or_abort;
+using fwd::warp_wait_or_abort;
 
 template <int D, int BN>
 __global__ void __launch_bounds__(kThreadsFwd, 2)
@@ -154,61 +155,61 @@ __global__ void __launch_bounds__(kThreadsFwd, 2)
     }
   } else if (warp == 5) {
     // ============================ MMA issuer ============================
-    if (lane == 0) {
-      const uint32_t tS = tmem + C::kColS;
-      const uint32_t tO = tmem + C::kColO;
-      const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV);
-      int it = 0;
-      bool ok = true;
-      bool q_ready = false;
-      // O += P_j V_j in two 64-key halves, each issued as soon as the softmax warps
-      // have written that half of P_j.
-      auto issue_pv = [&](int j) -> bool {
-        if (!wait_or_abort(&sb->v_full, j & 1, sb, p.err)) return false;
+    // The whole warp runs the loop converged (list entries, waits and operands are
+    // warp-uniform); one elected lane issues each MMA and commit.
+    const uint32_t tS = tmem + C::kColS;
+    const uint32_t tO = tmem + C::kColO;
+    const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV);
+    int it = 0;
+    bool ok = true;
+    bool q_ready = false;
+    // O += P_j V_j in two 64-key halves, each issued as soon as the softmax warps
+    // have written that half of P_j.
+    auto issue_pv = [&](int j) -> bool {
+      if (!warp_wait_or_abort(&sb->v_full, j & 1, sb, p.err)) return false;
 #pragma unroll
-        for (int hv = 0; hv < BN / 64; ++hv) {
-          if (!wait_or_abort(&sb->p_half[hv], j & 1, sb, p.err)) return false;
-          tc_fence_after();
-#pragma unroll
-          for (int kk = hv * 4; kk < hv * 4 + 4; ++kk) {
-            // V tile is MN-major (d contiguous): LBO = stride between 64-wide d chunks,
-            // SBO = stride between 8-key groups; a k-step covers 16 keys = 2 groups.
-            const uint64_t bdesc = smem_desc_sw128(aV + kk * 2048, BN * 128, 1024);
-            mma_ts(tO, tS + kk * 8, bdesc, C::kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
-          }
-        }
-        mma_commit(&sb->v_empty);
-        return true;
-      };
-      for (int e = beg; e < end && ok; ++e) {
-        if (!block_ok(p.col_idx[e], gtile)) continue;
-        if (!q_ready) {
-          if (!wait_or_abort(&sb->q_full, 0, sb, p.err)) { ok = false; break; }
-          q_ready = true;
-        }
-        if (it > 0 && !issue_pv(it - 1)) { ok = false; break; }
-        if (!wait_or_abort(&sb->k_full, it & 1, sb, p.err)) { ok = false; break; }
+      for (int hv = 0; hv < BN / 64; ++hv) {
+        if (!warp_wait_or_abort(&sb->p_half[hv], j & 1, sb, p.err)) return false;
         tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          // Q and K tiles are K-major, 128-byte swizzled; a k-step is 16 elements (32 B)
-          // inside a 64-element chunk; chunks are whole row-blocks apart.
-          const uint32_t koff = (kk & 3) * 32;
-          const uint64_t adesc = smem_desc_sw128(aQ + (kk >> 2) * (C::M * 128) + koff, 16, 1024);
-          const uint64_t bdesc = smem_desc_sw128(aK + (kk >> 2) * (BN * 128) + koff, 16, 1024);
-          mma_ss(tS, adesc, bdesc, C::kIdescQK, kk > 0 ? 1u : 0u);
+        for (int kk = hv * 4; kk < hv * 4 + 4; ++kk) {
+          // V tile is MN-major (d contiguous): LBO = stride between 64-wide d chunks,
+          // SBO = stride between 8-key groups; a k-step covers 16 keys = 2 groups.
+          const uint64_t bdesc = smem_desc_sw128(aV + kk * 2048, BN * 128, 1024);
+          mma_ts_warp(tO, tS + kk * 8, bdesc, C::kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
         }
-        mma_commit(&sb->s_full);
-        mma_commit(&sb->k_empty);
-        ++it;
       }
-      if (ok && it > 0) {
-        if (issue_pv(it - 1)) mma_commit(&sb->o_full);
+      mma_commit_warp(&sb->v_empty);
+      return true;
+    };
+    for (int e = beg; e < end && ok; ++e) {
+      if (!block_ok(p.col_idx[e], gtile)) continue;
+      if (!q_ready) {
+        if (!warp_wait_or_abort(&sb->q_full, 0, sb, p.err)) { ok = false; break; }
+        q_ready = true;
       }
-      // Drain every MMA this thread issued before TMEM is released.
-      mma_commit(&sb->drain);
-      mbar_wait(&sb->drain, 0, kDrainNs);
+      if (it > 0 && !issue_pv(it - 1)) { ok = false; break; }
+      if (!warp_wait_or_abort(&sb->k_full, it & 1, sb, p.err)) { ok = false; break; }
+      tc_fence_after();
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        // Q and K tiles are K-major, 128-byte swizzled; a k-step is 16 elements (32 B)
+        // inside a 64-element chunk; chunks are whole row-blocks apart.
+        const uint32_t koff = (kk & 3) * 32;
+        const uint64_t adesc = smem_desc_sw128(aQ + (kk >> 2) * (C::M * 128) + koff, 16, 1024);
+        const uint64_t bdesc = smem_desc_sw128(aK + (kk >> 2) * (BN * 128) + koff, 16, 1024);
+        mma_ss_warp(tS, adesc, bdesc, C::kIdescQK, kk > 0 ? 1u : 0u);
+      }
+      mma_commit_warp(&sb->s_full);
+      mma_commit_warp(&sb->k_empty);
+      ++it;
     }
+    if (ok && it > 0) {
+      if (issue_pv(it - 1)) mma_commit_warp(&sb->o_full);
+    }
+    // Drain every MMA this warp issued before TMEM is released.
+    mma_commit_warp(&sb->drain);
+    mbar_wait(&sb->drain, 0, kDrainNs);
   } else {
     // ============================ softmax warps ============================
     const int r = tid;                       // query row within the tile (TMEM lane)

@@ -26,6 +26,12 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, Ba
   }
 }
 
+// The same wait made by a whole warp, with a warp-uniform result.
+template <typename Barriers>
+__device__ __forceinline__ bool warp_wait_or_abort(uint64_t* bar, uint32_t parity, Barriers* sb, const DevErr& e) {
+  return __all_sync(0xffffffffu, wait_or_abort(bar, parity, sb, e));
+}
+
 constexpr uint64_t kDrainNs = 2000000000ull;  // waits for already-issued async work
 
 // Exponentials of one S row (re-read from TMEM in 64-column halves), the bf16 P
