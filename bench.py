@@ -48,16 +48,18 @@ WORKLOADS = {
     # name: (n_tokens, Hq, Hkv, d, block, rope_base, tau)
     "llama3.1-8b-layer-128k": (131072, 32, 8, 128, 128, 500000.0, 0.05),
     "llama3.1-8b-layer-32k": (32768, 32, 8, 128, 128, 500000.0, 0.05),
+    "llama3.1-8b-layer-64k": (65536, 32, 8, 128, 128, 500000.0, 0.05),
     "qwen3-14b-layer-64k": (65536, 40, 8, 128, 128, 1000000.0, 0.05),
 }
 # Roofline denominators measured on B200 (a STREAM-style copy and a bf16 GEMM;
 # MEASURED_PEAKS.json, when present, takes precedence).
 FALLBACK_PEAKS = {"bf16_tflops": 1667.9, "bf16_tflops_sustained": 1378.8, "hbm_gbs": 6452.5}
-# DRAM bytes per bsa_fwd launch on the 128K layer: the ncu capture of the 32K layer
-# (dram__bytes_read.sum + dram__bytes_write.sum = 407.6 + 233.3 = 640.9 MB per launch)
-# scaled by rows processed (x4).  Valid only for the kernel source it was taken on.
-BSA_FWD_TRAFFIC = {"bytes": 2.562e9, "source_sha256_prefix": "e5d86b04b78dbb9e",
-                   "note": "ncu dram bytes of the 32K layer launch x4 rows"}
+# DRAM bytes per bsa_fwd launch on the 128K layer: the ncu capture of the 64K layer
+# (dram__bytes_read.sum + dram__bytes_write.sum = 842.4 + 502.8 = 1345.2 MB per launch)
+# scaled by rows processed (x2); the 32K capture (642.4 MB, x2.09 to 64K) confirms the
+# scaling.  Valid only for the kernel source it was taken on.
+BSA_FWD_TRAFFIC = {"bytes": 2.690e9, "source_sha256_prefix": "090feeb3d9772452",
+                   "note": "ncu dram bytes of the 64K layer launch x2 rows (32K capture x4: 2.57 GB)"}
 
 
 def bsa_fwd_traffic():
