@@ -3,6 +3,7 @@
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include <map>
@@ -96,6 +97,14 @@ struct ScoreParams {
   float scale_log2;
   DevErr err;
   int64_t n_entries;     // entries of I_hat / m_hat (bounds of the debug build)
+  // Pass 1 runs the P V contraction of CTAs whose tiles are all >= 32 with one fp16
+  // P on a dense fp16 copy of V; a finite |v| outside the fp16 range sets
+  // *v_overflow and every CTA takes the bf16 hi/lo contraction instead.
+  const __nv_bfloat16* v_src;
+  int64_t v_stride_tok, v_stride_head;
+  __half* v_half;        // [n_kv, Hkv, D]
+  uint32_t* v_overflow;  // in the workspace header (byte 8)
+  int n_kv;              // key / value tokens (q_offset + n_tokens)
 };
 
 struct SelectParams {
@@ -158,9 +167,11 @@ cudaError_t launch_bsa_fwd(int head_dim, int block, const CUtensorMap& tmQ, cons
 cudaError_t launch_bsa_fwd_grouped(int head_dim, int block, const CUtensorMap& tmQ, const CUtensorMap& tmK,
                                    const CUtensorMap& tmV, const FwdParams& p, int n_kv_heads, cudaStream_t stream);
 cudaError_t launch_score(int head_dim, int block, const CUtensorMap& tmQs, const CUtensorMap& tmK,
-                         const CUtensorMap& tmV, const ScoreParams& p, cudaStream_t stream);
+                         const CUtensorMap& tmV, const CUtensorMap& tmVh, const ScoreParams& p, cudaStream_t stream);
 cudaError_t launch_score_pass1(int head_dim, int block, const CUtensorMap& tmQs, const CUtensorMap& tmK,
-                               const CUtensorMap& tmV, const ScoreParams& p, int grid, cudaStream_t stream);
+                               const CUtensorMap& tmV, const CUtensorMap& tmVh, const ScoreParams& p, int grid,
+                               cudaStream_t stream);
+cudaError_t launch_v_to_half(const ScoreParams& p, int head_dim, cudaStream_t stream);
 cudaError_t launch_select(const SelectParams& p, cudaStream_t stream);
 cudaError_t launch_pooled(int head_dim, PoolParams p, cudaStream_t stream);
 

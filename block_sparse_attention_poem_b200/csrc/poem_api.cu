@@ -76,11 +76,14 @@ size_t tri_entries(const poem_shape* s, const Layout& L) {
   return (size_t)s->n_q_heads * (size_t)poem::row_entries(L.T, L.t0);
 }
 
-// Score workspace: header (error word), then the dense outputs o [rows, D] fp32 and
-// the log-sum-exps [rows] of the sampled queries (pass 1 -> pass 2).
+// Score workspace: header (error word; the fp16-range flag of V at byte 8), the dense
+// outputs o [rows, D] fp32 and log-sum-exps [rows] of the sampled queries (pass 1 ->
+// pass 2), then the fp16 copy of V [n_kv, Hkv, D] for pass 1's fp16 P V contraction.
 size_t score_ws_bytes(const poem_shape* s, int T) {
   const size_t rows = (size_t)s->n_q_heads * T * s->n_sample;
-  return poem::kWsHeader + round_up(rows * s->head_dim * sizeof(float), 256) + round_up(rows * sizeof(float), 256);
+  const size_t vh = (size_t)(s->q_offset + s->n_tokens) * s->n_kv_heads * s->head_dim * 2;
+  return poem::kWsHeader + round_up(rows * s->head_dim * sizeof(float), 256) + round_up(rows * sizeof(float), 256) +
+         round_up(vh, 256);
 }
 
 size_t select_ws_bytes(const poem_shape* s, const Layout& L) {
@@ -113,14 +116,15 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 // [n_tokens, n_heads, head_dim] bf16 viewed as a 3-D tensor (head_dim, head, token);
 // box = 64 elements x 1 head x box_rows tokens, 128-byte swizzle.
 poem_status make_map_3d(CUtensorMap* m, const void* base, int head_dim, int n_heads, int n_tokens, int64_t st_head,
-                        int64_t st_tok, int box_rows) {
+                        int64_t st_tok, int box_rows,
+                        CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
   auto fn = encode_fn();
   if (!fn) return arg_fail(POEM_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
   cuuint64_t dims[3] = {(cuuint64_t)head_dim, (cuuint64_t)n_heads, (cuuint64_t)n_tokens};
   cuuint64_t strides[2] = {(cuuint64_t)st_head * 2, (cuuint64_t)st_tok * 2};
   cuuint32_t box[3] = {64, 1, (cuuint32_t)box_rows};
   cuuint32_t es[3] = {1, 1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+  CUresult r = fn(m, dtype, 3, const_cast<void*>(base), dims, strides, box, es,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) {
@@ -193,11 +197,24 @@ poem_status poem_score(const poem_shape* shape, const poem_bf16* q, const poem_b
   uint8_t* base = reinterpret_cast<uint8_t*>(ws);
   const size_t off_o = poem::kWsHeader;
   const size_t off_lse = off_o + round_up(rows * shape->head_dim * sizeof(float), 256);
+  const size_t off_vh = off_lse + round_up(rows * sizeof(float), 256);
+  // dense fp16 copy of V for pass 1: [n_kv, Hkv, D], head stride D, token stride Hkv D
+  CUtensorMap tmVh;
+  if ((st = make_map_3d(&tmVh, base + off_vh, shape->head_dim, shape->n_kv_heads, L.n_kv, shape->head_dim,
+                        (int64_t)shape->n_kv_heads * shape->head_dim, shape->block,
+                        CU_TENSOR_MAP_DATA_TYPE_FLOAT16)) != POEM_OK)
+    return st;
   poem::ScoreParams p{};
   p.I_hat = I_hat;
   p.m_hat = m_hat;
   p.ws_o = reinterpret_cast<float*>(base + off_o);
   p.ws_lse = reinterpret_cast<float*>(base + off_lse);
+  p.v_src = reinterpret_cast<const __nv_bfloat16*>(v);
+  p.v_stride_tok = shape->kv_stride_tok;
+  p.v_stride_head = shape->kv_stride_head;
+  p.v_half = reinterpret_cast<__half*>(base + off_vh);
+  p.v_overflow = reinterpret_cast<uint32_t*>(base + 8);
+  p.n_kv = L.n_kv;
   p.n_tokens = shape->n_tokens;
   p.n_q_heads = shape->n_q_heads;
   p.n_kv_heads = shape->n_kv_heads;
@@ -209,7 +226,7 @@ poem_status poem_score(const poem_shape* shape, const poem_bf16* q, const poem_b
   p.scale_log2 = L.scale * poem::kLog2e;
   p.err = dev_err(ws);
   p.n_entries = (int64_t)tri_entries(shape, L);
-  cudaError_t e = poem::launch_score(shape->head_dim, shape->block, tmQs, tmK, tmV, p, (cudaStream_t)stream);
+  cudaError_t e = poem::launch_score(shape->head_dim, shape->block, tmQs, tmK, tmV, tmVh, p, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "poem_score launch");
   return POEM_OK;
 }

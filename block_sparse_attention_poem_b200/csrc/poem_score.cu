@@ -382,13 +382,16 @@ cudaError_t launch_pass2(const CUtensorMap& tmQs, const CUtensorMap& tmK, const 
   return cudaGetLastError();
 }
 
-// Pass 1 (poem_score_pass1.cu: o and lse of the sampled queries), then pass 2.
+// The fp16 copy of V, pass 1 (poem_score_pass1.cu: o and lse of the sampled
+// queries), then pass 2.
 template <int D, int BN>
 cudaError_t launch_score_t(const CUtensorMap& tmQs, const CUtensorMap& tmK, const CUtensorMap& tmV,
-                           const ScoreParams& p, cudaStream_t stream) {
+                           const CUtensorMap& tmVh, const ScoreParams& p, cudaStream_t stream) {
   const int ctas_per_g = (p.n_tiles * p.group + 7) / 8;
   const int grid = p.n_kv_heads * ctas_per_g;
-  cudaError_t e = launch_score_pass1(D, BN, tmQs, tmK, tmV, p, grid, stream);
+  cudaError_t e = launch_v_to_half(p, D, stream);
+  if (e != cudaSuccess) return e;
+  e = launch_score_pass1(D, BN, tmQs, tmK, tmV, tmVh, p, grid, stream);
   if (e != cudaSuccess) return e;
   return launch_pass2<D, BN>(tmQs, tmK, tmV, p, grid, stream);
 }
@@ -396,11 +399,11 @@ cudaError_t launch_score_t(const CUtensorMap& tmQs, const CUtensorMap& tmK, cons
 }  // namespace
 
 cudaError_t launch_score(int head_dim, int block, const CUtensorMap& tmQs, const CUtensorMap& tmK,
-                         const CUtensorMap& tmV, const ScoreParams& p, cudaStream_t stream) {
-  if (head_dim == 128 && block == 128) return launch_score_t<128, 128>(tmQs, tmK, tmV, p, stream);
-  if (head_dim == 128 && block == 64) return launch_score_t<128, 64>(tmQs, tmK, tmV, p, stream);
-  if (head_dim == 64 && block == 128) return launch_score_t<64, 128>(tmQs, tmK, tmV, p, stream);
-  if (head_dim == 64 && block == 64) return launch_score_t<64, 64>(tmQs, tmK, tmV, p, stream);
+                         const CUtensorMap& tmV, const CUtensorMap& tmVh, const ScoreParams& p, cudaStream_t stream) {
+  if (head_dim == 128 && block == 128) return launch_score_t<128, 128>(tmQs, tmK, tmV, tmVh, p, stream);
+  if (head_dim == 128 && block == 64) return launch_score_t<128, 64>(tmQs, tmK, tmV, tmVh, p, stream);
+  if (head_dim == 64 && block == 128) return launch_score_t<64, 128>(tmQs, tmK, tmV, tmVh, p, stream);
+  if (head_dim == 64 && block == 64) return launch_score_t<64, 64>(tmQs, tmK, tmV, tmVh, p, stream);
   return cudaErrorInvalidValue;
 }
 

@@ -6,8 +6,16 @@
 // logits (log2 units) -- o is the dense reference output of the reading note
 // "Attention deletion error", Section 4.1, against which pass 2 (poem_score.cu)
 // measures every block's deviation I_b = || P_b V_b - m_b o || (Equation (4)).
-// P enters the P V contraction as a bf16 hi/lo pair (two MMAs into one accumulator,
-// ~16 significant bits), because I_b can cancel and needs o to ~1e-6 relative.
+// I_b can cancel, so o is needed to ~1e-6 relative.  P enters the P V contraction
+//   - as one fp16 matrix (11 significant bits, one MMA) on an fp16 copy of V, in the
+//     CTAs whose query tiles are all >= 32: o averages over >= 32 blocks of keys and
+//     its error stays far inside the score tolerance (a simulation against the fp64
+//     oracle on the Llama-shaped 32K layer: 3% of the tolerance for tiles >= 32);
+//     P is scaled by 2^6 (reference max - 6) so it stays in fp16's normal range;
+//   - as a bf16 hi/lo pair (two MMAs into one accumulator, ~16 significant bits) in
+//     the CTAs with earlier tiles, where few keys are visible (tile 0's one block
+//     cancels exactly), and everywhere when a finite |v| exceeds the fp16 range
+//     (the V copy then raises a flag in the workspace).
 //
 // Packing as in pass 2: one CTA per SM holds 8 groups of 16 sampled queries of one KV
 // head (2 adjacent tiles x 4 query heads for 4-way GQA), gathered by one 4-D TMA box
@@ -60,6 +68,8 @@ struct P1Cfg {
   static constexpr int kThreads = 192;
   static constexpr uint32_t kIdescQK = idesc_bf16_f32(M, BN, 0);
   static constexpr uint32_t kIdescPV = idesc_bf16_f32(M, D, 1);
+  static constexpr uint32_t kIdescPVh = idesc_f16_f32(M, D, 1);  // fp16 P x fp16 V
+  static constexpr int kHalfMinTile = 32;  // smallest global tile of a CTA taking the fp16 P
 };
 
 struct P1Barriers {
@@ -77,6 +87,67 @@ struct P1Barriers {
 using fwd::kDrainNs;
 using fwd::wait_or_abort;
 using score::exp_split_store_regs;
+
+// The exponentials of a register-held row as one fp16 P: k-step kk (keys 16 kk ..
+// 16 kk + 15) in columns [8 kk, 8 kk + 8) of the row's S buffer.  Returns sum p.
+template <int BN, bool MASKED>
+__device__ __forceinline__ float exp_f16_store_regs(uint32_t tS, const uint32_t (&a)[BN / 32][32], float sl2,
+                                                    float m_use, int lim) {
+  const uint64_t scale2 = f2_pack(sl2, sl2);
+  const uint64_t negm2 = f2_pack(-m_use, -m_use);
+  uint64_t acc = f2_pack(0.f, 0.f);
+#pragma unroll
+  for (int c = 0; c < BN / 32; ++c) {
+    uint32_t out[16];
+#pragma unroll
+    for (int x = 0; x < 16; ++x) {
+      const int col = c * 32 + 2 * x;
+      const uint64_t xv = f2_fma(f2_pack(__uint_as_float(a[c][2 * x]), __uint_as_float(a[c][2 * x + 1])), scale2, negm2);
+      float x0, x1;
+      f2_unpack(xv, x0, x1);
+      float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+      if (MASKED) {
+        if (col > lim) p0 = 0.f;
+        if (col + 1 > lim) p1 = 0.f;
+      }
+      acc = f2_add(acc, f2_pack(p0, p1));
+      out[x] = pack_f16x2(p0, p1);
+    }
+    tmem_st16(tS + c * 16, out);
+  }
+  float a0, a1;
+  f2_unpack(acc, a0, a1);
+  return a0 + a1;
+}
+
+// ---- V -> fp16 -----------------------------------------------------------------
+// One thread converts 8 consecutive channels of one (token, KV head) row of V into the
+// dense fp16 copy [n_kv, Hkv, D] (exact for every bf16 value in fp16's range); a finite
+// |v| above the fp16 maximum sets the flag.
+__global__ void __launch_bounds__(256) v_to_half_kernel(const ScoreParams p, int head_dim) {
+  const int per_row = head_dim / 8;
+  const int64_t n_items = (int64_t)p.n_kv * p.n_kv_heads * per_row;
+  bool over = false;
+  for (int64_t it = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; it < n_items;
+       it += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t row = it / per_row;
+    const int c8 = (int)(it - row * per_row) * 8;
+    const int64_t t = row / p.n_kv_heads;
+    const int h = (int)(row - t * p.n_kv_heads);
+    const uint4 raw = *reinterpret_cast<const uint4*>(p.v_src + t * p.v_stride_tok + h * p.v_stride_head + c8);
+    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int x = 0; x < 4; ++x) {
+      const float lo = bf16lo_to_f32(w[x]), hi = bf16hi_to_f32(w[x]);
+      over |= (fabsf(lo) > 65504.f && fabsf(lo) <= 3.402823466e38f) ||
+              (fabsf(hi) > 65504.f && fabsf(hi) <= 3.402823466e38f);
+      o[x] = pack_f16x2(lo, hi);
+    }
+    *reinterpret_cast<uint4*>(p.v_half + row * head_dim + c8) = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+  if (__any_sync(0xffffffffu, over) && (threadIdx.x & 31) == 0) atomicOr(p.v_overflow, 1u);
+}
 using score::load_row;
 using score::row_max_regs;
 
@@ -94,7 +165,8 @@ __device__ __forceinline__ void p1_cta_coords(int cta, int ctas_per_g, int& g, i
 template <int D, int BN>
 __global__ void __launch_bounds__(P1Cfg<D, BN>::kThreads, 1)
     poem_score_pass1_kernel(const __grid_constant__ CUtensorMap tmQs, const __grid_constant__ CUtensorMap tmK,
-                            const __grid_constant__ CUtensorMap tmV, const ScoreParams p) {
+                            const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmVh,
+                            const ScoreParams p) {
   using C = P1Cfg<D, BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -115,6 +187,8 @@ __global__ void __launch_bounds__(P1Cfg<D, BN>::kThreads, 1)
   const int t0 = p.q_tile0;
   const int nb = z_last / G + 1 + t0;  // key blocks 0 .. largest (global) tile of the CTA
   const int i_lo = z0 / G + t0;        // blocks < i_lo need no causal mask
+  // fp16 P for this CTA (uniform): all its tiles >= 32 and V inside fp16's range
+  const bool half_p = (i_lo >= C::kHalfMinTile) && (*p.v_overflow == 0);
 
   if (tid == 0) {
     mbar_init(&sb->q_full, 1);
@@ -147,7 +221,8 @@ __global__ void __launch_bounds__(P1Cfg<D, BN>::kThreads, 1)
     if (lane == 0) {
       tma_prefetch_desc(&tmQs);
       tma_prefetch_desc(&tmK);
-      tma_prefetch_desc(&tmV);
+      const CUtensorMap* mapV = half_p ? &tmVh : &tmV;  // 2-byte elements either way
+      tma_prefetch_desc(mapV);
       mbar_arrive_expect_tx(&sb->q_full, C::kQBytes);
       for (int zl = 0; zl < C::kGroups; ++zl) {
         const int z = z0 + zl;  // groups past the end read out-of-range tiles: zero-filled
@@ -174,7 +249,7 @@ __global__ void __launch_bounds__(P1Cfg<D, BN>::kThreads, 1)
           const int s = vb & 1;
           mbar_arrive_expect_tx(&sb->v_full[s], C::kKVBytes);
           for (int c = 0; c < C::kChunks; ++c)
-            tma_load_3d(sV + s * C::kKVBytes + c * (BN * 128), &tmV, &sb->v_full[s], c * 64, g, vb * BN);
+            tma_load_3d(sV + s * C::kKVBytes + c * (BN * 128), mapV, &sb->v_full[s], c * 64, g, vb * BN);
           ++vb;
           progressed = true;
         }
@@ -203,12 +278,21 @@ __global__ void __launch_bounds__(P1Cfg<D, BN>::kThreads, 1)
       tc_fence_after();
       const uint32_t tP = tmem + s * 128;
       const uint32_t aVs = aV + sv * C::kKVBytes;
+      if (half_p) {
 #pragma unroll
-      for (int kk = 0; kk < BN / 16; ++kk) {
-        // keys [16 kk, 16 kk + 16): P_hi words at [16 kk, +8), P_lo at [16 kk + 8, +8)
-        const uint64_t bdesc = smem_desc_sw128(aVs + kk * 2048, BN * 128, 1024);
-        mma_ts_warp(tO, tP + kk * 16, bdesc, C::kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
-        mma_ts_warp(tO, tP + kk * 16 + 8, bdesc, C::kIdescPV, 1u);
+        for (int kk = 0; kk < BN / 16; ++kk) {
+          // keys [16 kk, 16 kk + 16): fp16 P words at [8 kk, +8)
+          const uint64_t bdesc = smem_desc_sw128(aVs + kk * 2048, BN * 128, 1024);
+          mma_ts_warp(tO, tP + kk * 8, bdesc, C::kIdescPVh, (j > 0 || kk > 0) ? 1u : 0u);
+        }
+      } else {
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk) {
+          // keys [16 kk, 16 kk + 16): P_hi words at [16 kk, +8), P_lo at [16 kk + 8, +8)
+          const uint64_t bdesc = smem_desc_sw128(aVs + kk * 2048, BN * 128, 1024);
+          mma_ts_warp(tO, tP + kk * 16, bdesc, C::kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
+          mma_ts_warp(tO, tP + kk * 16 + 8, bdesc, C::kIdescPV, 1u);
+        }
       }
       mma_commit_warp(&sb->v_empty[sv]);
       mma_commit_warp(&sb->acc_full[j & 1]);
@@ -285,9 +369,15 @@ __global__ void __launch_bounds__(P1Cfg<D, BN>::kThreads, 1)
         }
       }
       l_run *= alpha;
-      const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
-      l_run += (b < i_lo) ? exp_split_store_regs<BN, false>(tS, a, sl2, m_use, lim)
-                          : exp_split_store_regs<BN, true>(tS, a, sl2, m_use, lim);
+      // reference of the weights: the running max, lowered by 6 for fp16 P so that
+      // P <= 2^14 and weights down to 2^-20 of the reference keep full fp16 precision
+      const float m_use = (m_run == -INFINITY) ? 0.f : (half_p ? m_run - 6.0f : m_run);
+      if (half_p)
+        l_run += (b < i_lo) ? exp_f16_store_regs<BN, false>(tS, a, sl2, m_use, lim)
+                            : exp_f16_store_regs<BN, true>(tS, a, sl2, m_use, lim);
+      else
+        l_run += (b < i_lo) ? exp_split_store_regs<BN, false>(tS, a, sl2, m_use, lim)
+                            : exp_split_store_regs<BN, true>(tS, a, sl2, m_use, lim);
       tmem_st_wait();
       tc_fence_before();
       warp_arrive(&sb->p_full[s]);
@@ -312,7 +402,8 @@ __global__ void __launch_bounds__(P1Cfg<D, BN>::kThreads, 1)
                                 __uint_as_float(ov[4 * x + 2]) * inv_l, __uint_as_float(ov[4 * x + 3]) * inv_l);
         }
       }
-      if (valid && in_ws) p.ws_lse[srow] = (l_run > 0.f) ? m_run + __log2f(l_run) : -INFINITY;
+      const float m_use = (m_run == -INFINITY) ? 0.f : (half_p ? m_run - 6.0f : m_run);
+      if (valid && in_ws) p.ws_lse[srow] = (l_run > 0.f) ? m_use + __log2f(l_run) : -INFINITY;
     }
   }
 
@@ -327,22 +418,33 @@ __global__ void __launch_bounds__(P1Cfg<D, BN>::kThreads, 1)
 
 template <int D, int BN>
 cudaError_t launch_p1_t(const CUtensorMap& tmQs, const CUtensorMap& tmK, const CUtensorMap& tmV,
-                        const ScoreParams& p, int grid, cudaStream_t stream) {
+                        const CUtensorMap& tmVh, const ScoreParams& p, int grid, cudaStream_t stream) {
   using C = P1Cfg<D, BN>;
   cudaError_t e = ensure_smem_limit(poem_score_pass1_kernel<D, BN>, C::kSmemBytes);
   if (e != cudaSuccess) return e;
-  poem_score_pass1_kernel<D, BN><<<grid, C::kThreads, C::kSmemBytes, stream>>>(tmQs, tmK, tmV, p);
+  poem_score_pass1_kernel<D, BN><<<grid, C::kThreads, C::kSmemBytes, stream>>>(tmQs, tmK, tmV, tmVh, p);
   return cudaGetLastError();
 }
 
 }  // namespace
 
+cudaError_t launch_v_to_half(const ScoreParams& p, int head_dim, cudaStream_t stream) {
+  cudaError_t e = cudaMemsetAsync(p.v_overflow, 0, sizeof(uint32_t), stream);
+  if (e != cudaSuccess) return e;
+  const int64_t items = (int64_t)p.n_kv * p.n_kv_heads * (head_dim / 8);
+  const int64_t want = (items + 255) / 256;
+  const int grid = (int)(want < 148 * 16 ? (want > 0 ? want : 1) : 148 * 16);
+  v_to_half_kernel<<<grid, 256, 0, stream>>>(p, head_dim);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_score_pass1(int head_dim, int block, const CUtensorMap& tmQs, const CUtensorMap& tmK,
-                               const CUtensorMap& tmV, const ScoreParams& p, int grid, cudaStream_t stream) {
-  if (head_dim == 128 && block == 128) return launch_p1_t<128, 128>(tmQs, tmK, tmV, p, grid, stream);
-  if (head_dim == 128 && block == 64) return launch_p1_t<128, 64>(tmQs, tmK, tmV, p, grid, stream);
-  if (head_dim == 64 && block == 128) return launch_p1_t<64, 128>(tmQs, tmK, tmV, p, grid, stream);
-  if (head_dim == 64 && block == 64) return launch_p1_t<64, 64>(tmQs, tmK, tmV, p, grid, stream);
+                               const CUtensorMap& tmV, const CUtensorMap& tmVh, const ScoreParams& p, int grid,
+                               cudaStream_t stream) {
+  if (head_dim == 128 && block == 128) return launch_p1_t<128, 128>(tmQs, tmK, tmV, tmVh, p, grid, stream);
+  if (head_dim == 128 && block == 64) return launch_p1_t<128, 64>(tmQs, tmK, tmV, tmVh, p, grid, stream);
+  if (head_dim == 64 && block == 128) return launch_p1_t<64, 128>(tmQs, tmK, tmV, tmVh, p, grid, stream);
+  if (head_dim == 64 && block == 64) return launch_p1_t<64, 64>(tmQs, tmK, tmV, tmVh, p, grid, stream);
   return cudaErrorInvalidValue;
 }
 

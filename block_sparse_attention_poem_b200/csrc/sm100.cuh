@@ -230,6 +230,18 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(uint32_t M, uint32_t N, ui
   return (1u << 4) | (1u << 7) | (1u << 10) | (b_mn_major << 16) | ((N >> 3) << 17) | ((M >> 4) << 24);
 }
 
+// Instruction descriptor, kind::f16 with fp16 A/B and fp32 D (A/B format 0 = f16).
+__host__ __device__ constexpr uint32_t idesc_f16_f32(uint32_t M, uint32_t N, uint32_t b_mn_major) {
+  return (1u << 4) | (b_mn_major << 16) | ((N >> 3) << 17) | ((M >> 4) << 24);
+}
+
+// Round two floats to fp16 (nearest-even) and pack: lo in bits [0,16), hi in [16,32).
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
 // Shared-memory matrix descriptor for a 128-byte-swizzled operand.
 // start: byte address; lbo/sbo: leading / stride byte offsets; version 1 (sm_100);
 // layout type 2 = SWIZZLE_128B.

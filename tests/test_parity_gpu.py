@@ -329,6 +329,9 @@ SCORE_CASES = [
     (1280, 5, 1, 128, 128, 1000000.0, 1),   # 5-way GQA: packed groups straddle tiles
     (1024, 8, 2, 128, 128, 500000.0, 2),
     (1024, 2, 1, 64, 64, 10000.0, 3),
+    # more than 32 tiles: the CTAs beyond tile 32 take pass 1's fp16 P V contraction
+    (6400, 5, 1, 128, 128, 1000000.0, 4),
+    (4096, 2, 1, 64, 64, 10000.0, 5),
 ]
 
 
@@ -383,17 +386,27 @@ def test_score_shift_invariance(poem):
     assert np.array_equal(m0, m1)
 
 
-def test_score_large_value_range(poem):
-    """Values scaled by powers of two up to 2^16 (far beyond unit scale): the scores
-    scale with V and still match the oracle (the P V contraction keeps V in bf16)."""
-    x = poem_synth.heavy_block_layer(2048, 4, 1, 128, block=128, seed=21)
-    for scale in (2.0 ** -8, 2.0 ** 16):
+def test_score_values_beyond_fp16_range_take_the_bf16_contraction(poem):
+    """Pass 1 runs the P V contraction of CTAs whose tiles are all >= 32 with one fp16 P
+    on an fp16 copy of V.  A finite |v| above the fp16 maximum (65504) sets the range
+    flag in the score workspace (byte 8) and every CTA takes the bf16 hi/lo
+    contraction; both give oracle scores (64 tiles: CTAs on both sides of tile 32)."""
+    x = poem_synth.heavy_block_layer(8192, 4, 1, 128, block=128, seed=21)
+    for scale, flag in ((1.0, 0), (2.0 ** -8, 0), (2.0 ** 16, 1)):
         xs = dict(x)
         xs["v"] = (x["v"].float() * scale).to(torch.bfloat16)  # a power of two: exact in bf16
-        Ig, mg, status = _gpu_score(poem, xs, 128)
-        assert status == 0
+        q, k, v = to_dev(xs)
+        shape = poem.make_shape(q, k, block=128)
+        ne = poem.n_score_entries(4, 64)
+        Ih = torch.full((ne,), float("nan"), device="cuda")
+        mh = torch.full((ne,), float("nan"), device="cuda")
+        s_b, _, _ = poem.poem_workspace_size(shape)
+        ws = poem.alloc_workspace(s_b)
+        poem.poem_score(q, k, v, Ih, mh, ws, shape=shape)
+        assert poem.poem_check_status(ws) == 0
+        assert int(ws[8:12].view(torch.int32).item()) == flag, scale
         Ir, mr = problem_from(xs, 128).score_all()
-        assert score_err_excess(Ig, Ir, mg, mr, max_value_norm(xs["v"])) <= 1.0, scale
+        assert score_err_excess(Ih.cpu().numpy(), Ir, mh.cpu().numpy(), mr, max_value_norm(xs["v"])) <= 1.0, scale
 
 
 # ---------------------------------------------------------------------------
