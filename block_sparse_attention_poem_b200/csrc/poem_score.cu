@@ -26,15 +26,14 @@
 // and its score row has q_tile0 + i + 1 entries (row_off layout).
 //
 // Pass 2 pipeline (one CTA per SM, TMEM fully allocated):
-//   TMEM  S0 [0,128)  S1 [128,256)  -- S double-buffered: S_{b+1} is computed while
-//                                      the softmax of block b runs
-//         accumulators [256,384) and [384,512): P_b V_b of block b goes to
-//         accumulator b % 2, double-buffered for the norm warps
+//   TMEM  S buffers s = 0, 1, 2 at [128 s, 128 s + BN): the MMAs run up to two blocks
+//         ahead of the softmax; the P_b V_b accumulator at [384, 384 + D), read by the
+//         norm warps while the next blocks' S are computed
 //   smem  Q tile, 3-stage K ring, 2-stage V ring (192 KB at d = 128)
 //   warps 0-3 softmax, warps 4-7 the norm of P_b V_b - m_b o with o held in
-//   registers; warp 8 issues TMA loads; warp 9 issues the MMAs, converged, from one
-//   elected lane.
-//   MMA order: S_0, S_1, PV_0, S_2, PV_1, ...
+//   registers; warp 8 issues TMA loads (K and V rings independently); warp 9 issues
+//   the MMAs, converged, from one elected lane.
+//   MMA order: S_0, S_1, S_2, PV_0, S_3, PV_1, ...
 //
 // Precision: P enters the P V contraction as a hi/lo pair of bf16 matrices
 // (P = P_hi + P_lo, two MMAs into the same accumulator), about 16 significant
@@ -68,8 +67,8 @@ struct ScoreCfg {
   // at least 120 KB so that one CTA (holding all 512 TMEM columns) occupies an SM
   static constexpr int kSmemBytes = (kOffM + 2 * 128 * 4 + 1024) > 122880 ? (kOffM + 2 * 128 * 4 + 1024) : 122880;
   static constexpr uint32_t kTmemCols = 512;
-  static constexpr uint32_t kColS = 0;     // S buffer s at [128 s, 128 s + BN)
-  static constexpr uint32_t kColAcc = 256; // accumulator s at [256 + 128 s, 256 + 128 s + D)
+  static constexpr uint32_t kColS = 0;     // S buffer s (0, 1, 2) at [128 s, 128 s + BN)
+  static constexpr uint32_t kColAcc = 384; // P_b V_b accumulator at [384, 384 + D)
   static constexpr int kWarpProd = 8;      // warps 0-3 softmax, 4-7 norm, 8 TMA, 9 MMA
   static constexpr int kWarpMma = 9;
   static constexpr int kThreads = 320;
@@ -80,8 +79,8 @@ struct ScoreCfg {
 struct ScoreBarriers {
   uint64_t q_full;
   uint64_t k_full[3], k_empty[3], v_full[2], v_empty[2];
-  uint64_t s_full[2], p_full[2];
-  uint64_t acc_full[2], acc_empty[2];  // accumulator s done / released by the norm warps (pass 2)
+  uint64_t s_full[3], p_full[3];
+  uint64_t acc_full, acc_empty;  // P_b V_b complete / read by the norm warps
   uint64_t m_ready[2], m_empty[2];
   uint64_t drain;
   uint32_t tmem_base;
@@ -151,17 +150,17 @@ __global__ void __launch_bounds__(ScoreCfg<D, BN>::kThreads, 1)
     for (int s = 0; s < 3; ++s) {
       mbar_init(&sb->k_full[s], 1);
       mbar_init(&sb->k_empty[s], 1);
+      mbar_init(&sb->s_full[s], 1);
+      mbar_init(&sb->p_full[s], 4);  // barriers signalled by 4 warps: one arrival per warp
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&sb->v_full[s], 1);
       mbar_init(&sb->v_empty[s], 1);
-      mbar_init(&sb->s_full[s], 1);
-      mbar_init(&sb->p_full[s], 4);  // barriers signalled by 4 warps: one arrival per warp
-      mbar_init(&sb->acc_full[s], 1);
-      mbar_init(&sb->acc_empty[s], 4);
       mbar_init(&sb->m_ready[s], 4);
       mbar_init(&sb->m_empty[s], 4);
     }
+    mbar_init(&sb->acc_full, 1);
+    mbar_init(&sb->acc_empty, 4);
     mbar_init(&sb->drain, 1);
     sb->abort_flag = 0;
     fence_barrier_init();
@@ -187,47 +186,60 @@ __global__ void __launch_bounds__(ScoreCfg<D, BN>::kThreads, 1)
           tma_load_4d(sQ + c * (C::M * 128) + zl * (C::kRowsPerGroup * 128), &tmQs, &sb->q_full, c * 64, hq, 0,
                       i);
       }
-      int k_issued = 0, v_issued = 0;
-      for (int b = 0; b < nb && !sb->abort_flag; ++b) {
-        // stage of block b and the completion of its empty barrier to wait for
-        // (#(b / stages - 1); a fresh barrier passes the parity-1 wait at once)
-        const int sk = b % C::kStagesK, sv = b & 1;
-        if (!wait_or_abort(&sb->k_empty[sk], ((b / C::kStagesK) & 1) ^ 1, sb, p.err)) break;
-        mbar_arrive_expect_tx(&sb->k_full[sk], C::kKVBytes);
-        for (int c = 0; c < C::kChunks; ++c)
-          tma_load_3d(sK + sk * C::kKVBytes + c * (BN * 128), &tmK, &sb->k_full[sk], c * 64, g, b * BN);
-        ++k_issued;
-        if (!wait_or_abort(&sb->v_empty[sv], ((b >> 1) & 1) ^ 1, sb, p.err)) break;
-        mbar_arrive_expect_tx(&sb->v_full[sv], C::kKVBytes);
-        for (int c = 0; c < C::kChunks; ++c)
-          tma_load_3d(sV + sv * C::kKVBytes + c * (BN * 128), &tmV, &sb->v_full[sv], c * 64, g, b * BN);
-        ++v_issued;
+      // K and V rings advance independently: K_b is loaded once S_{b-3} has released
+      // its stage, V_b once P V_{b-2} has.
+      int kb = 0, vb = 0;
+      uint64_t t_last = globaltimer_ns();
+      while ((kb < nb || vb < nb) && !sb->abort_flag) {
+        bool progressed = false;
+        // a fresh stage passes the parity-1 test at once; later, completion #(b/stages - 1)
+        if (kb < nb && mbar_try_wait(&sb->k_empty[kb % 3], ((kb / 3) & 1) ^ 1)) {
+          const int st = kb % 3;
+          mbar_arrive_expect_tx(&sb->k_full[st], C::kKVBytes);
+          for (int c = 0; c < C::kChunks; ++c)
+            tma_load_3d(sK + st * C::kKVBytes + c * (BN * 128), &tmK, &sb->k_full[st], c * 64, g, kb * BN);
+          ++kb;
+          progressed = true;
+        }
+        if (vb < kb && mbar_try_wait(&sb->v_empty[vb & 1], ((vb >> 1) & 1) ^ 1)) {
+          const int st = vb & 1;
+          mbar_arrive_expect_tx(&sb->v_full[st], C::kKVBytes);
+          for (int c = 0; c < C::kChunks; ++c)
+            tma_load_3d(sV + st * C::kKVBytes + c * (BN * 128), &tmV, &sb->v_full[st], c * 64, g, vb * BN);
+          ++vb;
+          progressed = true;
+        }
+        if (progressed) {
+          t_last = globaltimer_ns();
+        } else if (globaltimer_ns() - t_last > p.err.timeout_ns) {
+          sb->abort_flag = 1;
+          raise_err(p.err, kErrTimeout);
+          break;
+        }
       }
       // Drain: the last load issued into each stage must have landed.
       mbar_wait(&sb->q_full, 0, kDrainNs);
-      for (int b = max(0, k_issued - C::kStagesK); b < k_issued; ++b)
-        mbar_wait(&sb->k_full[b % C::kStagesK], (b / C::kStagesK) & 1, kDrainNs);
-      for (int b = max(0, v_issued - 2); b < v_issued; ++b) mbar_wait(&sb->v_full[b & 1], (b >> 1) & 1, kDrainNs);
+      for (int x = max(0, kb - 3); x < kb; ++x) mbar_wait(&sb->k_full[x % 3], (x / 3) & 1, kDrainNs);
+      for (int x = max(0, vb - 2); x < vb; ++x) mbar_wait(&sb->v_full[x & 1], (x >> 1) & 1, kDrainNs);
     }
   } else if (warp == C::kWarpMma) {
     // ============================ MMA issuer ============================
     // The whole warp runs this loop converged (waits and operands are warp-uniform);
     // one elected lane issues each MMA and commit.
-    // Order S_0, S_1, PV_0, S_2, PV_1, ...: S_b lands in S buffer b % 2 and P_b V_b in
-    // accumulator b % 2, started fresh once the norm warps have read the accumulator's
-    // previous block (b - 2).
+    // Order S_0, S_1, S_2, PV_0, S_3, PV_1, ...: S_b lands in S buffer b % 3 (free once
+    // P V_{b-3}, issued just before, has read it), P_b V_b in the accumulator, started
+    // fresh once the norm warps have read P V_{b-1}.
     const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV);
+    const uint32_t tAcc = tmem + C::kColAcc;
     bool ok = warp_wait(&sb->q_full, 0, sb, p.err);
     auto issue_pv = [&](int j) -> bool {
-      const int s = j & 1;
-      const uint32_t par = (j >> 1) & 1;
-      if (!warp_wait(&sb->p_full[s], par, sb, p.err)) return false;
-      if (!warp_wait(&sb->v_full[s], par, sb, p.err)) return false;
-      if (j >= 2 && !warp_wait(&sb->acc_empty[s], par ^ 1, sb, p.err)) return false;
+      const int s = j % 3, sv = j & 1;
+      if (!warp_wait(&sb->p_full[s], (j / 3) & 1, sb, p.err)) return false;
+      if (!warp_wait(&sb->v_full[sv], (j >> 1) & 1, sb, p.err)) return false;
+      if (j >= 1 && !warp_wait(&sb->acc_empty, (j - 1) & 1, sb, p.err)) return false;
       tc_fence_after();
       const uint32_t tP = tmem + C::kColS + s * 128;
-      const uint32_t tAcc = tmem + C::kColAcc + s * 128;
-      const uint32_t aVs = aV + s * C::kKVBytes;
+      const uint32_t aVs = aV + sv * C::kKVBytes;
 #pragma unroll
       for (int kk = 0; kk < BN / 16; ++kk) {
         // keys [16 kk, 16 kk + 16): P_hi words at [16 kk, +8), P_lo at [16 kk + 8, +8)
@@ -235,17 +247,17 @@ __global__ void __launch_bounds__(ScoreCfg<D, BN>::kThreads, 1)
         mma_ts_warp(tAcc, tP + kk * 16, bdesc, C::kIdescPV, kk > 0 ? 1u : 0u);
         mma_ts_warp(tAcc, tP + kk * 16 + 8, bdesc, C::kIdescPV, 1u);
       }
-      mma_commit_warp(&sb->v_empty[s]);
-      mma_commit_warp(&sb->acc_full[s]);
+      mma_commit_warp(&sb->v_empty[sv]);
+      mma_commit_warp(&sb->acc_full);
       return true;
     };
     for (int b = 0; b < nb && ok; ++b) {
-      const int s = b & 1;
-      const int sk = b % C::kStagesK;
-      if (!warp_wait(&sb->k_full[sk], (b / C::kStagesK) & 1, sb, p.err)) { ok = false; break; }
+      if (b >= 3 && !issue_pv(b - 3)) { ok = false; break; }
+      const int s = b % 3;
+      if (!warp_wait(&sb->k_full[s], (b / 3) & 1, sb, p.err)) { ok = false; break; }
       tc_fence_after();
       const uint32_t tS = tmem + C::kColS + s * 128;
-      const uint32_t aKs = aK + sk * C::kKVBytes;
+      const uint32_t aKs = aK + s * C::kKVBytes;
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
         const uint32_t koff = (kk & 3) * 32;
@@ -254,10 +266,10 @@ __global__ void __launch_bounds__(ScoreCfg<D, BN>::kThreads, 1)
         mma_ss_warp(tS, adesc, bdesc, C::kIdescQK, kk > 0 ? 1u : 0u);
       }
       mma_commit_warp(&sb->s_full[s]);
-      mma_commit_warp(&sb->k_empty[sk]);
-      if (b > 0 && !issue_pv(b - 1)) { ok = false; break; }
+      mma_commit_warp(&sb->k_empty[s]);
     }
-    if (ok && nb > 0) issue_pv(nb - 1);
+    for (int j = max(0, nb - 3); j < nb && ok; ++j)
+      if (!issue_pv(j)) ok = false;
     mma_commit_warp(&sb->drain);
     mbar_wait(&sb->drain, 0, kDrainNs);
   } else if (warp < 4) {
@@ -277,17 +289,17 @@ __global__ void __launch_bounds__(ScoreCfg<D, BN>::kThreads, 1)
     const float lse2 = (valid && in_ws) ? p.ws_lse[srow] : 0.f;
     bool ok = true;
     for (int b = 0; b < nb; ++b) {
-      const int s = b & 1;
+      const int s = b % 3, sm = b & 1;
       const uint32_t tS = tmem + lane_off + C::kColS + s * 128;
-      if (!warp_wait(&sb->s_full[s], (b >> 1) & 1, sb, p.err)) { ok = false; break; }
+      if (!warp_wait(&sb->s_full[s], (b / 3) & 1, sb, p.err)) { ok = false; break; }
       tc_fence_after();
       const int lim = qpos - b * BN;
       const float msum = (b < i_lo) ? exp_split_store<BN, false>(tS, sl2, lse2, lim)
                                     : exp_split_store<BN, true>(tS, sl2, lse2, lim);
-      // hand m_b to the norm warps (slot s is free once block b-2's norm read it)
-      if (b >= 2 && !warp_wait(&sb->m_empty[s], ((b >> 1) & 1) ^ 1, sb, p.err)) ok = false;
-      sm_m[s * 128 + r] = valid ? msum : 0.f;
-      warp_arrive(&sb->m_ready[s]);
+      // hand m_b to the norm warps (slot b % 2 is free once block b-2's norm read it)
+      if (b >= 2 && !warp_wait(&sb->m_empty[sm], ((b >> 1) & 1) ^ 1, sb, p.err)) ok = false;
+      sm_m[sm * 128 + r] = valid ? msum : 0.f;
+      warp_arrive(&sb->m_ready[sm]);
       tmem_st_wait();
       tc_fence_before();
       warp_arrive(&sb->p_full[s]);
@@ -322,13 +334,12 @@ __global__ void __launch_bounds__(ScoreCfg<D, BN>::kThreads, 1)
     const int64_t tri = row_off(p.n_tiles, t0, hq, i);
     for (int b = 0; b < nb; ++b) {
       const int s = b & 1;
-      const uint32_t par = (b >> 1) & 1;
-      if (!warp_wait(&sb->acc_full[s], par, sb, p.err)) break;
-      if (!warp_wait(&sb->m_ready[s], par, sb, p.err)) break;
+      if (!warp_wait(&sb->acc_full, b & 1, sb, p.err)) break;
+      if (!warp_wait(&sb->m_ready[s], (b >> 1) & 1, sb, p.err)) break;
       tc_fence_after();
       const float mb_row = sm_m[s * 128 + r];
       warp_arrive(&sb->m_empty[s]);
-      const uint32_t tAcc = tmem + lane_off + C::kColAcc + s * 128;
+      const uint32_t tAcc = tmem + lane_off + C::kColAcc;
       const uint64_t negm2 = f2_pack(-mb_row, -mb_row);
       uint64_t acc2 = f2_pack(0.f, 0.f);
 #pragma unroll
@@ -344,9 +355,9 @@ __global__ void __launch_bounds__(ScoreCfg<D, BN>::kThreads, 1)
           acc2 = f2_fma(e, e, acc2);
         }
       }
-      // P V_b has been read: the accumulator may take block b + 2.
+      // P V_b has been read: the accumulator may take block b + 1.
       tc_fence_before();
-      warp_arrive(&sb->acc_empty[s]);
+      warp_arrive(&sb->acc_empty);
       float a0, a1;
       f2_unpack(acc2, a0, a1);
       float Ib = valid ? sqrtf(a0 + a1) : 0.f;
