@@ -19,7 +19,7 @@
 //              max grows by more than 2^8, epilogue).
 //   warp 8     TMA producer: Q_A and Q_B once, then K_b, V_b for every block b of the
 //              union, in ascending order, into a ring of shared-memory slots.
-//   warp 9     MMA issuer (one thread).  At each union block b, for head x = A, B:
+//   warp 9     MMA issuer (converged warp; one elected lane issues).  At each union block b, for head x = A, B:
 //              first O_x += P_x V_x for x's previous block (if one is pending), then,
 //              if b is in x's list, S_x = Q_x K_b^T.  A head's P V therefore waits at
 //              most one union step, so each V tile is released one step after its
@@ -72,6 +72,7 @@ using fwd::block_ok;
 using fwd::exp_pack_store;
 using fwd::kDrainNs;
 using fwd::wait_or_abort;
+using fwd::warp_wait_or_abort;
 
 // The two rows of a CTA: query heads 2p and 2p + 1 of KV group g at local tile i.
 struct PairRow {
@@ -204,7 +205,9 @@ __global__ void __launch_bounds__(kThreadsGrouped, 1)
     }
   } else if (warp == 9) {
     // ============================ MMA issuer ============================
-    if (lane == 0) {
+    // The whole warp runs the schedule converged (list entries, waits and operands are
+    // warp-uniform); one elected lane issues each MMA and commit.
+    {
       int hk = 0;
       const PairRow R[2] = {pair_row(p, unit, 0, &hk, false), pair_row(p, unit, 1, &hk, false)};
       const uint32_t aRing = smem_u32(sRing);
@@ -216,7 +219,7 @@ __global__ void __launch_bounds__(kThreadsGrouped, 1)
       bool pend_rel[2] = {false, false};  // whether that P V is the V tile's last use
       bool ok = true;
       auto wait_tile = [&](int n) -> bool {
-        return wait_or_abort(&sb->slot_full[n % C::kSlots], (n / C::kSlots) & 1, sb, p.err);
+        return warp_wait_or_abort(&sb->slot_full[n % C::kSlots], (n / C::kSlots) & 1, sb, p.err);
       };
       // O_x += P_x V (in two 64-key halves, each as soon as that half of P_x is written)
       auto issue_pv = [&](int x) -> bool {
@@ -227,25 +230,25 @@ __global__ void __launch_bounds__(kThreadsGrouped, 1)
         const uint32_t tO = tS + 128u;
 #pragma unroll
         for (int hv = 0; hv < BN / 64; ++hv) {
-          if (!wait_or_abort(&sb->p_half[x][hv], k[x] & 1, sb, p.err)) return false;
+          if (!warp_wait_or_abort(&sb->p_half[x][hv], k[x] & 1, sb, p.err)) return false;
           tc_fence_after();
 #pragma unroll
           for (int kk = hv * 4; kk < hv * 4 + 4; ++kk) {
             // V tile is MN-major (d contiguous): LBO = stride between 64-wide d chunks,
             // SBO = stride between 8-key groups; a k-step covers 16 keys = 2 groups.
             const uint64_t bdesc = smem_desc_sw128(aV + kk * 2048, BN * 128, 1024);
-            mma_ts(tO, tS + kk * 8, bdesc, C::kIdescPV, (k[x] > 0 || kk > 0) ? 1u : 0u);
+            mma_ts_warp(tO, tS + kk * 8, bdesc, C::kIdescPV, (k[x] > 0 || kk > 0) ? 1u : 0u);
           }
         }
-        if (pend_rel[x]) mma_commit(&sb->slot_empty[n % C::kSlots]);
+        if (pend_rel[x]) mma_commit_warp(&sb->slot_empty[n % C::kSlots]);
         ++k[x];
         pend[x] = false;
-        if (e[x] >= R[x].end) mma_commit(&sb->o_full[x]);  // that was the head's last block
+        if (e[x] >= R[x].end) mma_commit_warp(&sb->o_full[x]);  // that was the head's last block
         return true;
       };
       // S_x = Q_x K^T with the K tile of load index n
       auto issue_qk = [&](int x, int n, bool release) -> bool {
-        if (nq[x] == 0 && !wait_or_abort(&sb->q_full[x], 0, sb, p.err)) return false;
+        if (nq[x] == 0 && !warp_wait_or_abort(&sb->q_full[x], 0, sb, p.err)) return false;
         if (!wait_tile(n)) return false;
         tc_fence_after();
         const uint32_t aQ = smem_u32(smem + C::kOffQ + x * C::kQBytes);
@@ -258,10 +261,10 @@ __global__ void __launch_bounds__(kThreadsGrouped, 1)
           const uint32_t koff = (kk & 3) * 32;
           const uint64_t adesc = smem_desc_sw128(aQ + (kk >> 2) * (C::M * 128) + koff, 16, 1024);
           const uint64_t bdesc = smem_desc_sw128(aK + (kk >> 2) * (BN * 128) + koff, 16, 1024);
-          mma_ss(tS, adesc, bdesc, C::kIdescQK, kk > 0 ? 1u : 0u);
+          mma_ss_warp(tS, adesc, bdesc, C::kIdescQK, kk > 0 ? 1u : 0u);
         }
-        mma_commit(&sb->s_full[x]);
-        if (release) mma_commit(&sb->slot_empty[n % C::kSlots]);
+        mma_commit_warp(&sb->s_full[x]);
+        if (release) mma_commit_warp(&sb->slot_empty[n % C::kSlots]);
         ++nq[x];
         return true;
       };
@@ -286,8 +289,8 @@ __global__ void __launch_bounds__(kThreadsGrouped, 1)
       }
       for (int x = 0; x < 2 && ok; ++x)
         if (pend[x]) ok = issue_pv(x);
-      // Drain every MMA this thread issued before TMEM is released.
-      mma_commit(&sb->drain);
+      // Drain every MMA this warp issued before TMEM is released.
+      mma_commit_warp(&sb->drain);
       mbar_wait(&sb->drain, 0, kDrainNs);
     }
   } else {

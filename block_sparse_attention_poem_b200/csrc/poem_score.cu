@@ -35,10 +35,14 @@
 //   the MMAs, converged, from one elected lane.
 //   MMA order: S_0, S_1, S_2, PV_0, S_3, PV_1, ...
 //
-// Precision: P enters the P V contraction as a hi/lo pair of bf16 matrices
-// (P = P_hi + P_lo, two MMAs into the same accumulator), about 16 significant
-// bits, so that o, r_b and I_b keep ~1e-6 relative accuracy; a single bf16 P
-// gives ~1e-3 and would move near-tied blocks across the selection cut.
+// Precision: on a CTA's first query tiles (below score::kHalfMinTile) P enters the
+// P V contraction as a hi/lo pair of bf16 matrices (P = P_hi + P_lo, two MMAs into
+// the same accumulator), about 16 significant bits: there one or a few blocks hold
+// nearly all of a query's mass and r_b cancels almost exactly.  Later CTAs take one
+// fp16 P (11 significant bits, scaled by 2^6 so that small weights stay normal)
+// against the fp16 copy of V: r_b's rounding error is then ~1e-5 m_b |v|, inside
+// the score tolerance.  A single bf16 P (8 bits) would move near-tied blocks across
+// the selection cut.  m_b always sums the unrounded fp32 weights.
 //
 // Every mbarrier wait below is made at most one phase behind the barrier (each
 // wait's completion is a precondition of the barrier's next phase), so parity
@@ -74,6 +78,8 @@ struct ScoreCfg {
   static constexpr int kThreads = 320;
   static constexpr uint32_t kIdescQK = idesc_bf16_f32(M, BN, 0);
   static constexpr uint32_t kIdescPV = idesc_bf16_f32(M, D, 1);
+  static constexpr uint32_t kIdescPVh = idesc_f16_f32(M, D, 1);  // fp16 P x fp16 V
+  static constexpr float kHalfScaleLog2 = 6.0f;                  // fp16 P holds 2^6 p
 };
 
 struct ScoreBarriers {
@@ -116,13 +122,15 @@ __device__ __forceinline__ void score_cta_coords(int cta, int ctas_per_g, int& g
   z0 = c * 8;
 }
 
+using score::exp_f16_store_regs;
 using score::exp_split_store;
-using score::row_max;
+using score::load_row;
 
 template <int D, int BN>
 __global__ void __launch_bounds__(ScoreCfg<D, BN>::kThreads, 1)
     poem_score_pass2_kernel(const __grid_constant__ CUtensorMap tmQs, const __grid_constant__ CUtensorMap tmK,
-                      const __grid_constant__ CUtensorMap tmV, const ScoreParams p) {
+                      const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmVh,
+                      const ScoreParams p) {
   using C = ScoreCfg<D, BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -144,6 +152,8 @@ __global__ void __launch_bounds__(ScoreCfg<D, BN>::kThreads, 1)
   const int t0 = p.q_tile0;            // global index of local query tile 0
   const int nb = z_last / G + 1 + t0;  // key blocks 0 .. largest (global) tile of the CTA
   const int i_lo = z0 / G + t0;        // smallest global tile of the CTA: blocks < i_lo need no mask
+  // the fp16 copy of V was written (and its range flag set) before pass 1 ran
+  const bool half_p = (i_lo >= score::kHalfMinTile) && (*p.v_overflow == 0);
 
   if (tid == 0) {
     mbar_init(&sb->q_full, 1);
@@ -176,7 +186,8 @@ __global__ void __launch_bounds__(ScoreCfg<D, BN>::kThreads, 1)
     if (lane == 0) {
       tma_prefetch_desc(&tmQs);
       tma_prefetch_desc(&tmK);
-      tma_prefetch_desc(&tmV);
+      const CUtensorMap* mapV = half_p ? &tmVh : &tmV;  // 2-byte elements either way
+      tma_prefetch_desc(mapV);
       mbar_arrive_expect_tx(&sb->q_full, C::kQBytes);
       for (int zl = 0; zl < C::kGroups; ++zl) {
         const int z = z0 + zl;  // groups past the end read out-of-range tiles: zero-filled
@@ -205,7 +216,7 @@ __global__ void __launch_bounds__(ScoreCfg<D, BN>::kThreads, 1)
           const int st = vb & 1;
           mbar_arrive_expect_tx(&sb->v_full[st], C::kKVBytes);
           for (int c = 0; c < C::kChunks; ++c)
-            tma_load_3d(sV + st * C::kKVBytes + c * (BN * 128), &tmV, &sb->v_full[st], c * 64, g, vb * BN);
+            tma_load_3d(sV + st * C::kKVBytes + c * (BN * 128), mapV, &sb->v_full[st], c * 64, g, vb * BN);
           ++vb;
           progressed = true;
         }
@@ -240,12 +251,21 @@ __global__ void __launch_bounds__(ScoreCfg<D, BN>::kThreads, 1)
       tc_fence_after();
       const uint32_t tP = tmem + C::kColS + s * 128;
       const uint32_t aVs = aV + sv * C::kKVBytes;
+      if (half_p) {
 #pragma unroll
-      for (int kk = 0; kk < BN / 16; ++kk) {
-        // keys [16 kk, 16 kk + 16): P_hi words at [16 kk, +8), P_lo at [16 kk + 8, +8)
-        const uint64_t bdesc = smem_desc_sw128(aVs + kk * 2048, BN * 128, 1024);
-        mma_ts_warp(tAcc, tP + kk * 16, bdesc, C::kIdescPV, kk > 0 ? 1u : 0u);
-        mma_ts_warp(tAcc, tP + kk * 16 + 8, bdesc, C::kIdescPV, 1u);
+        for (int kk = 0; kk < BN / 16; ++kk) {
+          // keys [16 kk, 16 kk + 16): fp16 P words at [8 kk, 8 kk + 8)
+          const uint64_t bdesc = smem_desc_sw128(aVs + kk * 2048, BN * 128, 1024);
+          mma_ts_warp(tAcc, tP + kk * 8, bdesc, C::kIdescPVh, kk > 0 ? 1u : 0u);
+        }
+      } else {
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk) {
+          // keys [16 kk, 16 kk + 16): P_hi words at [16 kk, +8), P_lo at [16 kk + 8, +8)
+          const uint64_t bdesc = smem_desc_sw128(aVs + kk * 2048, BN * 128, 1024);
+          mma_ts_warp(tAcc, tP + kk * 16, bdesc, C::kIdescPV, kk > 0 ? 1u : 0u);
+          mma_ts_warp(tAcc, tP + kk * 16 + 8, bdesc, C::kIdescPV, 1u);
+        }
       }
       mma_commit_warp(&sb->v_empty[sv]);
       mma_commit_warp(&sb->acc_full);
@@ -294,8 +314,19 @@ __global__ void __launch_bounds__(ScoreCfg<D, BN>::kThreads, 1)
       if (!warp_wait(&sb->s_full[s], (b / 3) & 1, sb, p.err)) { ok = false; break; }
       tc_fence_after();
       const int lim = qpos - b * BN;
-      const float msum = (b < i_lo) ? exp_split_store<BN, false>(tS, sl2, lse2, lim)
-                                    : exp_split_store<BN, true>(tS, sl2, lse2, lim);
+      float msum;
+      if (half_p) {
+        // 2^6 p in fp16; m_b is the sum of the unscaled fp32 weights
+        uint32_t a[BN / 32][32];
+        load_row<BN>(tS, a);
+        const float m16 = lse2 - C::kHalfScaleLog2;
+        msum = ((b < i_lo) ? exp_f16_store_regs<BN, false>(tS, a, sl2, m16, lim)
+                           : exp_f16_store_regs<BN, true>(tS, a, sl2, m16, lim)) *
+               (1.0f / 64.0f);
+      } else {
+        msum = (b < i_lo) ? exp_split_store<BN, false>(tS, sl2, lse2, lim)
+                          : exp_split_store<BN, true>(tS, sl2, lse2, lim);
+      }
       // hand m_b to the norm warps (slot b % 2 is free once block b-2's norm read it)
       if (b >= 2 && !warp_wait(&sb->m_empty[sm], ((b >> 1) & 1) ^ 1, sb, p.err)) ok = false;
       sm_m[sm * 128 + r] = valid ? msum : 0.f;
@@ -308,7 +339,8 @@ __global__ void __launch_bounds__(ScoreCfg<D, BN>::kThreads, 1)
   } else {
     // ====================== pass 2: norm warps 4-7 ======================
     // The row's dense output o (pass 1) stays in registers; per block b the
-    // accumulator b % 2 holds P_b V_b, and I_b = || P_b V_b - m_b o ||.
+    // accumulator holds P_b V_b (2^6 P_b V_b with the fp16 P), and
+    // I_b = || P_b V_b - m_b o ||.
     const int r = tid - 128;                 // TMEM lane = row
     const int zl = r >> 4;
     const int j = r & 15;
@@ -340,7 +372,8 @@ __global__ void __launch_bounds__(ScoreCfg<D, BN>::kThreads, 1)
       const float mb_row = sm_m[s * 128 + r];
       warp_arrive(&sb->m_empty[s]);
       const uint32_t tAcc = tmem + lane_off + C::kColAcc;
-      const uint64_t negm2 = f2_pack(-mb_row, -mb_row);
+      const float acc_scale = half_p ? 64.0f : 1.0f;  // the accumulator holds acc_scale P_b V_b
+      const uint64_t negm2 = f2_pack(-mb_row * acc_scale, -mb_row * acc_scale);
       uint64_t acc2 = f2_pack(0.f, 0.f);
 #pragma unroll
       for (int c = 0; c < D / 16; ++c) {
@@ -360,7 +393,7 @@ __global__ void __launch_bounds__(ScoreCfg<D, BN>::kThreads, 1)
       warp_arrive(&sb->acc_empty);
       float a0, a1;
       f2_unpack(acc2, a0, a1);
-      float Ib = valid ? sqrtf(a0 + a1) : 0.f;
+      float Ib = valid ? sqrtf(a0 + a1) * (1.0f / acc_scale) : 0.f;
       float mb = valid ? mb_row : 0.f;
 #pragma unroll
       for (int off = 8; off > 0; off >>= 1) {  // max over the 16 queries of the group
@@ -385,11 +418,11 @@ __global__ void __launch_bounds__(ScoreCfg<D, BN>::kThreads, 1)
 
 template <int D, int BN>
 cudaError_t launch_pass2(const CUtensorMap& tmQs, const CUtensorMap& tmK, const CUtensorMap& tmV,
-                         const ScoreParams& p, int grid, cudaStream_t stream) {
+                         const CUtensorMap& tmVh, const ScoreParams& p, int grid, cudaStream_t stream) {
   using C = ScoreCfg<D, BN>;
   cudaError_t e = ensure_smem_limit(poem_score_pass2_kernel<D, BN>, C::kSmemBytes);
   if (e != cudaSuccess) return e;
-  poem_score_pass2_kernel<D, BN><<<grid, C::kThreads, C::kSmemBytes, stream>>>(tmQs, tmK, tmV, p);
+  poem_score_pass2_kernel<D, BN><<<grid, C::kThreads, C::kSmemBytes, stream>>>(tmQs, tmK, tmV, tmVh, p);
   return cudaGetLastError();
 }
 
@@ -404,7 +437,7 @@ cudaError_t launch_score_t(const CUtensorMap& tmQs, const CUtensorMap& tmK, cons
   if (e != cudaSuccess) return e;
   e = launch_score_pass1(D, BN, tmQs, tmK, tmV, tmVh, p, grid, stream);
   if (e != cudaSuccess) return e;
-  return launch_pass2<D, BN>(tmQs, tmK, tmV, p, grid, stream);
+  return launch_pass2<D, BN>(tmQs, tmK, tmV, tmVh, p, grid, stream);
 }
 
 }  // namespace

@@ -69,7 +69,6 @@ struct P1Cfg {
   static constexpr uint32_t kIdescQK = idesc_bf16_f32(M, BN, 0);
   static constexpr uint32_t kIdescPV = idesc_bf16_f32(M, D, 1);
   static constexpr uint32_t kIdescPVh = idesc_f16_f32(M, D, 1);  // fp16 P x fp16 V
-  static constexpr int kHalfMinTile = 32;  // smallest global tile of a CTA taking the fp16 P
 };
 
 struct P1Barriers {
@@ -86,39 +85,8 @@ struct P1Barriers {
 
 using fwd::kDrainNs;
 using fwd::wait_or_abort;
+using score::exp_f16_store_regs;
 using score::exp_split_store_regs;
-
-// The exponentials of a register-held row as one fp16 P: k-step kk (keys 16 kk ..
-// 16 kk + 15) in columns [8 kk, 8 kk + 8) of the row's S buffer.  Returns sum p.
-template <int BN, bool MASKED>
-__device__ __forceinline__ float exp_f16_store_regs(uint32_t tS, const uint32_t (&a)[BN / 32][32], float sl2,
-                                                    float m_use, int lim) {
-  const uint64_t scale2 = f2_pack(sl2, sl2);
-  const uint64_t negm2 = f2_pack(-m_use, -m_use);
-  uint64_t acc = f2_pack(0.f, 0.f);
-#pragma unroll
-  for (int c = 0; c < BN / 32; ++c) {
-    uint32_t out[16];
-#pragma unroll
-    for (int x = 0; x < 16; ++x) {
-      const int col = c * 32 + 2 * x;
-      const uint64_t xv = f2_fma(f2_pack(__uint_as_float(a[c][2 * x]), __uint_as_float(a[c][2 * x + 1])), scale2, negm2);
-      float x0, x1;
-      f2_unpack(xv, x0, x1);
-      float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
-      if (MASKED) {
-        if (col > lim) p0 = 0.f;
-        if (col + 1 > lim) p1 = 0.f;
-      }
-      acc = f2_add(acc, f2_pack(p0, p1));
-      out[x] = pack_f16x2(p0, p1);
-    }
-    tmem_st16(tS + c * 16, out);
-  }
-  float a0, a1;
-  f2_unpack(acc, a0, a1);
-  return a0 + a1;
-}
 
 // ---- V -> fp16 -----------------------------------------------------------------
 // One thread converts 8 consecutive channels of one (token, KV head) row of V into the
@@ -188,7 +156,7 @@ __global__ void __launch_bounds__(P1Cfg<D, BN>::kThreads, 1)
   const int nb = z_last / G + 1 + t0;  // key blocks 0 .. largest (global) tile of the CTA
   const int i_lo = z0 / G + t0;        // blocks < i_lo need no causal mask
   // fp16 P for this CTA (uniform): all its tiles >= 32 and V inside fp16's range
-  const bool half_p = (i_lo >= C::kHalfMinTile) && (*p.v_overflow == 0);
+  const bool half_p = (i_lo >= score::kHalfMinTile) && (*p.v_overflow == 0);
 
   if (tid == 0) {
     mbar_init(&sb->q_full, 1);

@@ -1,11 +1,18 @@
 // score_common.cuh -- device helpers shared by the two score passes (poem_score.cu,
 // poem_score_pass1.cu): the exponentials of one sampled-query row of S written back
-// as a bf16 hi/lo pair for the P V contraction, and the row maximum of S.
+// as a bf16 hi/lo pair or as one fp16 P for the P V contraction, and the row maximum
+// of S.
 #pragma once
 #include "common.cuh"
 
 namespace poem {
 namespace score {
+
+// A CTA whose smallest global query tile is at least this takes the single fp16 P
+// (with V in fp16) in both passes; earlier tiles take the bf16 hi/lo pair.  On the
+// first tiles one or a few blocks carry nearly all of a query's mass, r_b cancels
+// almost exactly against m_b o, and the fp16 rounding of P would dominate I_b.
+constexpr int kHalfMinTile = 32;
 
 // p = 2^(s * scale * log2e - m) for one row's BN scores (re-read from TMEM in 64-column
 // halves; masked columns > lim exactly 0 when MASKED), written back over S as
@@ -142,6 +149,38 @@ __device__ __forceinline__ float row_max_regs(const uint32_t (&a)[BN / 32][32], 
       m[(x >> 1) & 3] = fmax3(m[(x >> 1) & 3], v0, v1);
     }
   return fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3]));
+}
+
+// The exponentials of a register-held row as one fp16 P: k-step kk (keys 16 kk ..
+// 16 kk + 15) in columns [8 kk, 8 kk + 8) of the row's S buffer.  Returns sum p.
+template <int BN, bool MASKED>
+__device__ __forceinline__ float exp_f16_store_regs(uint32_t tS, const uint32_t (&a)[BN / 32][32], float sl2,
+                                                    float m_use, int lim) {
+  const uint64_t scale2 = f2_pack(sl2, sl2);
+  const uint64_t negm2 = f2_pack(-m_use, -m_use);
+  uint64_t acc = f2_pack(0.f, 0.f);
+#pragma unroll
+  for (int c = 0; c < BN / 32; ++c) {
+    uint32_t out[16];
+#pragma unroll
+    for (int x = 0; x < 16; ++x) {
+      const int col = c * 32 + 2 * x;
+      const uint64_t xv = f2_fma(f2_pack(__uint_as_float(a[c][2 * x]), __uint_as_float(a[c][2 * x + 1])), scale2, negm2);
+      float x0, x1;
+      f2_unpack(xv, x0, x1);
+      float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+      if (MASKED) {
+        if (col > lim) p0 = 0.f;
+        if (col + 1 > lim) p1 = 0.f;
+      }
+      acc = f2_add(acc, f2_pack(p0, p1));
+      out[x] = pack_f16x2(p0, p1);
+    }
+    tmem_st16(tS + c * 16, out);
+  }
+  float a0, a1;
+  f2_unpack(acc, a0, a1);
+  return a0 + a1;
 }
 
 }  // namespace score

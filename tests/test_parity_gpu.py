@@ -329,7 +329,7 @@ SCORE_CASES = [
     (1280, 5, 1, 128, 128, 1000000.0, 1),   # 5-way GQA: packed groups straddle tiles
     (1024, 8, 2, 128, 128, 500000.0, 2),
     (1024, 2, 1, 64, 64, 10000.0, 3),
-    # more than 32 tiles: the CTAs beyond tile 32 take pass 1's fp16 P V contraction
+    # more than 32 tiles: the CTAs beyond tile 32 take both passes' fp16 P V contraction
     (6400, 5, 1, 128, 128, 1000000.0, 4),
     (4096, 2, 1, 64, 64, 10000.0, 5),
 ]
@@ -387,8 +387,8 @@ def test_score_shift_invariance(poem):
 
 
 def test_score_values_beyond_fp16_range_take_the_bf16_contraction(poem):
-    """Pass 1 runs the P V contraction of CTAs whose tiles are all >= 32 with one fp16 P
-    on an fp16 copy of V.  A finite |v| above the fp16 maximum (65504) sets the range
+    """Both score passes run the P V contraction of CTAs whose tiles are all >= 32 with
+    one fp16 P on an fp16 copy of V.  A finite |v| above the fp16 maximum (65504) sets the range
     flag in the score workspace (byte 8) and every CTA takes the bf16 hi/lo
     contraction; both give oracle scores (64 tiles: CTAs on both sides of tile 32)."""
     x = poem_synth.heavy_block_layer(8192, 4, 1, 128, block=128, seed=21)
