@@ -30,9 +30,12 @@
 //         ahead of the softmax; the P_b V_b accumulator at [384, 384 + D), read by the
 //         norm warps while the next blocks' S are computed
 //   smem  Q tile, 3-stage K ring, 2-stage V ring (192 KB at d = 128)
-//   warps 0-3 softmax, warps 4-7 the norm of P_b V_b - m_b o with o held in
-//   registers; warp 8 issues TMA loads (K and V rings independently); warp 9 issues
-//   the MMAs, converged, from one elected lane.
+//   warps 0-3 and 8-11 softmax (two warpgroups taking alternate key blocks: with
+//   lse known the blocks are independent), warps 4-7 the norm of P_b V_b - m_b o with
+//   o held in registers; warp 12 issues TMA loads (K and V rings independently);
+//   warp 13 issues the MMAs, converged, from one elected lane; warps 14-15 idle.
+//   Registers per thread: 128 at launch; the norm warpgroup raises its budget to
+//   200 and warps 12-15 lower theirs to 56 (128 + 200 + 128 + 56 = 4 x 128).
 //   MMA order: S_0, S_1, S_2, PV_0, S_3, PV_1, ...
 //
 // Precision: on a CTA's first query tiles (below score::kHalfMinTile) P enters the
@@ -73,9 +76,12 @@ struct ScoreCfg {
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kColS = 0;     // S buffer s (0, 1, 2) at [128 s, 128 s + BN)
   static constexpr uint32_t kColAcc = 384; // P_b V_b accumulator at [384, 384 + D)
-  static constexpr int kWarpProd = 8;      // warps 0-3 softmax, 4-7 norm, 8 TMA, 9 MMA
-  static constexpr int kWarpMma = 9;
-  static constexpr int kThreads = 320;
+  static constexpr int kWarpProd = 12;     // warps 0-3, 8-11 softmax, 4-7 norm, 12 TMA, 13 MMA
+  static constexpr int kWarpMma = 13;
+  static constexpr int kThreads = 512;
+  static constexpr uint32_t kRegNorm = 200;  // per-thread registers after the reallocation
+  static constexpr uint32_t kRegProd = 56;
+  static_assert(128 + kRegNorm + 128 + kRegProd == 4 * 128, "register budget of the launch");
   static constexpr uint32_t kIdescQK = idesc_bf16_f32(M, BN, 0);
   static constexpr uint32_t kIdescPV = idesc_bf16_f32(M, D, 1);
   static constexpr uint32_t kIdescPVh = idesc_f16_f32(M, D, 1);  // fp16 P x fp16 V
@@ -122,9 +128,8 @@ __device__ __forceinline__ void score_cta_coords(int cta, int ctas_per_g, int& g
   z0 = c * 8;
 }
 
-using score::exp_f16_store_regs;
+using score::exp_f16_store;
 using score::exp_split_store;
-using score::load_row;
 
 template <int D, int BN>
 __global__ void __launch_bounds__(ScoreCfg<D, BN>::kThreads, 1)
@@ -181,120 +186,125 @@ __global__ void __launch_bounds__(ScoreCfg<D, BN>::kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = sb->tmem_base;
 
-  if (warp == C::kWarpProd) {
-    // ============================ TMA producer ============================
-    if (lane == 0) {
-      tma_prefetch_desc(&tmQs);
-      tma_prefetch_desc(&tmK);
-      const CUtensorMap* mapV = half_p ? &tmVh : &tmV;  // 2-byte elements either way
-      tma_prefetch_desc(mapV);
-      mbar_arrive_expect_tx(&sb->q_full, C::kQBytes);
-      for (int zl = 0; zl < C::kGroups; ++zl) {
-        const int z = z0 + zl;  // groups past the end read out-of-range tiles: zero-filled
-        const int i = z / G;
-        const int hq = g * G + (z - i * G);
-        for (int c = 0; c < C::kChunks; ++c)
-          tma_load_4d(sQ + c * (C::M * 128) + zl * (C::kRowsPerGroup * 128), &tmQs, &sb->q_full, c * 64, hq, 0,
-                      i);
-      }
-      // K and V rings advance independently: K_b is loaded once S_{b-3} has released
-      // its stage, V_b once P V_{b-2} has.
-      int kb = 0, vb = 0;
-      uint64_t t_last = globaltimer_ns();
-      while ((kb < nb || vb < nb) && !sb->abort_flag) {
-        bool progressed = false;
-        // a fresh stage passes the parity-1 test at once; later, completion #(b/stages - 1)
-        if (kb < nb && mbar_try_wait(&sb->k_empty[kb % 3], ((kb / 3) & 1) ^ 1)) {
-          const int st = kb % 3;
-          mbar_arrive_expect_tx(&sb->k_full[st], C::kKVBytes);
+  if (warp >= C::kWarpProd) {
+    // warps 12-15 (one warpgroup): lower the register budget, one instruction for all four
+    warpgroup_reg_dec<C::kRegProd>();
+    if (warp == C::kWarpProd) {
+      // ============================ TMA producer ============================
+      if (lane == 0) {
+        tma_prefetch_desc(&tmQs);
+        tma_prefetch_desc(&tmK);
+        const CUtensorMap* mapV = half_p ? &tmVh : &tmV;  // 2-byte elements either way
+        tma_prefetch_desc(mapV);
+        mbar_arrive_expect_tx(&sb->q_full, C::kQBytes);
+        for (int zl = 0; zl < C::kGroups; ++zl) {
+          const int z = z0 + zl;  // groups past the end read out-of-range tiles: zero-filled
+          const int i = z / G;
+          const int hq = g * G + (z - i * G);
           for (int c = 0; c < C::kChunks; ++c)
-            tma_load_3d(sK + st * C::kKVBytes + c * (BN * 128), &tmK, &sb->k_full[st], c * 64, g, kb * BN);
-          ++kb;
-          progressed = true;
+            tma_load_4d(sQ + c * (C::M * 128) + zl * (C::kRowsPerGroup * 128), &tmQs, &sb->q_full, c * 64, hq, 0,
+                        i);
         }
-        if (vb < kb && mbar_try_wait(&sb->v_empty[vb & 1], ((vb >> 1) & 1) ^ 1)) {
-          const int st = vb & 1;
-          mbar_arrive_expect_tx(&sb->v_full[st], C::kKVBytes);
-          for (int c = 0; c < C::kChunks; ++c)
-            tma_load_3d(sV + st * C::kKVBytes + c * (BN * 128), mapV, &sb->v_full[st], c * 64, g, vb * BN);
-          ++vb;
-          progressed = true;
+        // K and V rings advance independently: K_b is loaded once S_{b-3} has released
+        // its stage, V_b once P V_{b-2} has.
+        int kb = 0, vb = 0;
+        uint64_t t_last = globaltimer_ns();
+        while ((kb < nb || vb < nb) && !sb->abort_flag) {
+          bool progressed = false;
+          // a fresh stage passes the parity-1 test at once; later, completion #(b/stages - 1)
+          if (kb < nb && mbar_try_wait(&sb->k_empty[kb % 3], ((kb / 3) & 1) ^ 1)) {
+            const int st = kb % 3;
+            mbar_arrive_expect_tx(&sb->k_full[st], C::kKVBytes);
+            for (int c = 0; c < C::kChunks; ++c)
+              tma_load_3d(sK + st * C::kKVBytes + c * (BN * 128), &tmK, &sb->k_full[st], c * 64, g, kb * BN);
+            ++kb;
+            progressed = true;
+          }
+          if (vb < kb && mbar_try_wait(&sb->v_empty[vb & 1], ((vb >> 1) & 1) ^ 1)) {
+            const int st = vb & 1;
+            mbar_arrive_expect_tx(&sb->v_full[st], C::kKVBytes);
+            for (int c = 0; c < C::kChunks; ++c)
+              tma_load_3d(sV + st * C::kKVBytes + c * (BN * 128), mapV, &sb->v_full[st], c * 64, g, vb * BN);
+            ++vb;
+            progressed = true;
+          }
+          if (progressed) {
+            t_last = globaltimer_ns();
+          } else if (globaltimer_ns() - t_last > p.err.timeout_ns) {
+            sb->abort_flag = 1;
+            raise_err(p.err, kErrTimeout);
+            break;
+          }
         }
-        if (progressed) {
-          t_last = globaltimer_ns();
-        } else if (globaltimer_ns() - t_last > p.err.timeout_ns) {
-          sb->abort_flag = 1;
-          raise_err(p.err, kErrTimeout);
-          break;
-        }
+        // Drain: the last load issued into each stage must have landed.
+        mbar_wait(&sb->q_full, 0, kDrainNs);
+        for (int x = max(0, kb - 3); x < kb; ++x) mbar_wait(&sb->k_full[x % 3], (x / 3) & 1, kDrainNs);
+        for (int x = max(0, vb - 2); x < vb; ++x) mbar_wait(&sb->v_full[x & 1], (x >> 1) & 1, kDrainNs);
       }
-      // Drain: the last load issued into each stage must have landed.
-      mbar_wait(&sb->q_full, 0, kDrainNs);
-      for (int x = max(0, kb - 3); x < kb; ++x) mbar_wait(&sb->k_full[x % 3], (x / 3) & 1, kDrainNs);
-      for (int x = max(0, vb - 2); x < vb; ++x) mbar_wait(&sb->v_full[x & 1], (x >> 1) & 1, kDrainNs);
-    }
-  } else if (warp == C::kWarpMma) {
-    // ============================ MMA issuer ============================
-    // The whole warp runs this loop converged (waits and operands are warp-uniform);
-    // one elected lane issues each MMA and commit.
-    // Order S_0, S_1, S_2, PV_0, S_3, PV_1, ...: S_b lands in S buffer b % 3 (free once
-    // P V_{b-3}, issued just before, has read it), P_b V_b in the accumulator, started
-    // fresh once the norm warps have read P V_{b-1}.
-    const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV);
-    const uint32_t tAcc = tmem + C::kColAcc;
-    bool ok = warp_wait(&sb->q_full, 0, sb, p.err);
-    auto issue_pv = [&](int j) -> bool {
-      const int s = j % 3, sv = j & 1;
-      if (!warp_wait(&sb->p_full[s], (j / 3) & 1, sb, p.err)) return false;
-      if (!warp_wait(&sb->v_full[sv], (j >> 1) & 1, sb, p.err)) return false;
-      if (j >= 1 && !warp_wait(&sb->acc_empty, (j - 1) & 1, sb, p.err)) return false;
-      tc_fence_after();
-      const uint32_t tP = tmem + C::kColS + s * 128;
-      const uint32_t aVs = aV + sv * C::kKVBytes;
-      if (half_p) {
-#pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk) {
-          // keys [16 kk, 16 kk + 16): fp16 P words at [8 kk, 8 kk + 8)
-          const uint64_t bdesc = smem_desc_sw128(aVs + kk * 2048, BN * 128, 1024);
-          mma_ts_warp(tAcc, tP + kk * 8, bdesc, C::kIdescPVh, kk > 0 ? 1u : 0u);
+    } else if (warp == C::kWarpMma) {
+      // ============================ MMA issuer ============================
+      // The whole warp runs this loop converged (waits and operands are warp-uniform);
+      // one elected lane issues each MMA and commit.
+      // Order S_0, S_1, S_2, PV_0, S_3, PV_1, ...: S_b lands in S buffer b % 3 (free once
+      // P V_{b-3}, issued just before, has read it), P_b V_b in the accumulator, started
+      // fresh once the norm warps have read P V_{b-1}.
+      const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV);
+      const uint32_t tAcc = tmem + C::kColAcc;
+      bool ok = warp_wait(&sb->q_full, 0, sb, p.err);
+      auto issue_pv = [&](int j) -> bool {
+        const int s = j % 3, sv = j & 1;
+        if (!warp_wait(&sb->p_full[s], (j / 3) & 1, sb, p.err)) return false;
+        if (!warp_wait(&sb->v_full[sv], (j >> 1) & 1, sb, p.err)) return false;
+        if (j >= 1 && !warp_wait(&sb->acc_empty, (j - 1) & 1, sb, p.err)) return false;
+        tc_fence_after();
+        const uint32_t tP = tmem + C::kColS + s * 128;
+        const uint32_t aVs = aV + sv * C::kKVBytes;
+        if (half_p) {
+  #pragma unroll
+          for (int kk = 0; kk < BN / 16; ++kk) {
+            // keys [16 kk, 16 kk + 16): fp16 P words at [8 kk, 8 kk + 8)
+            const uint64_t bdesc = smem_desc_sw128(aVs + kk * 2048, BN * 128, 1024);
+            mma_ts_warp(tAcc, tP + kk * 8, bdesc, C::kIdescPVh, kk > 0 ? 1u : 0u);
+          }
+        } else {
+  #pragma unroll
+          for (int kk = 0; kk < BN / 16; ++kk) {
+            // keys [16 kk, 16 kk + 16): P_hi words at [16 kk, +8), P_lo at [16 kk + 8, +8)
+            const uint64_t bdesc = smem_desc_sw128(aVs + kk * 2048, BN * 128, 1024);
+            mma_ts_warp(tAcc, tP + kk * 16, bdesc, C::kIdescPV, kk > 0 ? 1u : 0u);
+            mma_ts_warp(tAcc, tP + kk * 16 + 8, bdesc, C::kIdescPV, 1u);
+          }
         }
-      } else {
-#pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk) {
-          // keys [16 kk, 16 kk + 16): P_hi words at [16 kk, +8), P_lo at [16 kk + 8, +8)
-          const uint64_t bdesc = smem_desc_sw128(aVs + kk * 2048, BN * 128, 1024);
-          mma_ts_warp(tAcc, tP + kk * 16, bdesc, C::kIdescPV, kk > 0 ? 1u : 0u);
-          mma_ts_warp(tAcc, tP + kk * 16 + 8, bdesc, C::kIdescPV, 1u);
+        mma_commit_warp(&sb->v_empty[sv]);
+        mma_commit_warp(&sb->acc_full);
+        return true;
+      };
+      for (int b = 0; b < nb && ok; ++b) {
+        if (b >= 3 && !issue_pv(b - 3)) { ok = false; break; }
+        const int s = b % 3;
+        if (!warp_wait(&sb->k_full[s], (b / 3) & 1, sb, p.err)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t tS = tmem + C::kColS + s * 128;
+        const uint32_t aKs = aK + s * C::kKVBytes;
+  #pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t koff = (kk & 3) * 32;
+          const uint64_t adesc = smem_desc_sw128(aQ + (kk >> 2) * (C::M * 128) + koff, 16, 1024);
+          const uint64_t bdesc = smem_desc_sw128(aKs + (kk >> 2) * (BN * 128) + koff, 16, 1024);
+          mma_ss_warp(tS, adesc, bdesc, C::kIdescQK, kk > 0 ? 1u : 0u);
         }
+        mma_commit_warp(&sb->s_full[s]);
+        mma_commit_warp(&sb->k_empty[s]);
       }
-      mma_commit_warp(&sb->v_empty[sv]);
-      mma_commit_warp(&sb->acc_full);
-      return true;
-    };
-    for (int b = 0; b < nb && ok; ++b) {
-      if (b >= 3 && !issue_pv(b - 3)) { ok = false; break; }
-      const int s = b % 3;
-      if (!warp_wait(&sb->k_full[s], (b / 3) & 1, sb, p.err)) { ok = false; break; }
-      tc_fence_after();
-      const uint32_t tS = tmem + C::kColS + s * 128;
-      const uint32_t aKs = aK + s * C::kKVBytes;
-#pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        const uint32_t koff = (kk & 3) * 32;
-        const uint64_t adesc = smem_desc_sw128(aQ + (kk >> 2) * (C::M * 128) + koff, 16, 1024);
-        const uint64_t bdesc = smem_desc_sw128(aKs + (kk >> 2) * (BN * 128) + koff, 16, 1024);
-        mma_ss_warp(tS, adesc, bdesc, C::kIdescQK, kk > 0 ? 1u : 0u);
-      }
-      mma_commit_warp(&sb->s_full[s]);
-      mma_commit_warp(&sb->k_empty[s]);
-    }
-    for (int j = max(0, nb - 3); j < nb && ok; ++j)
-      if (!issue_pv(j)) ok = false;
-    mma_commit_warp(&sb->drain);
-    mbar_wait(&sb->drain, 0, kDrainNs);
-  } else if (warp < 4) {
-    // ====================== pass 2: softmax warps 0-3 ======================
-    const int r = tid;
+      for (int j = max(0, nb - 3); j < nb && ok; ++j)
+        if (!issue_pv(j)) ok = false;
+      mma_commit_warp(&sb->drain);
+      mbar_wait(&sb->drain, 0, kDrainNs);
+    }  // warps 14-15 idle
+  } else if (warp < 4 || warp >= 8) {
+    // ================= pass 2: softmax warps 0-3 (even blocks), 8-11 (odd) =================
+    const int wg = warp >> 3;
+    const int r = tid & 127;
     const int zl = r >> 4;
     const int j = r & 15;
     const int z = z0 + zl;
@@ -303,12 +313,14 @@ __global__ void __launch_bounds__(ScoreCfg<D, BN>::kThreads, 1)
     const int hq = g * G + (valid ? z - i * G : 0);
     const int qpos = valid ? (i + t0) * BN + j * p.sample_stride : -1;
     const int64_t srow = ((int64_t)hq * p.n_tiles + i) * p.n_sample + j;
-    const uint32_t lane_off = ((uint32_t)(warp * 32) << 16);
+    const uint32_t lane_off = ((uint32_t)((warp & 3) * 32) << 16);
     const float sl2 = p.scale_log2;
     const bool in_ws = POEM_IN_BOUNDS(p.err, srow, (int64_t)p.n_q_heads * p.n_tiles * p.n_sample);
     const float lse2 = (valid && in_ws) ? p.ws_lse[srow] : 0.f;
     bool ok = true;
-    for (int b = 0; b < nb; ++b) {
+    // Block b's wait on s_full[b % 3] is at most one phase behind: S_{b+3} needs
+    // P V_b, which needs this warpgroup's P_b.  m_b goes to slot b & 1 = wg.
+    for (int b = wg; b < nb; b += 2) {
       const int s = b % 3, sm = b & 1;
       const uint32_t tS = tmem + lane_off + C::kColS + s * 128;
       if (!warp_wait(&sb->s_full[s], (b / 3) & 1, sb, p.err)) { ok = false; break; }
@@ -317,11 +329,9 @@ __global__ void __launch_bounds__(ScoreCfg<D, BN>::kThreads, 1)
       float msum;
       if (half_p) {
         // 2^6 p in fp16; m_b is the sum of the unscaled fp32 weights
-        uint32_t a[BN / 32][32];
-        load_row<BN>(tS, a);
         const float m16 = lse2 - C::kHalfScaleLog2;
-        msum = ((b < i_lo) ? exp_f16_store_regs<BN, false>(tS, a, sl2, m16, lim)
-                           : exp_f16_store_regs<BN, true>(tS, a, sl2, m16, lim)) *
+        msum = ((b < i_lo) ? exp_f16_store<BN, false>(tS, sl2, m16, lim)
+                           : exp_f16_store<BN, true>(tS, sl2, m16, lim)) *
                (1.0f / 64.0f);
       } else {
         msum = (b < i_lo) ? exp_split_store<BN, false>(tS, sl2, lse2, lim)
@@ -341,6 +351,7 @@ __global__ void __launch_bounds__(ScoreCfg<D, BN>::kThreads, 1)
     // The row's dense output o (pass 1) stays in registers; per block b the
     // accumulator holds P_b V_b (2^6 P_b V_b with the fp16 P), and
     // I_b = || P_b V_b - m_b o ||.
+    warpgroup_reg_inc<C::kRegNorm>();
     const int r = tid - 128;                 // TMEM lane = row
     const int zl = r >> 4;
     const int j = r & 15;

@@ -60,6 +60,48 @@ __device__ __forceinline__ float exp_split_store(uint32_t tS, float sl2, float m
   return a0 + a1;
 }
 
+// p = 2^(s * scale * log2e - m) for one row's BN scores as one fp16 P (re-read from
+// TMEM in 64-column halves; masked columns > lim exactly 0 when MASKED): k-step kk
+// (keys 16 kk .. 16 kk + 15) goes to columns [8 kk, 8 kk + 8) of the row's S buffer,
+// which hold scores already read.  Returns sum p.
+template <int BN, bool MASKED>
+__device__ __forceinline__ float exp_f16_store(uint32_t tS, float sl2, float m_use, int lim) {
+  const uint64_t scale2 = f2_pack(sl2, sl2);
+  const uint64_t negm2 = f2_pack(-m_use, -m_use);
+  uint64_t acc = f2_pack(0.f, 0.f);
+#pragma unroll
+  for (int cp = 0; cp < BN / 64; ++cp) {
+    uint32_t a[2][32];
+    tmem_ld32(tS + cp * 64, a[0]);
+    tmem_ld32(tS + cp * 64 + 32, a[1]);
+    tmem_ld_wait();
+    tmem_reg_fence(a[0]);
+    tmem_reg_fence(a[1]);
+#pragma unroll
+    for (int hf = 0; hf < 2; ++hf) {
+      uint32_t out[16];
+#pragma unroll
+      for (int x = 0; x < 16; ++x) {
+        const int col = cp * 64 + hf * 32 + 2 * x;
+        const uint64_t xv = f2_fma(f2_pack(__uint_as_float(a[hf][2 * x]), __uint_as_float(a[hf][2 * x + 1])), scale2, negm2);
+        float x0, x1;
+        f2_unpack(xv, x0, x1);
+        float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+        if (MASKED) {
+          if (col > lim) p0 = 0.f;
+          if (col + 1 > lim) p1 = 0.f;
+        }
+        acc = f2_add(acc, f2_pack(p0, p1));
+        out[x] = pack_f16x2(p0, p1);
+      }
+      tmem_st16(tS + cp * 32 + hf * 16, out);
+    }
+  }
+  float a0, a1;
+  f2_unpack(acc, a0, a1);
+  return a0 + a1;
+}
+
 // Maximum of one row's visible scores (columns <= lim when MASKED), read in 64-column halves.
 template <int BN, bool MASKED>
 __device__ __forceinline__ float row_max(uint32_t tS, int lim) {

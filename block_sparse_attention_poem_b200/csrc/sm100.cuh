@@ -321,6 +321,20 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
 
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
+// ---- per-warpgroup register budget -----------------------------------------------------
+// Executed by all four warps of a warpgroup.  The increases a kernel makes must be
+// covered by its decreases: the pool is the launch's threads x registers per thread.
+template <uint32_t N>
+__device__ __forceinline__ void warpgroup_reg_inc() {
+  static_assert(N % 8 == 0 && N >= 24 && N <= 256, "setmaxnreg operand");
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void warpgroup_reg_dec() {
+  static_assert(N % 8 == 0 && N >= 24 && N <= 256, "setmaxnreg operand");
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // ---- math helpers ----------------------------------------------------------------------
 __device__ __forceinline__ float ex2_approx(float x) {  // hardware 2^x (MUFU)
   float y;
