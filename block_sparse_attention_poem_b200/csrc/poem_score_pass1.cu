@@ -23,20 +23,26 @@
 //
 // Pipeline:
 //   TMEM  S buffers s = 0, 1, 2 at [128 s, 128 s + BN); O at [384, 384 + D).  With
-//         three S buffers the MMAs run up to two blocks ahead of the softmax, so the
-//         softmax warps process blocks back to back.
+//         three S buffers the MMAs run up to two blocks ahead of the softmax.
 //   smem  Q tile, 3-stage K ring, 2-stage V ring (192 KB at d = 128).
-//   warps 0-3: online softmax, one sampled query per thread (running max with a lazy
-//         rescale of O when the max grows by more than 2^8); warp 4: TMA, K and V
-//         rings advancing independently; warp 5: MMAs, converged, issued by one
-//         elected lane.
+//   warps 0-3 / 4-7: online softmax of the even / odd key blocks, one sampled query
+//         per thread.  The running state passes between the two warpgroups through
+//         shared memory: block b's reference max (published right after its row max)
+//         and the row sum through b (published after its exponentials).  The
+//         reference moves only when the max grows by more than 2^8, and O is then
+//         rescaled once P V_{b-1} has completed.  The warpgroup of the last block
+//         writes o and lse.  Warp 8: TMA, K and V rings advancing independently;
+//         warp 9: MMAs, converged, issued by one elected lane; warps 10-11 idle.
+//   Registers per thread: 168 at launch; warps 8-11 lower theirs to 56 and the two
+//   softmax warpgroups raise theirs to 224 (224 + 224 + 56 = 3 x 168).
 //   MMA order: S_0, S_1, S_2, PV_0, S_3, PV_1, ...  (S_b follows P V_{b-3}, which
 //   freed its S buffer).
 //
 // Every mbarrier wait is made at most one phase behind its barrier.  A rescale of O at
-// block b waits for P V_{b-1} on accumulator barrier (b - 1) % 2: S_b complete implies
-// P V_{b-3} complete, and P V_{b+1} cannot start before this block's P, so that
-// barrier is within one phase of the wait.  The end of the sweep waits on its own
+// block b waits for P V_{b-1} on accumulator barrier (b - 1) % 2: P V_{b+1} cannot
+// start before this block's P, so that barrier is within one phase of the wait; the
+// hand-off barriers of block b - 1 likewise cannot move on before block b has
+// published its own state.  The end of the sweep waits on its own
 // barrier (o_full), committed once after the last P V.
 #include "common.cuh"
 #include "fwd_common.cuh"
@@ -59,13 +65,18 @@ struct P1Cfg {
   static constexpr int kOffK = kOffQ + kQBytes;
   static constexpr int kOffV = kOffK + kStagesK * kKVBytes;
   static constexpr int kOffBar = kOffV + kStagesV * kKVBytes;
+  static constexpr int kOffX = kOffBar + 256;  // [2][128] reference maxima, [2][128] row sums
   // at least 120 KB so that one CTA (holding all 512 TMEM columns) occupies an SM
-  static constexpr int kSmemBytes = (kOffBar + 256 + 1024) > 122880 ? (kOffBar + 256 + 1024) : 122880;
+  static constexpr int kSmemBytes =
+      (kOffX + 4 * 128 * 4 + 1024) > 122880 ? (kOffX + 4 * 128 * 4 + 1024) : 122880;
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kColO = 384;
-  static constexpr int kWarpProd = 4;
-  static constexpr int kWarpMma = 5;
-  static constexpr int kThreads = 192;
+  static constexpr int kWarpProd = 8;
+  static constexpr int kWarpMma = 9;
+  static constexpr int kThreads = 384;
+  static constexpr uint32_t kRegSoftmax = 224;  // per-thread registers after the reallocation
+  static constexpr uint32_t kRegProd = 56;
+  static_assert(2 * kRegSoftmax + kRegProd == 3 * 168, "register budget of the launch");
   static constexpr uint32_t kIdescQK = idesc_bf16_f32(M, BN, 0);
   static constexpr uint32_t kIdescPV = idesc_bf16_f32(M, D, 1);
   static constexpr uint32_t kIdescPVh = idesc_f16_f32(M, D, 1);  // fp16 P x fp16 V
@@ -78,6 +89,7 @@ struct P1Barriers {
   uint64_t s_full[3], p_full[3];
   uint64_t acc_full[2];  // P V_j complete, on barrier j % 2
   uint64_t o_full;       // the last P V complete
+  uint64_t ref_ready[2], l_ready[2];  // block b's reference max / row sum, slot b % 2
   uint64_t drain;
   uint32_t tmem_base;
   volatile int abort_flag;
@@ -142,6 +154,8 @@ __global__ void __launch_bounds__(P1Cfg<D, BN>::kThreads, 1)
   uint8_t* sK = smem + C::kOffK;
   uint8_t* sV = smem + C::kOffV;
   P1Barriers* sb = reinterpret_cast<P1Barriers*>(smem + C::kOffBar);
+  float* x_ref = reinterpret_cast<float*>(smem + C::kOffX);  // [2][128]
+  float* x_l = x_ref + 2 * 128;                               // [2][128]
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
@@ -170,6 +184,8 @@ __global__ void __launch_bounds__(P1Cfg<D, BN>::kThreads, 1)
       mbar_init(&sb->v_full[s], 1);
       mbar_init(&sb->v_empty[s], 1);
       mbar_init(&sb->acc_full[s], 1);
+      mbar_init(&sb->ref_ready[s], 4);  // one arrival per softmax warp
+      mbar_init(&sb->l_ready[s], 4);
     }
     mbar_init(&sb->o_full, 1);
     mbar_init(&sb->drain, 1);
@@ -182,115 +198,121 @@ __global__ void __launch_bounds__(P1Cfg<D, BN>::kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = sb->tmem_base;
 
-  if (warp == C::kWarpProd) {
-    // ============================ TMA producer ============================
-    // K and V rings advance independently: K_b is loaded once S_{b-3} has released its
-    // stage, V_b once P V_{b-2} has.
-    if (lane == 0) {
-      tma_prefetch_desc(&tmQs);
-      tma_prefetch_desc(&tmK);
-      const CUtensorMap* mapV = half_p ? &tmVh : &tmV;  // 2-byte elements either way
-      tma_prefetch_desc(mapV);
-      mbar_arrive_expect_tx(&sb->q_full, C::kQBytes);
-      for (int zl = 0; zl < C::kGroups; ++zl) {
-        const int z = z0 + zl;  // groups past the end read out-of-range tiles: zero-filled
-        const int i = z / G;
-        const int hq = g * G + (z - i * G);
-        for (int c = 0; c < C::kChunks; ++c)
-          tma_load_4d(sQ + c * (C::M * 128) + zl * (C::kRowsPerGroup * 128), &tmQs, &sb->q_full, c * 64, hq, 0,
-                      i);
-      }
-      int kb = 0, vb = 0;
-      uint64_t t_last = globaltimer_ns();
-      while ((kb < nb || vb < nb) && !sb->abort_flag) {
-        bool progressed = false;
-        // a fresh stage passes the parity-1 test at once; later, completion #(b/stages - 1)
-        if (kb < nb && mbar_try_wait(&sb->k_empty[kb % 3], ((kb / 3) & 1) ^ 1)) {
-          const int s = kb % 3;
-          mbar_arrive_expect_tx(&sb->k_full[s], C::kKVBytes);
+  if (warp >= C::kWarpProd) {
+    // warps 8-11 (one warpgroup): lower the register budget, one instruction for all four
+    warpgroup_reg_dec<C::kRegProd>();
+    if (warp == C::kWarpProd) {
+      // ============================ TMA producer ============================
+      // K and V rings advance independently: K_b is loaded once S_{b-3} has released its
+      // stage, V_b once P V_{b-2} has.
+      if (lane == 0) {
+        tma_prefetch_desc(&tmQs);
+        tma_prefetch_desc(&tmK);
+        const CUtensorMap* mapV = half_p ? &tmVh : &tmV;  // 2-byte elements either way
+        tma_prefetch_desc(mapV);
+        mbar_arrive_expect_tx(&sb->q_full, C::kQBytes);
+        for (int zl = 0; zl < C::kGroups; ++zl) {
+          const int z = z0 + zl;  // groups past the end read out-of-range tiles: zero-filled
+          const int i = z / G;
+          const int hq = g * G + (z - i * G);
           for (int c = 0; c < C::kChunks; ++c)
-            tma_load_3d(sK + s * C::kKVBytes + c * (BN * 128), &tmK, &sb->k_full[s], c * 64, g, kb * BN);
-          ++kb;
-          progressed = true;
+            tma_load_4d(sQ + c * (C::M * 128) + zl * (C::kRowsPerGroup * 128), &tmQs, &sb->q_full, c * 64, hq, 0,
+                        i);
         }
-        if (vb < kb && mbar_try_wait(&sb->v_empty[vb & 1], ((vb >> 1) & 1) ^ 1)) {
-          const int s = vb & 1;
-          mbar_arrive_expect_tx(&sb->v_full[s], C::kKVBytes);
-          for (int c = 0; c < C::kChunks; ++c)
-            tma_load_3d(sV + s * C::kKVBytes + c * (BN * 128), mapV, &sb->v_full[s], c * 64, g, vb * BN);
-          ++vb;
-          progressed = true;
+        int kb = 0, vb = 0;
+        uint64_t t_last = globaltimer_ns();
+        while ((kb < nb || vb < nb) && !sb->abort_flag) {
+          bool progressed = false;
+          // a fresh stage passes the parity-1 test at once; later, completion #(b/stages - 1)
+          if (kb < nb && mbar_try_wait(&sb->k_empty[kb % 3], ((kb / 3) & 1) ^ 1)) {
+            const int s = kb % 3;
+            mbar_arrive_expect_tx(&sb->k_full[s], C::kKVBytes);
+            for (int c = 0; c < C::kChunks; ++c)
+              tma_load_3d(sK + s * C::kKVBytes + c * (BN * 128), &tmK, &sb->k_full[s], c * 64, g, kb * BN);
+            ++kb;
+            progressed = true;
+          }
+          if (vb < kb && mbar_try_wait(&sb->v_empty[vb & 1], ((vb >> 1) & 1) ^ 1)) {
+            const int s = vb & 1;
+            mbar_arrive_expect_tx(&sb->v_full[s], C::kKVBytes);
+            for (int c = 0; c < C::kChunks; ++c)
+              tma_load_3d(sV + s * C::kKVBytes + c * (BN * 128), mapV, &sb->v_full[s], c * 64, g, vb * BN);
+            ++vb;
+            progressed = true;
+          }
+          if (progressed) {
+            t_last = globaltimer_ns();
+          } else if (globaltimer_ns() - t_last > p.err.timeout_ns) {
+            sb->abort_flag = 1;
+            raise_err(p.err, kErrTimeout);
+            break;
+          }
         }
-        if (progressed) {
-          t_last = globaltimer_ns();
-        } else if (globaltimer_ns() - t_last > p.err.timeout_ns) {
-          sb->abort_flag = 1;
-          raise_err(p.err, kErrTimeout);
-          break;
-        }
+        // Drain: the last load issued into each stage must have landed.
+        mbar_wait(&sb->q_full, 0, kDrainNs);
+        for (int b = max(0, kb - 3); b < kb; ++b) mbar_wait(&sb->k_full[b % 3], (b / 3) & 1, kDrainNs);
+        for (int b = max(0, vb - 2); b < vb; ++b) mbar_wait(&sb->v_full[b & 1], (b >> 1) & 1, kDrainNs);
       }
-      // Drain: the last load issued into each stage must have landed.
-      mbar_wait(&sb->q_full, 0, kDrainNs);
-      for (int b = max(0, kb - 3); b < kb; ++b) mbar_wait(&sb->k_full[b % 3], (b / 3) & 1, kDrainNs);
-      for (int b = max(0, vb - 2); b < vb; ++b) mbar_wait(&sb->v_full[b & 1], (b >> 1) & 1, kDrainNs);
-    }
-  } else if (warp == C::kWarpMma) {
-    // ============================ MMA issuer ============================
-    const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV);
-    const uint32_t tO = tmem + C::kColO;
-    bool ok = warp_wait(&sb->q_full, 0, sb, p.err);
-    auto issue_pv = [&](int j) -> bool {
-      const int s = j % 3, sv = j & 1;
-      if (!warp_wait(&sb->p_full[s], (j / 3) & 1, sb, p.err)) return false;
-      if (!warp_wait(&sb->v_full[sv], (j >> 1) & 1, sb, p.err)) return false;
-      tc_fence_after();
-      const uint32_t tP = tmem + s * 128;
-      const uint32_t aVs = aV + sv * C::kKVBytes;
-      if (half_p) {
-#pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk) {
-          // keys [16 kk, 16 kk + 16): fp16 P words at [8 kk, +8)
-          const uint64_t bdesc = smem_desc_sw128(aVs + kk * 2048, BN * 128, 1024);
-          mma_ts_warp(tO, tP + kk * 8, bdesc, C::kIdescPVh, (j > 0 || kk > 0) ? 1u : 0u);
+    } else if (warp == C::kWarpMma) {
+      // ============================ MMA issuer ============================
+      const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV);
+      const uint32_t tO = tmem + C::kColO;
+      bool ok = warp_wait(&sb->q_full, 0, sb, p.err);
+      auto issue_pv = [&](int j) -> bool {
+        const int s = j % 3, sv = j & 1;
+        if (!warp_wait(&sb->p_full[s], (j / 3) & 1, sb, p.err)) return false;
+        if (!warp_wait(&sb->v_full[sv], (j >> 1) & 1, sb, p.err)) return false;
+        tc_fence_after();
+        const uint32_t tP = tmem + s * 128;
+        const uint32_t aVs = aV + sv * C::kKVBytes;
+        if (half_p) {
+  #pragma unroll
+          for (int kk = 0; kk < BN / 16; ++kk) {
+            // keys [16 kk, 16 kk + 16): fp16 P words at [8 kk, +8)
+            const uint64_t bdesc = smem_desc_sw128(aVs + kk * 2048, BN * 128, 1024);
+            mma_ts_warp(tO, tP + kk * 8, bdesc, C::kIdescPVh, (j > 0 || kk > 0) ? 1u : 0u);
+          }
+        } else {
+  #pragma unroll
+          for (int kk = 0; kk < BN / 16; ++kk) {
+            // keys [16 kk, 16 kk + 16): P_hi words at [16 kk, +8), P_lo at [16 kk + 8, +8)
+            const uint64_t bdesc = smem_desc_sw128(aVs + kk * 2048, BN * 128, 1024);
+            mma_ts_warp(tO, tP + kk * 16, bdesc, C::kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
+            mma_ts_warp(tO, tP + kk * 16 + 8, bdesc, C::kIdescPV, 1u);
+          }
         }
-      } else {
-#pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk) {
-          // keys [16 kk, 16 kk + 16): P_hi words at [16 kk, +8), P_lo at [16 kk + 8, +8)
-          const uint64_t bdesc = smem_desc_sw128(aVs + kk * 2048, BN * 128, 1024);
-          mma_ts_warp(tO, tP + kk * 16, bdesc, C::kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
-          mma_ts_warp(tO, tP + kk * 16 + 8, bdesc, C::kIdescPV, 1u);
+        mma_commit_warp(&sb->v_empty[sv]);
+        mma_commit_warp(&sb->acc_full[j & 1]);
+        if (j == nb - 1) mma_commit_warp(&sb->o_full);
+        return true;
+      };
+      for (int b = 0; b < nb && ok; ++b) {
+        if (b >= 3 && !issue_pv(b - 3)) { ok = false; break; }
+        const int s = b % 3;
+        if (!warp_wait(&sb->k_full[s], (b / 3) & 1, sb, p.err)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t tS = tmem + s * 128;
+        const uint32_t aKs = aK + s * C::kKVBytes;
+  #pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t koff = (kk & 3) * 32;
+          const uint64_t adesc = smem_desc_sw128(aQ + (kk >> 2) * (C::M * 128) + koff, 16, 1024);
+          const uint64_t bdesc = smem_desc_sw128(aKs + (kk >> 2) * (BN * 128) + koff, 16, 1024);
+          mma_ss_warp(tS, adesc, bdesc, C::kIdescQK, kk > 0 ? 1u : 0u);
         }
+        mma_commit_warp(&sb->s_full[s]);
+        mma_commit_warp(&sb->k_empty[s]);
       }
-      mma_commit_warp(&sb->v_empty[sv]);
-      mma_commit_warp(&sb->acc_full[j & 1]);
-      if (j == nb - 1) mma_commit_warp(&sb->o_full);
-      return true;
-    };
-    for (int b = 0; b < nb && ok; ++b) {
-      if (b >= 3 && !issue_pv(b - 3)) { ok = false; break; }
-      const int s = b % 3;
-      if (!warp_wait(&sb->k_full[s], (b / 3) & 1, sb, p.err)) { ok = false; break; }
-      tc_fence_after();
-      const uint32_t tS = tmem + s * 128;
-      const uint32_t aKs = aK + s * C::kKVBytes;
-#pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        const uint32_t koff = (kk & 3) * 32;
-        const uint64_t adesc = smem_desc_sw128(aQ + (kk >> 2) * (C::M * 128) + koff, 16, 1024);
-        const uint64_t bdesc = smem_desc_sw128(aKs + (kk >> 2) * (BN * 128) + koff, 16, 1024);
-        mma_ss_warp(tS, adesc, bdesc, C::kIdescQK, kk > 0 ? 1u : 0u);
-      }
-      mma_commit_warp(&sb->s_full[s]);
-      mma_commit_warp(&sb->k_empty[s]);
-    }
-    for (int j = max(0, nb - 3); j < nb && ok; ++j)
-      if (!issue_pv(j)) ok = false;
-    mma_commit_warp(&sb->drain);
-    mbar_wait(&sb->drain, 0, kDrainNs);
+      for (int j = max(0, nb - 3); j < nb && ok; ++j)
+        if (!issue_pv(j)) ok = false;
+      mma_commit_warp(&sb->drain);
+      mbar_wait(&sb->drain, 0, kDrainNs);
+    }  // warps 10-11 idle
   } else {
     // ============================ softmax warps ============================
-    const int r = tid;                       // TMEM lane = sampled row
+    warpgroup_reg_inc<C::kRegSoftmax>();
+    const int wg = warp >> 2;                // 0: even blocks, 1: odd blocks
+    const int r = tid & 127;                 // TMEM lane = sampled row
     const int zl = r >> 4;
     const int j = r & 15;
     const int z = z0 + zl;
@@ -299,30 +321,40 @@ __global__ void __launch_bounds__(P1Cfg<D, BN>::kThreads, 1)
     const int hq = g * G + (valid ? z - i * G : 0);
     const int qpos = valid ? (i + t0) * BN + j * p.sample_stride : -1;  // key position; -1: padding row
     const int64_t srow = ((int64_t)hq * p.n_tiles + i) * p.n_sample + j;
-    const uint32_t lane_off = ((uint32_t)(warp * 32) << 16);
+    const uint32_t lane_off = ((uint32_t)((warp & 3) * 32) << 16);
     const uint32_t tO = tmem + lane_off + C::kColO;
     const float sl2 = p.scale_log2;
-    float m_run = -INFINITY, l_run = 0.f;
+    float m_run = -INFINITY;                 // reference max after this warpgroup's last block
+    float l_run = 0.f;                       // row sum through that block
     bool ok = true;
-    for (int b = 0; b < nb; ++b) {
+    for (int b = wg; b < nb; b += 2) {
       const int s = b % 3;
       const uint32_t tS = tmem + lane_off + s * 128;
+      // S_b ready (S_{b+3} needs P V_b, hence this warpgroup's P_b)
       if (!warp_wait(&sb->s_full[s], (b / 3) & 1, sb, p.err)) { ok = false; break; }
       tc_fence_after();
       const int lim = qpos - b * BN;  // columns <= lim are visible to this query
       uint32_t a[BN / 32][32];        // the row of S, read once
       load_row<BN>(tS, a);
       const float mx = (b < i_lo) ? row_max_regs<BN, false>(a, lim) : row_max_regs<BN, true>(a, lim);
-      const float m_new = fmaxf(m_run, mx * sl2);
-      const bool grow = (m_new > m_run + 8.0f);
-      float alpha = 1.f;
-      if (grow) {
-        alpha = (m_run == -INFINITY) ? 0.f : ex2_approx(m_run - m_new);
-        m_run = m_new;
+      // the reference through block b - 1 (the other warpgroup's)
+      float m_prev = -INFINITY;
+      if (b > 0) {
+        if (!warp_wait(&sb->ref_ready[(b - 1) & 1], ((b - 1) >> 1) & 1, sb, p.err)) { ok = false; break; }
+        m_prev = x_ref[((b - 1) & 1) * 128 + r];
       }
+      const float m_new = fmaxf(m_prev, mx * sl2);
+      const bool grow = (m_new > m_prev + 8.0f);
+      float alpha = 1.f, m_cur = m_prev;
+      if (grow) {
+        alpha = (m_prev == -INFINITY) ? 0.f : ex2_approx(m_prev - m_new);
+        m_cur = m_new;
+      }
+      x_ref[(b & 1) * 128 + r] = m_cur;
+      warp_arrive(&sb->ref_ready[b & 1]);
       if (b >= 1 && __any_sync(0xffffffffu, grow)) {
-        // O holds P V_0 .. P V_{b-1} once P V_{b-1} is complete; P V_b waits for this
-        // block's P, so O may then be rescaled in place.
+        // O holds P V_0 .. P V_{b-1} (against m_prev) once P V_{b-1} is complete; P V_b
+        // waits for this block's P, so O may then be rescaled in place.
         if (!warp_wait(&sb->acc_full[(b - 1) & 1], ((b - 1) >> 1) & 1, sb, p.err)) { ok = false; break; }
         tc_fence_after();
 #pragma unroll
@@ -336,22 +368,33 @@ __global__ void __launch_bounds__(P1Cfg<D, BN>::kThreads, 1)
           tmem_st32(tO + c * 32, ov);
         }
       }
-      l_run *= alpha;
       // reference of the weights: the running max, lowered by 6 for fp16 P so that
       // P <= 2^14 and weights down to 2^-20 of the reference keep full fp16 precision
-      const float m_use = (m_run == -INFINITY) ? 0.f : (half_p ? m_run - 6.0f : m_run);
+      const float m_use = (m_cur == -INFINITY) ? 0.f : (half_p ? m_cur - 6.0f : m_cur);
+      float bsum;
       if (half_p)
-        l_run += (b < i_lo) ? exp_f16_store_regs<BN, false>(tS, a, sl2, m_use, lim)
-                            : exp_f16_store_regs<BN, true>(tS, a, sl2, m_use, lim);
+        bsum = (b < i_lo) ? exp_f16_store_regs<BN, false>(tS, a, sl2, m_use, lim)
+                          : exp_f16_store_regs<BN, true>(tS, a, sl2, m_use, lim);
       else
-        l_run += (b < i_lo) ? exp_split_store_regs<BN, false>(tS, a, sl2, m_use, lim)
-                            : exp_split_store_regs<BN, true>(tS, a, sl2, m_use, lim);
+        bsum = (b < i_lo) ? exp_split_store_regs<BN, false>(tS, a, sl2, m_use, lim)
+                          : exp_split_store_regs<BN, true>(tS, a, sl2, m_use, lim);
       tmem_st_wait();
       tc_fence_before();
       warp_arrive(&sb->p_full[s]);
+      // the row sum through b - 1, then through b
+      float l_prev = 0.f;
+      if (b > 0) {
+        if (!warp_wait(&sb->l_ready[(b - 1) & 1], ((b - 1) >> 1) & 1, sb, p.err)) { ok = false; break; }
+        l_prev = x_l[((b - 1) & 1) * 128 + r];
+      }
+      l_run = l_prev * alpha + bsum;
+      m_run = m_cur;
+      x_l[(b & 1) * 128 + r] = l_run;
+      warp_arrive(&sb->l_ready[b & 1]);
     }
-    // ---- epilogue: o = O / l and lse = m + log2(l) (log2 units) ----
-    if (__all_sync(0xffffffffu, ok && !sb->abort_flag) && warp_wait(&sb->o_full, 0, sb, p.err)) {
+    // ---- epilogue (the warpgroup of the last block): o = O / l, lse = m + log2(l) ----
+    if (((nb - 1) & 1) == wg && __all_sync(0xffffffffu, ok && !sb->abort_flag) &&
+        warp_wait(&sb->o_full, 0, sb, p.err)) {
       tc_fence_after();
       const float inv_l = (l_run > 0.f) ? 1.f / l_run : 0.f;
       float* dst = p.ws_o + srow * D;
