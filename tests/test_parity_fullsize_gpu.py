@@ -46,7 +46,7 @@ def _sample_units(hq, T, extra):
     return sorted(units)
 
 
-def _survey_units(hq, T):
+def _strided_units(hq, T):
     """Every 16th tile of every 4th head, and the first and last three tiles of every head."""
     units = {(h, i) for h in range(0, hq, 4) for i in range(0, T, 16)}
     units |= {(h, i) for h in range(hq) for i in (0, 1, 2, T - 3, T - 2, T - 1) if 0 <= i < T}
@@ -105,7 +105,7 @@ def test_llama_layer_128k(poem):
     n, hq, hkv, d, B = 131072, 32, 8, 128, 128
     x = poem_synth.heavy_block_layer(n, hq, hkv, d, block=B, rope_base=500000.0, seed=0)
     T = n // B
-    units = _survey_units(hq, T)
+    units = _strided_units(hq, T)
     assert len(units) >= 128
     rp = _check_layer(poem, x, B, 0.05, units, full_units=[(h, T - 1) for h in range(hq)], row_sample=True)
     assert rp[-1] > 0
@@ -116,7 +116,7 @@ def test_qwen3_14b_layer_64k(poem):
     n, hq, hkv, d, B = 65536, 40, 8, 128, 128
     x = poem_synth.heavy_block_layer(n, hq, hkv, d, block=B, rope_base=1000000.0, seed=0)
     T = n // B
-    units = _survey_units(hq, T)
+    units = _strided_units(hq, T)
     assert len(units) >= 96
     _check_layer(poem, x, B, 0.05, units, full_units=[(h, T - 1) for h in range(hq)], row_sample=True)
 
