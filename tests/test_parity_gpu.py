@@ -332,6 +332,10 @@ SCORE_CASES = [
     # more than 32 tiles: the CTAs beyond tile 32 take both passes' fp16 P V contraction
     (6400, 5, 1, 128, 128, 1000000.0, 4),
     (4096, 2, 1, 64, 64, 10000.0, 5),
+    # 8-way GQA: a CTA holds one tile of 8 heads, so tile 0's CTA sweeps a single block
+    # (the second softmax warpgroup of each pass gets none) and the sweep lengths take
+    # both parities
+    (1536, 16, 2, 128, 128, 500000.0, 6),
 ]
 
 
