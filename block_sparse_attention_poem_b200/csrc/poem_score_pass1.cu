@@ -258,10 +258,13 @@ __global__ void __launch_bounds__(P1Cfg<D, BN>::kThreads, 1)
       const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV);
       const uint32_t tO = tmem + C::kColO;
       bool ok = warp_wait(&sb->q_full, 0, sb, p.err);
-      auto issue_pv = [&](int j) -> bool {
+      // `ready`: the step's barriers were all found complete by one joint test.
+      auto issue_pv = [&](int j, bool ready) -> bool {
         const int s = j % 3, sv = j & 1;
-        if (!warp_wait(&sb->p_full[s], (j / 3) & 1, sb, p.err)) return false;
-        if (!warp_wait(&sb->v_full[sv], (j >> 1) & 1, sb, p.err)) return false;
+        if (!ready) {
+          if (!warp_wait(&sb->p_full[s], (j / 3) & 1, sb, p.err)) return false;
+          if (!warp_wait(&sb->v_full[sv], (j >> 1) & 1, sb, p.err)) return false;
+        }
         tc_fence_after();
         const uint32_t tP = tmem + s * 128;
         const uint32_t aVs = aV + sv * C::kKVBytes;
@@ -287,9 +290,19 @@ __global__ void __launch_bounds__(P1Cfg<D, BN>::kThreads, 1)
         return true;
       };
       for (int b = 0; b < nb && ok; ++b) {
-        if (b >= 3 && !issue_pv(b - 3)) { ok = false; break; }
         const int s = b % 3;
-        if (!warp_wait(&sb->k_full[s], (b / 3) & 1, sb, p.err)) { ok = false; break; }
+        // Every barrier of this step (P V_{b-3}'s P and V, S_b's K) tested at once:
+        // normally all are complete, and one test latency replaces three successive
+        // waits.  Otherwise each is waited for in turn, bounded.
+        bool ready = mbar_test_wait(&sb->k_full[s], (b / 3) & 1);
+        if (b >= 3) {
+          const int j = b - 3;
+          ready = ready & mbar_test_wait(&sb->p_full[j % 3], (j / 3) & 1) &
+                  mbar_test_wait(&sb->v_full[j & 1], (j >> 1) & 1);
+        }
+        ready = __all_sync(0xffffffffu, ready);
+        if (b >= 3 && !issue_pv(b - 3, ready)) { ok = false; break; }
+        if (!ready && !warp_wait(&sb->k_full[s], (b / 3) & 1, sb, p.err)) { ok = false; break; }
         tc_fence_after();
         const uint32_t tS = tmem + s * 128;
         const uint32_t aKs = aK + s * C::kKVBytes;
@@ -304,7 +317,7 @@ __global__ void __launch_bounds__(P1Cfg<D, BN>::kThreads, 1)
         mma_commit_warp(&sb->k_empty[s]);
       }
       for (int j = max(0, nb - 3); j < nb && ok; ++j)
-        if (!issue_pv(j)) ok = false;
+        if (!issue_pv(j, false)) ok = false;
       mma_commit_warp(&sb->drain);
       mbar_wait(&sb->drain, 0, kDrainNs);
     }  // warps 10-11 idle

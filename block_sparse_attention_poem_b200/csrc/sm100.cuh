@@ -86,6 +86,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking test of an mbarrier phase (acquire semantics, as try_wait): several
+// tests can be in flight at once, where successive try_waits each pay their latency.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // One arrival for a whole converged warp: the lanes meet at __syncwarp (which also
 // orders their earlier memory writes before lane 0's release-arrive).  Barriers
 // signalled this way count warps, not threads; arriving once per warp instead of
