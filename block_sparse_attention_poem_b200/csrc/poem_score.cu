@@ -35,7 +35,7 @@
 //   o held in registers; warp 12 issues TMA loads (K and V rings independently);
 //   warp 13 issues the MMAs, converged, from one elected lane; warps 14-15 idle.
 //   Registers per thread: 128 at launch; the norm warpgroup raises its budget to
-//   200 and warps 12-15 lower theirs to 56 (128 + 200 + 128 + 56 = 4 x 128).
+//   184 and warps 12-15 lower theirs to 72 (128 + 184 + 128 + 72 = 4 x 128).
 //   MMA order: S_0, S_1, S_2, PV_0, S_3, PV_1, ...
 //
 // Precision: on a CTA's first query tiles (below score::kHalfMinTile) P enters the
@@ -79,8 +79,8 @@ struct ScoreCfg {
   static constexpr int kWarpProd = 12;     // warps 0-3, 8-11 softmax, 4-7 norm, 12 TMA, 13 MMA
   static constexpr int kWarpMma = 13;
   static constexpr int kThreads = 512;
-  static constexpr uint32_t kRegNorm = 200;  // per-thread registers after the reallocation
-  static constexpr uint32_t kRegProd = 56;
+  static constexpr uint32_t kRegNorm = 184;  // per-thread registers after the reallocation
+  static constexpr uint32_t kRegProd = 72;
   static_assert(128 + kRegNorm + 128 + kRegProd == 4 * 128, "register budget of the launch");
   static constexpr uint32_t kIdescQK = idesc_bf16_f32(M, BN, 0);
   static constexpr uint32_t kIdescPV = idesc_bf16_f32(M, D, 1);
@@ -251,10 +251,15 @@ __global__ void __launch_bounds__(ScoreCfg<D, BN>::kThreads, 1)
       const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV);
       const uint32_t tAcc = tmem + C::kColAcc;
       bool ok = warp_wait(&sb->q_full, 0, sb, p.err);
-      auto issue_pv = [&](int j) -> bool {
+      // `ready`: P_j, V_j (and this step's K) were all found complete by one joint
+      // test; the accumulator, which the norm warps release only shortly before it is
+      // needed, is always waited for on its own.
+      auto issue_pv = [&](int j, bool ready) -> bool {
         const int s = j % 3, sv = j & 1;
-        if (!warp_wait(&sb->p_full[s], (j / 3) & 1, sb, p.err)) return false;
-        if (!warp_wait(&sb->v_full[sv], (j >> 1) & 1, sb, p.err)) return false;
+        if (!ready) {
+          if (!warp_wait(&sb->p_full[s], (j / 3) & 1, sb, p.err)) return false;
+          if (!warp_wait(&sb->v_full[sv], (j >> 1) & 1, sb, p.err)) return false;
+        }
         if (j >= 1 && !warp_wait(&sb->acc_empty, (j - 1) & 1, sb, p.err)) return false;
         tc_fence_after();
         const uint32_t tP = tmem + C::kColS + s * 128;
@@ -280,9 +285,16 @@ __global__ void __launch_bounds__(ScoreCfg<D, BN>::kThreads, 1)
         return true;
       };
       for (int b = 0; b < nb && ok; ++b) {
-        if (b >= 3 && !issue_pv(b - 3)) { ok = false; break; }
         const int s = b % 3;
-        if (!warp_wait(&sb->k_full[s], (b / 3) & 1, sb, p.err)) { ok = false; break; }
+        bool ready = mbar_test_wait(&sb->k_full[s], (b / 3) & 1);
+        if (b >= 3) {
+          const int j = b - 3;
+          ready = ready & mbar_test_wait(&sb->p_full[j % 3], (j / 3) & 1) &
+                  mbar_test_wait(&sb->v_full[j & 1], (j >> 1) & 1);
+        }
+        ready = __all_sync(0xffffffffu, ready);
+        if (b >= 3 && !issue_pv(b - 3, ready)) { ok = false; break; }
+        if (!ready && !warp_wait(&sb->k_full[s], (b / 3) & 1, sb, p.err)) { ok = false; break; }
         tc_fence_after();
         const uint32_t tS = tmem + C::kColS + s * 128;
         const uint32_t aKs = aK + s * C::kKVBytes;
@@ -297,7 +309,7 @@ __global__ void __launch_bounds__(ScoreCfg<D, BN>::kThreads, 1)
         mma_commit_warp(&sb->k_empty[s]);
       }
       for (int j = max(0, nb - 3); j < nb && ok; ++j)
-        if (!issue_pv(j)) ok = false;
+        if (!issue_pv(j, false)) ok = false;
       mma_commit_warp(&sb->drain);
       mbar_wait(&sb->drain, 0, kDrainNs);
     }  // warps 14-15 idle
